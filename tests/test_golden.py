@@ -1,0 +1,34 @@
+"""Regression: the oracle still gives the stored result on the seeded tiny
+workload (tests/golden/tiny_oracle.json, written by make_golden.py)."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from compressed_kv_cache_routing_b200 import workloads as W
+from oracle import oracle
+from helpers import to_problem
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "tiny_oracle.json")
+
+
+def test_tiny_golden():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "make_golden", os.path.join(os.path.dirname(GOLDEN), "make_golden.py"))
+    mg = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mg)
+    with open(GOLDEN) as f:
+        doc = json.load(f)
+    w = W.generate("tiny")
+    prob = to_problem(w)
+    if mg.input_digest(prob) != doc["input_sha256"]:
+        pytest.fail("the tiny workload's inputs changed; regenerate the fixture only "
+                    "if the generator change is intended")
+    out, sel, scores, gap = oracle.decode(prob, want_scores=True)
+    assert sel[0, 0].tolist() == doc["sel"]
+    assert gap[0, 0] == doc["gap"]
+    n = len(doc["page_scores"])
+    assert np.array_equal(scores[0, 0, :n], np.array(doc["page_scores"]))
+    assert np.array_equal(out[0], np.array(doc["out"]))
