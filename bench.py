@@ -1,0 +1,394 @@
+"""Benchmark: BasisKV routed decode attention over a compressed paged KV cache.
+
+One step = one ``basiskv_decode_attn`` call (routing scores + top-k, exact QK
+on the selected pages, softmax, latent sum, combine and B_v) for every
+(sequence, KV head) of the workload, inputs resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the float64 CPU oracle arm
+
+Prints one JSON line (rank 0).  Multi-GPU: one process per GPU under
+torchrun; every rank runs its own replica of the workload (no collective on
+the data path: the units are independent), weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "compressed-KV decode attn context-tokens/s; HBM GB/s vs ~8 TB/s peak (1 B200)"
+UNIT = "context-tokens/s"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama3_8b_decode")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world, backend):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Largest value of x over all ranks (the slowest rank sets the time)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed loop runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, fl in rows for i, v in enumerate(fl) if v == "Active"})
+        return {"sm_mhz": float(np.median([r[0] for r in rows])), "sm_max_mhz": rows[0][1],
+                "reasons": reasons, "samples": len(rows)}
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch recorded by an ncu capture of this kernel, if the
+    capture matches the current kernel source (profiles/traffic.json)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        e = rec.get(f"{kernel}:{workload}")
+        if not e:
+            return None
+        import hashlib
+        h = hashlib.sha256()
+        for fn in sorted(e["sources"]):
+            with open(os.path.join(ROOT, fn), "rb") as f:
+                h.update(f.read())
+        return float(e["dram_bytes_per_launch"]) if h.hexdigest() == e["sources_sha256"] else None
+    except Exception:
+        return None
+
+
+def oracle_problem(w):
+    """Host copies of a workload's stored tensors for the oracle."""
+    import torch
+    from oracle import oracle
+    s = w.spec
+    bf16 = s.dtype == "bf16"
+
+    def host(t):
+        t = t.detach().cpu().contiguous()
+        return t.view(torch.int16).numpy() if bf16 else t.numpy()
+
+    return oracle.Problem(
+        q=host(w.q), z_pool=host(w.z_pool), r_pool=host(w.r_pool), k_pool=host(w.k_pool),
+        w_zk=w.w_zk.cpu().numpy(), b_r=w.b_r.cpu().numpy(), b_v=w.b_v.cpu().numpy(),
+        page_table=np.where(w.page_table >= 0, w.page_table, 0).astype(np.int32),
+        seq_lens=w.seq_lens, gqa_group=s.gqa_group, topk=s.topk, softmax_scale=s.softmax_scale,
+        dtype=oracle.BF16 if bf16 else oracle.F32)
+
+
+def cpu_oracle_timing(prob, w, budget_s: float):
+    """Time the oracle on a bounded sample of units: grow the sample until it
+    costs about budget_s of wall time.  Returns (tokens/s, cores, sample text)."""
+    from oracle import oracle
+    s = w.spec
+    U = s.batch * s.num_kv_heads
+    cores = oracle.max_threads()
+    order = np.random.default_rng(0).permutation(U)
+    done, spent, tokens = 0, 0.0, 0.0
+    n = max(1, min(U, cores))
+    while done < U and spent < budget_s:
+        units = order[done:done + n].tolist()
+        t0 = time.perf_counter()
+        oracle.decode(prob, units=units)
+        spent += time.perf_counter() - t0
+        tokens += sum(float(w.seq_lens[u // s.num_kv_heads]) / s.num_kv_heads for u in units)
+        done += len(units)
+        n = min(U - done, n * 2)
+    sample = (f"{done} of {U} (sequence, KV head) units of {s.name}, {cores} OpenMP threads, "
+              f"{spent:.1f} s; tokens counted as L_b/Hkv per unit")
+    return tokens / spent, cores, sample
+
+
+def run_reference(args, rank, world):
+    """The oracle arm: the float64 CPU oracle on this workload, each step a
+    bounded sample (one unit, its sequence cut to fit the time budget)."""
+    if rank != 0:
+        return 0
+    import torch
+    from compressed_kv_cache_routing_b200 import workloads as W
+    from oracle import oracle
+    spec = W.SPECS[args.workload]
+    w = W.generate(spec, device="cuda" if torch.cuda.is_available() else "cpu")
+    prob = oracle_problem(w)
+    cores = oracle.max_threads()
+    # per-step sample: unit 0 on every thread, sequence cut so the whole run
+    # stays near two minutes
+    total_steps = args.steps + args.warmup
+    L0 = int(w.seq_lens[0])
+    per_step_budget = 120.0 / max(1, total_steps)
+    units = list(range(min(cores, spec.num_kv_heads)))
+    probe = oracle.Problem(**{**prob.__dict__, "seq_lens": np.array([min(L0, spec.page_size * 8)] +
+                                                                   [0] * (spec.batch - 1), np.int32)})
+    t0 = time.perf_counter()
+    oracle.decode(probe, units=units)
+    t_probe = max(time.perf_counter() - t0, 1e-4)
+    L = int(min(L0, max(spec.page_size, spec.page_size * 8 * per_step_budget / t_probe)))
+    lens = np.zeros(spec.batch, np.int32)
+    lens[0] = L
+    step_prob = oracle.Problem(**{**prob.__dict__, "seq_lens": lens})
+    for _ in range(args.warmup):
+        oracle.decode(step_prob, units=units)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.decode(step_prob, units=units)
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * float(np.mean(times))
+    tokens = L * len(units) / spec.num_kv_heads
+    value = tokens / (ms * 1e-3)
+    sample = (f"sequence 0 cut to {L} tokens, KV heads {units}, {cores} OpenMP threads per step "
+              f"(tokens counted as L/Hkv per (sequence, KV head))")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload}, "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, rank, world, local):
+    import torch
+    from compressed_kv_cache_routing_b200 import basiskv as bk
+    from compressed_kv_cache_routing_b200 import build
+    from compressed_kv_cache_routing_b200 import workloads as W
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    build.build()
+    spec = W.SPECS[args.workload]
+    if rank:
+        spec = spec.with_(seed=spec.seed + 1000 * rank)
+    w = W.generate(spec, device=dev)
+    kv = bk.BasisKV.for_workload(w)
+    s = w.spec
+    out = torch.empty((s.batch, s.num_q_heads, s.head_dim), device=dev, dtype=torch.float32)
+    sel = torch.empty((s.batch, s.num_kv_heads, s.topk), device=dev, dtype=torch.int32)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2 // 4 + 1, device=dev, dtype=torch.float32)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        bk.basiskv_decode_attn(kv.handle, w.q, s.topk, s.softmax_scale, out, sel, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if bk.basiskv_get_status(kv.handle, clear=True):
+        raise SystemExit("device status error during warm-up")
+
+    K = args.steps
+    with ClockSampler(local) as clk:
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        bk.basiskv_profile_begin(kv.handle, K)
+        wall0 = time.perf_counter()
+        for _ in range(K):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize(dev)
+        wall = time.perf_counter() - wall0
+        barrier(world, dev)
+        route_ms, attn_ms, total_ms = bk.basiskv_profile_end(kv.handle, K)
+    clocks = clk.summary()
+    status = bk.basiskv_get_status(kv.handle, clear=True)
+    launch = bk.basiskv_last_launch(kv.handle)
+
+    ms_step = float(np.mean(total_ms))
+    ms_step_max = max_over_ranks(ms_step, world, dev)
+    tokens = w.context_tokens
+    value = tokens * world / (ms_step_max * 1e-3)
+    nbytes = w.algorithmic_bytes()
+    hbm_peak, peak_kind = peaks()
+    route_mean = float(np.mean(route_ms)) if launch["route_ctas"] else 0.0
+    attn_mean = float(np.mean(attn_ms))
+    if route_mean > 0 and nbytes["route"] >= nbytes["attn"]:
+        dom, dom_bytes, dom_ms = "route", nbytes["route"], route_mean
+        kname = "route_mma_kernel" if launch["route_tensor_core"] else "route_generic_kernel"
+    else:
+        dom, dom_bytes, dom_ms = "attn", nbytes["attn"], attn_mean
+        kname = "attn_mma_kernel" if launch["attn_tensor_core"] else "attn_generic_kernel"
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    traffic = ncu_traffic(kname, args.workload)
+
+    # end to end through the host-buffer entry point: q in, out (+ selection) back
+    q_host = w.q.cpu().pin_memory()
+    out_host = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    sel_host = torch.empty(sel.shape, dtype=torch.int32).pin_memory()
+    for _ in range(3):
+        bk.basiskv_decode_attn_host(kv.handle, q_host, s.topk, s.softmax_scale, out_host, sel_host,
+                                    stream=stream)
+    e2e_steps = max(5, min(K, 50))
+    e2e_times = []
+    for _ in range(e2e_steps):
+        flush.zero_()
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        bk.basiskv_decode_attn_host(kv.handle, q_host, s.topk, s.softmax_scale, out_host, sel_host,
+                                    stream=stream)
+        e2e_times.append(time.perf_counter() - t0)
+    e2e_s = max_over_ranks(float(np.mean(e2e_times)), world, dev)
+    h2d = q_host.numel() * q_host.element_size()
+    d2h = out_host.numel() * 4 + sel_host.numel() * 4
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        prob = oracle_problem(w)
+        v, cores, sample = cpu_oracle_timing(prob, w, args.cpu_budget_s)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_step_max, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": s.dtype, "data": "synthetic",
+            "config": {"workload": args.workload, "batch": s.batch, "kv_heads": s.num_kv_heads,
+                       "q_heads": s.num_q_heads, "head_dim": s.head_dim, "page": s.page_size,
+                       "rank_r": s.rank_r, "rank_s": s.rank_s, "topk": s.topk,
+                       "context_tokens": tokens, "algorithmic_bytes": nbytes["total"],
+                       "l2": "flushed between steps (2x L2 write, outside the per-step events)",
+                       "timing": "per-step CUDA events on the launching stream, mean of K",
+                       "parallelism": f"replicas x{world}, no data-path collective"},
+            "hbm": {"achieved_gbs": nbytes["total"] / (ms_step_max * 1e-3) / 1e9, "peak_gbs": hbm_peak,
+                    "frac": nbytes["total"] / (ms_step_max * 1e-3) / 1e9 / hbm_peak,
+                    "frac_of_8tbs": nbytes["total"] / (ms_step_max * 1e-3) / 8e12, "peak_kind": peak_kind},
+            "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": hbm_peak,
+                         "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": traffic,
+                         "algorithmic_bytes_per_launch": dom_bytes, "launch_ms": dom_ms,
+                         "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"},
+            "kernels_ms": {"route": route_mean, "attn": attn_mean,
+                           "route_p10_p90": [float(np.percentile(route_ms, 10)), float(np.percentile(route_ms, 90))] if route_mean else None,
+                           "step_p10_p90": [float(np.percentile(total_ms, 10)), float(np.percentile(total_ms, 90))]},
+            "launch": launch,
+            "gpu_launches": K * ((1 if launch["route_ctas"] else 0) + 1),
+            "e2e": {"value": tokens * world / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_s * 1e3,
+                    "how": "basiskv_decode_attn_host: pinned q H2D, decode, out+sel D2H, stream sync; host wall clock"},
+            "wall_ms_per_step_incl_flush": wall * 1e3 / K,
+            "clocks": clocks,
+            "device_status": status,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    kv.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,367 @@
+// Exact attention over the selected pages for BasisKV decode ("the original
+// Keys are then retrieved only for the selected pages to compute exact QK
+// scores"); values stay rank-r latents Z, and the weighted latent is
+// expanded by B_v in the fused combine.
+//
+// Grid: (splits, Hkv, batch).  Split sp of a (sequence, KV head) handles
+// selected entries [sp*pps, min((sp+1)*pps, k_b)).  Each warp keeps an
+// online-softmax state (running max m in log2 units, sum l, latent
+// accumulator acc[r]) for the G query heads and writes it as one partial;
+// the last CTA of the unit merges all partials and applies B_v.
+#pragma once
+
+#include "combine.cuh"
+#include "common.cuh"
+
+namespace basiskv {
+
+struct AttnArgs {
+  const void* q;             // [B][Hkv*G][d]
+  const void* k_pool;        // [slots][Hkv][P][d]
+  const void* z_pool;        // [slots][Hkv][P][r]
+  const float* b_v;          // [Hkv][r][d]
+  const int32_t* page_table; // [B][ld_pt]
+  const int32_t* seq_lens;   // [B]
+  const int32_t* sel;        // [B][Hkv][ld_sel] (routed units)
+  int32_t* sel_out;          // [B][Hkv][topk] or null
+  float* part_ml;            // [B*Hkv][np_cap][G][2]
+  float* part_acc;           // [B*Hkv][np_cap][G][r]
+  uint32_t* counters;        // [B*Hkv]
+  uint32_t* status;
+  float* out;                // [B][Hkv*G][d]
+  int ld_pt, ld_sel, num_slots, num_kv_heads, head_dim, page_size, rank_r, gqa_group;
+  int topk, pages_per_split, stages, np_cap;
+  float scale_log2;          // softmax_scale * log2(e)
+};
+
+constexpr int kAttnThreads = 128;
+constexpr int kAttnWarps = kAttnThreads / 32;
+
+struct AttnUnit {
+  int b, kvh, u, L, n, kb, j0, j1;
+  bool routed;
+};
+
+__device__ __forceinline__ AttnUnit attn_unit(const AttnArgs& a) {
+  AttnUnit au;
+  au.b = blockIdx.z;
+  au.kvh = blockIdx.y;
+  au.u = au.b * a.num_kv_heads + au.kvh;
+  au.L = a.seq_lens[au.b];
+  au.n = (au.L + a.page_size - 1) / a.page_size;
+  au.routed = a.topk < au.n;
+  au.kb = au.routed ? a.topk : au.n;
+  au.j0 = blockIdx.x * a.pages_per_split;
+  au.j1 = min(au.kb, au.j0 + a.pages_per_split);
+  return au;
+}
+
+// Logical page of selected entry jj, checked against [0, n).
+__device__ __forceinline__ int selected_page(const AttnArgs& a, const AttnUnit& au, int jj) {
+  if (!au.routed) return jj;
+  int p = __ldcg(a.sel + (size_t)au.u * a.ld_sel + jj);
+  if (p < 0 || p >= au.n) {
+    atomicOr(a.status, kStatusBadPage);
+    p = 0;
+  }
+  return p;
+}
+
+__device__ __forceinline__ int page_slot(const AttnArgs& a, const AttnUnit& au, int page) {
+  int slot = a.page_table[(size_t)au.b * a.ld_pt + page];
+  if (slot < 0 || slot >= a.num_slots) {
+    atomicOr(a.status, kStatusBadSlot);
+    slot = 0;
+  }
+  return slot;
+}
+
+// Units whose every page is used were not routed: list their pages.
+__device__ __forceinline__ void write_identity_selection(const AttnArgs& a, const AttnUnit& au) {
+  if (au.routed || blockIdx.x != 0 || a.sel_out == nullptr) return;
+  int32_t* so = a.sel_out + (size_t)au.u * a.topk;
+  for (int i = threadIdx.x; i < a.topk; i += blockDim.x) so[i] = i < au.n ? i : -1;
+}
+
+template <int NT>
+__device__ __forceinline__ void attn_finish(const AttnArgs& a, const AttnUnit& au, int parts_per_cta,
+                                            float* smem_f, int* flag) {
+  if (!arrive_last(a.counters + au.u, gridDim.x, flag)) return;
+  const int G = a.gqa_group;
+  CombineArgs c;
+  c.part_ml = a.part_ml + (size_t)au.u * a.np_cap * G * 2;
+  c.part_acc = a.part_acc + (size_t)au.u * a.np_cap * G * a.rank_r;
+  c.b_v = a.b_v + (size_t)au.kvh * a.rank_r * a.head_dim;
+  c.out = a.out + (size_t)au.u * G * a.head_dim;
+  c.np = gridDim.x * parts_per_cta;
+  c.g = G;
+  c.r = a.rank_r;
+  c.d = a.head_dim;
+  combine_unit<NT>(c, smem_f);
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core attention for bf16 pools.
+//
+// QK: S(16 x 8 tokens) = Qg(16 x d) . K^T, rows 0..G-1 of Qg hold the group's
+// queries (rows G..15 zero), K rows come from shared memory; the k index is
+// permuted exactly as in the routing kernel so each thread's B fragment is a
+// 16-byte load.  The S fragment (row g = head, columns 2t, 2t+1 = tokens) is
+// already the A fragment layout of the next product, so the probabilities
+// never leave registers.
+// PV: acc(16 x r) += Pg(16 x 16 tokens) . Z(16 tokens x r); row g of Pg holds
+// bf16 hi(p) of head g and row g+8 holds lo(p) = bf16(p - hi(p)), so
+// acc[g] + acc[g+8] is the latent sum with ~16-bit weights; Z fragments come
+// from ldmatrix.trans.
+// Each stage carries TPS tokens of one selected page (K then Z), staged by
+// bulk copies into a per-warp ring.
+template <int G, int D, int RR, int TPS>
+__global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const AttnArgs a) {
+  static_assert(G >= 1 && G <= 8, "GQA group must be 1..8");
+  static_assert(D % 32 == 0 && RR % 8 == 0 && TPS % 16 == 0, "shape");
+  constexpr int DS = D / 32;     // 32-wide spans of the head dim
+  constexpr int RT = RR / 8;     // n8 tiles of the latent
+  constexpr int NTS = TPS / 8;   // n8 token tiles per stage
+  constexpr int KBS = TPS / 16;  // k16 token blocks per stage
+  constexpr uint32_t kbytes = TPS * D * 2, zbytes = TPS * RR * 2;
+  constexpr uint32_t stage_bytes = kbytes + zbytes;
+
+  const AttnUnit au = attn_unit(a);
+  const int P = a.page_size, S = a.stages;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int sub = P / TPS;
+  const int items = max(0, au.j1 - au.j0) * sub;
+  const int mine = items > warp ? (items - warp + kAttnWarps - 1) / kAttnWarps : 0;
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ uint64_t bars[kAttnWarps][8];
+  __shared__ int flag;
+  uint8_t* ring = smem + (size_t)warp * S * stage_bytes;
+
+  // query fragments (A operand), rows >= G are zero
+  uint32_t qa[DS][2][2];
+  {
+    const __nv_bfloat16* qrow =
+        static_cast<const __nv_bfloat16*>(a.q) + ((size_t)au.u * G + (g < G ? g : 0)) * D;
+#pragma unroll
+    for (int s = 0; s < DS; ++s) {
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (g < G) v = __ldg(reinterpret_cast<const uint4*>(qrow + 32 * s + 8 * t));
+      qa[s][0][0] = v.x;
+      qa[s][0][1] = v.y;
+      qa[s][1][0] = v.z;
+      qa[s][1][1] = v.w;
+    }
+  }
+  if (lane == 0) {
+    for (int i = 0; i < S; ++i) mbar_init(&bars[warp][i], 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
+  pdl_wait_primary();  // the selection is written by the routing grid
+
+  const __nv_bfloat16* kpool = static_cast<const __nv_bfloat16*>(a.k_pool);
+  const __nv_bfloat16* zpool = static_cast<const __nv_bfloat16*>(a.z_pool);
+  const uint64_t pol = policy_evict_first();
+  auto issue = [&](int i) {  // lane 0: my i-th item into stage i % S
+    const int item = warp + i * kAttnWarps;
+    const int page = selected_page(a, au, au.j0 + item / sub);
+    const int slot = page_slot(a, au, page);
+    const size_t row0 = ((size_t)slot * a.num_kv_heads + au.kvh) * P + (size_t)(item % sub) * TPS;
+    uint64_t* bar = &bars[warp][i % S];
+    uint8_t* dst = ring + (size_t)(i % S) * stage_bytes;
+    mbar_arrive_expect_tx(bar, stage_bytes);
+    bulk_load(dst, kpool + row0 * D, kbytes, bar, pol);
+    bulk_load(dst + kbytes, zpool + row0 * RR, zbytes, bar, pol);
+  };
+  if (lane == 0)
+    for (int i = 0; i < S && i < mine; ++i) issue(i);
+
+  float m_run = -INFINITY, l_run = 0.f;
+  float acc[RT][4];
+#pragma unroll
+  for (int c = 0; c < RT; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.f;
+
+  bool ok = true;
+  int i = 0;
+  for (; i < mine; ++i) {
+    ok = mbar_wait(&bars[warp][i % S], (uint32_t)((i / S) & 1), a.status);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) break;
+    const int item = warp + i * kAttnWarps;
+    const int page = selected_page(a, au, au.j0 + item / sub);
+    const int valid = au.L - (page * P + (item % sub) * TPS);  // tokens of this stage in range
+    const __nv_bfloat16* ks = reinterpret_cast<const __nv_bfloat16*>(ring + (size_t)(i % S) * stage_bytes);
+    const __nv_bfloat16* zs = ks + TPS * D;
+
+    // exact QK for the group
+    float s[NTS][2];
+#pragma unroll
+    for (int nt = 0; nt < NTS; ++nt) {
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      const __nv_bfloat16* krow = ks + (nt * 8 + g) * D;
+#pragma unroll
+      for (int sp = 0; sp < DS; ++sp) {
+        const uint4 v = lds128(krow + 32 * sp + 8 * t);
+        mma_k16(d, qa[sp][0][0], 0u, qa[sp][0][1], 0u, v.x, v.y);
+        mma_k16(d, qa[sp][1][0], 0u, qa[sp][1][1], 0u, v.z, v.w);
+      }
+      const int tok = nt * 8 + 2 * t;
+      s[nt][0] = tok < valid ? d[0] * a.scale_log2 : -INFINITY;
+      s[nt][1] = tok + 1 < valid ? d[1] * a.scale_log2 : -INFINITY;
+    }
+    // online softmax for head g (the quad 4g..4g+3 shares the row)
+    float mloc = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < NTS; ++nt) mloc = fmaxf(mloc, fmaxf(s[nt][0], s[nt][1]));
+    mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
+    mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
+    const float m_new = fmaxf(m_run, mloc);
+    const float corr = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
+    const float base = (m_new == -INFINITY) ? 0.f : m_new;
+    float lsum = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < NTS; ++nt) {
+      s[nt][0] = exp2f(s[nt][0] - base);
+      s[nt][1] = exp2f(s[nt][1] - base);
+      lsum += s[nt][0] + s[nt][1];
+    }
+    l_run = l_run * corr + lsum;
+    m_run = m_new;
+#pragma unroll
+    for (int c = 0; c < RT; ++c) {
+      acc[c][0] *= corr;
+      acc[c][1] *= corr;
+      acc[c][2] *= corr;
+      acc[c][3] *= corr;
+    }
+    // latent sum P.Z
+    const int trow = (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+    for (int kb = 0; kb < KBS; ++kb) {
+      float h0, l0, h1, l1, h2, l2, h3, l3;
+      split_bf16(s[2 * kb][0], h0, l0);
+      split_bf16(s[2 * kb][1], h1, l1);
+      split_bf16(s[2 * kb + 1][0], h2, l2);
+      split_bf16(s[2 * kb + 1][1], h3, l3);
+      const uint32_t a0 = pack_bf16(h0, h1), a1 = pack_bf16(l0, l1);
+      const uint32_t a2 = pack_bf16(h2, h3), a3 = pack_bf16(l2, l3);
+      const __nv_bfloat16* zrow = zs + (kb * 16 + trow) * RR + 8 * (lane >> 4);
+#pragma unroll
+      for (int c2 = 0; c2 < RT / 2; ++c2) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_trans(b0, b1, b2, b3, zrow + 16 * c2);
+        mma_k16(acc[2 * c2], a0, a1, a2, a3, b0, b1);
+        mma_k16(acc[2 * c2 + 1], a0, a1, a2, a3, b2, b3);
+      }
+      if (RT & 1) {
+        uint32_t b0, b1;
+        ldsm_x2_trans(b0, b1, zs + (kb * 16 + trow) * RR + 8 * (RT - 1));
+        mma_k16(acc[RT - 1], a0, a1, a2, a3, b0, b1);
+      }
+    }
+    __syncwarp();
+    if (lane == 0 && i + S < mine) issue(i + S);
+  }
+  if (!ok && lane == 0)
+    for (int j = i; j < mine && j < i + S; ++j)
+      mbar_wait(&bars[warp][j % S], (uint32_t)((j / S) & 1), a.status);
+
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  if (g < G) {
+    const size_t part = ((size_t)au.u * a.np_cap + blockIdx.x * kAttnWarps + warp) * G + g;
+    if (t == 0) {
+      a.part_ml[part * 2] = m_run;
+      a.part_ml[part * 2 + 1] = l_run;
+    }
+    float* pa = a.part_acc + part * RR;
+#pragma unroll
+    for (int c = 0; c < RT; ++c) {
+      pa[8 * c + 2 * t] = acc[c][0] + acc[c][2];
+      pa[8 * c + 2 * t + 1] = acc[c][1] + acc[c][3];
+    }
+  }
+  write_identity_selection(a, au);
+  attn_finish<kAttnThreads>(a, au, kAttnWarps, reinterpret_cast<float*>(smem), &flag);
+}
+
+// ---------------------------------------------------------------------------
+// CUDA-core attention for any shape and for fp32 pools: one partial per CTA.
+template <typename T>
+__global__ void __launch_bounds__(kAttnThreads) attn_generic_kernel(const AttnArgs a) {
+  const AttnUnit au = attn_unit(a);
+  const int G = a.gqa_group, D = a.head_dim, RR = a.rank_r, P = a.page_size;
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ int flag;
+  float* qs = reinterpret_cast<float*>(smem);  // [G][D]
+  float* sc = qs + G * D;                      // [G][P]
+  float* accs = sc + G * P;                    // [G][RR]
+  float* corr = accs + G * RR;                 // [G]
+  float* mrun = corr + G;                      // [G]
+  float* lrun = mrun + G;                      // [G]
+  const T* q = static_cast<const T*>(a.q) + (size_t)au.u * G * D;
+  for (int i = threadIdx.x; i < G * D; i += blockDim.x) qs[i] = to_f32(q[i]);
+  for (int i = threadIdx.x; i < G * RR; i += blockDim.x) accs[i] = 0.f;
+  for (int i = threadIdx.x; i < G; i += blockDim.x) {
+    mrun[i] = -INFINITY;
+    lrun[i] = 0.f;
+  }
+  pdl_wait_primary();
+  __syncthreads();
+  const T* kpool = static_cast<const T*>(a.k_pool);
+  const T* zpool = static_cast<const T*>(a.z_pool);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int jj = au.j0; jj < au.j1; ++jj) {
+    const int page = selected_page(a, au, jj);
+    const int slot = page_slot(a, au, page);
+    const size_t row0 = ((size_t)slot * a.num_kv_heads + au.kvh) * P;
+    const int valid = min(P, au.L - page * P);
+    for (int idx = threadIdx.x; idx < valid * G; idx += blockDim.x) {
+      const int tok = idx / G, h = idx % G;
+      const T* kr = kpool + (row0 + tok) * D;
+      float dot = 0.f;
+      for (int c = 0; c < D; ++c) dot = fmaf(qs[h * D + c], to_f32(kr[c]), dot);
+      sc[h * P + tok] = dot * a.scale_log2;
+    }
+    __syncthreads();
+    for (int h = warp; h < G; h += kAttnWarps) {
+      float m = -INFINITY;
+      for (int tk = lane; tk < valid; tk += 32) m = fmaxf(m, sc[h * P + tk]);
+      m = warp_max(m);
+      const float m_new = fmaxf(mrun[h], m);
+      float sum = 0.f;
+      for (int tk = lane; tk < valid; tk += 32) {
+        const float p = exp2f(sc[h * P + tk] - m_new);
+        sc[h * P + tk] = p;
+        sum += p;
+      }
+      sum = warp_sum(sum);
+      if (lane == 0) {
+        const float cr = exp2f(mrun[h] - m_new);
+        corr[h] = cr;
+        lrun[h] = lrun[h] * cr + sum;
+        mrun[h] = m_new;
+      }
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < G * RR; idx += blockDim.x) {
+      const int h = idx / RR, i = idx % RR;
+      float acc = accs[idx] * corr[h];
+      for (int tk = 0; tk < valid; ++tk) acc = fmaf(sc[h * P + tk], to_f32(zpool[(row0 + tk) * RR + i]), acc);
+      accs[idx] = acc;
+    }
+    __syncthreads();
+  }
+  const size_t part0 = ((size_t)au.u * a.np_cap + blockIdx.x) * G;
+  for (int h = threadIdx.x; h < G; h += blockDim.x) {
+    a.part_ml[(part0 + h) * 2] = mrun[h];
+    a.part_ml[(part0 + h) * 2 + 1] = lrun[h];
+  }
+  for (int idx = threadIdx.x; idx < G * RR; idx += blockDim.x) a.part_acc[part0 * RR + idx] = accs[idx];
+  write_identity_selection(a, au);
+  attn_finish<kAttnThreads>(a, au, 1, reinterpret_cast<float*>(smem), &flag);
+}
+
+}  // namespace basiskv

@@ -1,0 +1,669 @@
+// Host side of the BasisKV decode-attention library: argument validation,
+// library-owned state, launch shapes and the C ABI declared in basiskv.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "../../include/basiskv.h"
+#include "attn.cuh"
+#include "route.cuh"
+
+using namespace basiskv;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+#define CUDA_TRY(call)                                                                      \
+  do {                                                                                      \
+    cudaError_t e_ = (call);                                                                \
+    if (e_ != cudaSuccess) return fail(BASISKV_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+constexpr int kMaxSplits = 16;
+constexpr int kPartsCap = kMaxSplits * kAttnWarps;  // partials per unit
+constexpr size_t kRouteSmemBudget = 96 * 1024;       // ring bytes per routing CTA
+constexpr size_t kAttnSmemBudget = 200 * 1024;       // ring bytes per attention CTA
+
+using KernelFn = void (*)(const RouteArgs);
+using AttnFn = void (*)(const AttnArgs);
+
+// ---- compiled tensor-core shapes ------------------------------------------
+struct RouteKey {
+  int g, r, s;
+  bool operator<(const RouteKey& o) const { return std::tie(g, r, s) < std::tie(o.g, o.r, o.s); }
+};
+struct AttnKey {
+  int g, d, r, tps;
+  bool operator<(const AttnKey& o) const {
+    return std::tie(g, d, r, tps) < std::tie(o.g, o.d, o.r, o.tps);
+  }
+};
+
+const std::map<RouteKey, KernelFn>& route_table() {
+  static const std::map<RouteKey, KernelFn> t = {
+#define RK(G, R, S) {RouteKey{G, R, S}, &route_mma_kernel<G, R, S>}
+      RK(4, 16, 8),  RK(4, 24, 8),  RK(4, 32, 8),  RK(4, 32, 16), RK(4, 64, 16),
+      RK(4, 64, 32), RK(4, 128, 0), RK(4, 32, 0),  RK(8, 32, 16), RK(8, 24, 8),
+      RK(8, 64, 32), RK(2, 32, 16), RK(1, 32, 16),
+#undef RK
+  };
+  return t;
+}
+
+const std::map<AttnKey, AttnFn>& attn_table() {
+  static const std::map<AttnKey, AttnFn> t = {
+#define AK(G, D, R, T) {AttnKey{G, D, R, T}, &attn_mma_kernel<G, D, R, T>}
+      AK(4, 128, 32, 64), AK(4, 128, 32, 32), AK(4, 128, 24, 32), AK(4, 128, 24, 16),
+      AK(4, 128, 16, 64), AK(4, 128, 64, 32), AK(4, 128, 128, 32), AK(4, 128, 128, 16),
+      AK(4, 64, 16, 16),  AK(4, 64, 32, 32),  AK(8, 128, 32, 64), AK(8, 128, 32, 32),
+      AK(8, 128, 24, 32), AK(8, 128, 64, 32), AK(2, 128, 32, 64), AK(1, 128, 32, 64),
+#undef AK
+  };
+  return t;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+struct basiskv_handle {
+  basiskv_params p;
+  int device = 0;
+  int num_sms = 148;
+  size_t elem = 2;
+  // device state
+  int32_t* d_page_table = nullptr;  // [max_batch][max_pages]
+  int32_t* d_seq_lens = nullptr;    // [max_batch]
+  float* d_scores = nullptr;        // [max_batch][Hkv][max_pages]
+  int32_t* d_sel = nullptr;         // [max_batch][Hkv][max_topk]
+  float* d_part_ml = nullptr;       // [max_batch*Hkv][kPartsCap][G][2]
+  float* d_part_acc = nullptr;      // [max_batch*Hkv][kPartsCap][G][r]
+  uint32_t* d_counters = nullptr;   // [2][max_batch*Hkv]
+  uint32_t* d_status = nullptr;
+  // host-buffer entry point staging
+  void* d_q_stage = nullptr;
+  float* d_out_stage = nullptr;
+  int32_t* d_sel_stage = nullptr;
+  // host mirror (launch sizing, validation)
+  std::vector<int32_t> h_table;
+  std::vector<int32_t> h_lens;
+  std::vector<int32_t> h_npages;
+  // kernels chosen at create
+  KernelFn route_fn = nullptr;
+  AttnFn attn_fn = nullptr;
+  int attn_tps = 0;
+  int route_stages = 0, attn_stages = 0;
+  size_t route_smem = 0, attn_smem = 0;
+  // profiling
+  std::vector<cudaEvent_t> events;  // 3 per recorded call
+  int prof_cap = 0, prof_calls = 0;
+  int last_launch[6] = {0, 0, 0, 0, 0, 0};
+};
+
+namespace {
+
+__global__ void set_entry_kernel(int32_t* table, int32_t* lens, int idx, int slot, int len) {
+  if (idx >= 0) table[idx] = slot;
+  *lens = len;
+}
+
+size_t combine_smem_floats(int np, int g, int r) { return (size_t)np * g + 3 * (size_t)g + (size_t)g * r; }
+
+int validate_params(const basiskv_params* p) {
+  if (!p) return fail(BASISKV_ERR_INVALID_ARG, "params is NULL");
+  if (p->max_batch <= 0 || p->num_kv_heads <= 0 || p->gqa_group < 1 || p->gqa_group > 8 ||
+      p->head_dim <= 0 || p->page_size <= 0 || p->rank_r <= 0 || p->rank_r > p->head_dim ||
+      p->rank_s < 0 || p->max_pages_per_seq <= 0 || p->max_topk <= 0 || p->num_slots <= 0)
+    return fail(BASISKV_ERR_INVALID_ARG,
+                "bad shape: need max_batch, Hkv, d, P, r, max_pages, max_topk, num_slots > 0, "
+                "1 <= G <= 8, r <= d, s >= 0");
+  if (p->max_batch > 65535 || p->num_kv_heads > 65535)
+    return fail(BASISKV_ERR_INVALID_ARG, "max_batch and num_kv_heads must be <= 65535");
+  if (p->dtype != BASISKV_DTYPE_BF16 && p->dtype != BASISKV_DTYPE_F32)
+    return fail(BASISKV_ERR_INVALID_ARG, "dtype must be BASISKV_DTYPE_BF16 or BASISKV_DTYPE_F32");
+  if (p->reserved != 0) return fail(BASISKV_ERR_INVALID_ARG, "reserved must be 0");
+  if (!p->z_pool || !p->k_pool || !p->w_zk || !p->b_v || (p->rank_s > 0 && (!p->r_pool || !p->b_r)))
+    return fail(BASISKV_ERR_INVALID_ARG, "pool or basis pointer is NULL");
+  const void* ptrs[] = {p->z_pool, p->k_pool, p->w_zk, p->b_v};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return fail(BASISKV_ERR_INVALID_ARG, "pools and bases must be 16-byte aligned");
+  if (p->rank_s > 0 && (!aligned16(p->r_pool) || !aligned16(p->b_r)))
+    return fail(BASISKV_ERR_INVALID_ARG, "pools and bases must be 16-byte aligned");
+  if ((size_t)p->max_batch * p->max_pages_per_seq > (size_t)1 << 31)
+    return fail(BASISKV_ERR_INVALID_ARG, "page table too large");
+  return BASISKV_OK;
+}
+
+// Pick the tensor-core kernels for this shape when the pools are bf16.
+void choose_kernels(basiskv_handle* h) {
+  const basiskv_params& p = h->p;
+  if (p.dtype != BASISKV_DTYPE_BF16) return;
+  const size_t es = 2;
+  auto rit = route_table().find(RouteKey{p.gqa_group, p.rank_r, p.rank_s});
+  if (rit != route_table().end() && p.page_size % 16 == 0 && p.head_dim % 32 == 0) {
+    const size_t stage = (size_t)p.page_size * (p.rank_r + p.rank_s) * es;
+    int st = (int)std::min<size_t>(kMaxStages, kRouteSmemBudget / (kRouteWarps * stage));
+    if (st >= 2) {
+      h->route_fn = rit->second;
+      h->route_stages = st;
+      h->route_smem = kRouteWarps * st * stage +
+                      sizeof(float) * (size_t)p.gqa_group * (p.head_dim + p.rank_r + p.rank_s);
+    }
+  }
+  for (int tps : {64, 32, 16}) {
+    if (p.page_size % tps) continue;
+    auto ait = attn_table().find(AttnKey{p.gqa_group, p.head_dim, p.rank_r, tps});
+    if (ait == attn_table().end()) continue;
+    const size_t stage = (size_t)tps * (p.head_dim + p.rank_r) * es;
+    int st = (int)std::min<size_t>(4, kAttnSmemBudget / (kAttnWarps * stage));
+    if (st < 1) continue;
+    if (st < 2 && tps > 16) continue;  // prefer a smaller stage with double buffering
+    h->attn_fn = ait->second;
+    h->attn_tps = tps;
+    h->attn_stages = st;
+    h->attn_smem = std::max(kAttnWarps * st * stage,
+                            sizeof(float) * combine_smem_floats(kPartsCap, p.gqa_group, p.rank_r));
+    break;
+  }
+}
+
+size_t generic_route_smem(const basiskv_params& p) {
+  return sizeof(float) * (size_t)p.gqa_group * (p.head_dim + p.rank_r + p.rank_s);
+}
+size_t generic_attn_smem(const basiskv_params& p) {
+  const size_t g = p.gqa_group;
+  const size_t own = g * (p.head_dim + p.page_size + p.rank_r) + 3 * g;
+  return sizeof(float) * std::max(own, combine_smem_floats(kMaxSplits, p.gqa_group, p.rank_r));
+}
+
+int set_smem_attr(const void* fn, size_t bytes) {
+  CUDA_TRY(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
+  return BASISKV_OK;
+}
+
+template <typename T>
+int set_generic_attrs(const basiskv_params& p) {
+  int rc = set_smem_attr((const void*)&route_generic_kernel<T>, generic_route_smem(p));
+  if (rc) return rc;
+  return set_smem_attr((const void*)&attn_generic_kernel<T>, generic_attn_smem(p));
+}
+
+struct LaunchPlan {
+  int batch = 0;
+  bool any_routed = false;
+  int route_ppc = 0, route_chunks = 0;
+  int attn_pps = 0, attn_splits = 0;
+};
+
+LaunchPlan plan(const basiskv_handle* h, int batch, int topk, bool force_route) {
+  LaunchPlan lp;
+  lp.batch = batch;
+  const basiskv_params& p = h->p;
+  long long route_pages = 0;
+  int max_routed = 0, max_kb = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int n = h->h_npages[b];
+    if (n > 0 && (force_route || topk < n)) {
+      route_pages += n;
+      max_routed = std::max(max_routed, n);
+    }
+    max_kb = std::max(max_kb, std::min(topk, n));
+  }
+  route_pages *= p.num_kv_heads;
+  lp.any_routed = max_routed > 0;
+  if (lp.any_routed) {
+    const long long target = (long long)h->num_sms * 8;  // about four waves of two CTAs
+    long long ppc = (route_pages + target - 1) / target;
+    ppc = std::max<long long>(kRouteWarps * 2, std::min<long long>(ppc, 512));
+    const int chunks = (int)((max_routed + ppc - 1) / ppc);
+    lp.route_ppc = (max_routed + chunks - 1) / chunks;  // even chunks for the longest sequence
+    lp.route_chunks = (max_routed + lp.route_ppc - 1) / lp.route_ppc;
+  }
+  const long long units = (long long)batch * p.num_kv_heads;
+  int splits = (int)std::max<long long>(1, ((long long)h->num_sms * 3 + units - 1) / std::max(1LL, units));
+  splits = std::min(splits, kMaxSplits);
+  splits = std::max(1, std::min(splits, std::max(1, max_kb)));
+  lp.attn_pps = std::max(1, (max_kb + splits - 1) / splits);
+  lp.attn_splits = std::max(1, (max_kb + lp.attn_pps - 1) / lp.attn_pps);
+  return lp;
+}
+
+RouteArgs route_args(basiskv_handle* h, int batch, const void* q, int topk, float* scores,
+                     int32_t* sel_out, int force, int ppc, int stages) {
+  const basiskv_params& p = h->p;
+  RouteArgs a;
+  a.q = q;
+  a.z_pool = p.z_pool;
+  a.r_pool = p.r_pool;
+  a.w_zk = p.w_zk;
+  a.b_r = p.b_r;
+  a.page_table = h->d_page_table;
+  a.seq_lens = h->d_seq_lens;
+  a.scores = scores;
+  a.sel = h->d_sel;
+  a.sel_out = sel_out;
+  a.counters = h->d_counters;
+  a.status = h->d_status;
+  a.ld_pt = p.max_pages_per_seq;
+  a.ld_sel = p.max_topk;
+  a.num_slots = p.num_slots;
+  a.num_kv_heads = p.num_kv_heads;
+  a.head_dim = p.head_dim;
+  a.page_size = p.page_size;
+  a.rank_r = p.rank_r;
+  a.rank_s = p.rank_s;
+  a.gqa_group = p.gqa_group;
+  a.topk = topk;
+  a.pages_per_cta = ppc;
+  a.stages = stages;
+  a.force = force;
+  a.fill_tail = force;
+  (void)batch;
+  return a;
+}
+
+int launch_route(basiskv_handle* h, const LaunchPlan& lp, const RouteArgs& a, cudaStream_t stream) {
+  const basiskv_params& p = h->p;
+  dim3 grid(lp.route_chunks, p.num_kv_heads, lp.batch);
+  if (h->route_fn) {
+    RouteArgs ra = a;
+    ra.stages = h->route_stages;
+    h->route_fn<<<grid, kRouteThreads, h->route_smem, stream>>>(ra);
+  } else if (p.dtype == BASISKV_DTYPE_BF16) {
+    route_generic_kernel<__nv_bfloat16><<<grid, kRouteThreads, generic_route_smem(p), stream>>>(a);
+  } else {
+    route_generic_kernel<float><<<grid, kRouteThreads, generic_route_smem(p), stream>>>(a);
+  }
+  CUDA_TRY(cudaGetLastError());
+  return BASISKV_OK;
+}
+
+int launch_attn(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk, float scale,
+                float* out, int32_t* sel_out, bool pdl, cudaStream_t stream) {
+  const basiskv_params& p = h->p;
+  AttnArgs a;
+  a.q = q;
+  a.k_pool = p.k_pool;
+  a.z_pool = p.z_pool;
+  a.b_v = p.b_v;
+  a.page_table = h->d_page_table;
+  a.seq_lens = h->d_seq_lens;
+  a.sel = h->d_sel;
+  a.sel_out = sel_out;
+  a.part_ml = h->d_part_ml;
+  a.part_acc = h->d_part_acc;
+  a.counters = h->d_counters + (size_t)p.max_batch * p.num_kv_heads;
+  a.status = h->d_status;
+  a.out = out;
+  a.ld_pt = p.max_pages_per_seq;
+  a.ld_sel = p.max_topk;
+  a.num_slots = p.num_slots;
+  a.num_kv_heads = p.num_kv_heads;
+  a.head_dim = p.head_dim;
+  a.page_size = p.page_size;
+  a.rank_r = p.rank_r;
+  a.gqa_group = p.gqa_group;
+  a.topk = topk;
+  a.pages_per_split = lp.attn_pps;
+  a.stages = h->attn_stages;
+  a.np_cap = kPartsCap;
+  a.scale_log2 = scale * 1.4426950408889634f;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(lp.attn_splits, p.num_kv_heads, lp.batch);
+  cfg.blockDim = dim3(kAttnThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  if (h->attn_fn) {
+    cfg.dynamicSmemBytes = h->attn_smem;
+    CUDA_TRY(cudaLaunchKernelEx(&cfg, h->attn_fn, a));
+  } else if (p.dtype == BASISKV_DTYPE_BF16) {
+    cfg.dynamicSmemBytes = generic_attn_smem(p);
+    CUDA_TRY(cudaLaunchKernelEx(&cfg, &attn_generic_kernel<__nv_bfloat16>, a));
+  } else {
+    cfg.dynamicSmemBytes = generic_attn_smem(p);
+    CUDA_TRY(cudaLaunchKernelEx(&cfg, &attn_generic_kernel<float>, a));
+  }
+  return BASISKV_OK;
+}
+
+int check_handle(basiskv_handle* h) {
+  if (!h) return fail(BASISKV_ERR_INVALID_ARG, "handle is NULL");
+  int dev = -1;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev != h->device) return fail(BASISKV_ERR_INVALID_ARG, "handle belongs to device %d, current is %d", h->device, dev);
+  return BASISKV_OK;
+}
+
+int check_call(basiskv_handle* h, int batch, const void* q, int topk) {
+  int rc = check_handle(h);
+  if (rc) return rc;
+  if (batch < 0 || batch > h->p.max_batch) return fail(BASISKV_ERR_INVALID_ARG, "batch %d outside [0, %d]", batch, h->p.max_batch);
+  if (topk <= 0 || topk > h->p.max_topk) return fail(BASISKV_ERR_INVALID_ARG, "topk %d outside [1, %d]", topk, h->p.max_topk);
+  if (!q || !aligned16(q)) return fail(BASISKV_ERR_INVALID_ARG, "q must be a 16-byte aligned device pointer");
+  return BASISKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int basiskv_version(void) { return 100; }
+
+const char* basiskv_last_error(void) { return g_last_error.c_str(); }
+
+int basiskv_create(const basiskv_params* p, basiskv_handle** out) {
+  if (!out) return fail(BASISKV_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  int rc = validate_params(p);
+  if (rc) return rc;
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  cudaDeviceProp prop;
+  CUDA_TRY(cudaGetDeviceProperties(&prop, dev));
+  if (prop.major != 10)
+    return fail(BASISKV_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", dev,
+                prop.major, prop.minor);
+
+  basiskv_handle* h = new basiskv_handle();
+  h->p = *p;
+  h->device = dev;
+  h->num_sms = prop.multiProcessorCount;
+  h->elem = p->dtype == BASISKV_DTYPE_BF16 ? 2 : 4;
+  const size_t B = p->max_batch, Hkv = p->num_kv_heads, U = B * Hkv, G = p->gqa_group;
+  auto cleanup_fail = [&](int code, const char* what) {
+    basiskv_destroy(h);
+    return fail(code, "%s", what);
+  };
+  struct A {
+    void** ptr;
+    size_t bytes;
+  } allocs[] = {
+      {(void**)&h->d_page_table, sizeof(int32_t) * B * p->max_pages_per_seq},
+      {(void**)&h->d_seq_lens, sizeof(int32_t) * B},
+      {(void**)&h->d_scores, sizeof(float) * U * p->max_pages_per_seq},
+      {(void**)&h->d_sel, sizeof(int32_t) * U * p->max_topk},
+      {(void**)&h->d_part_ml, sizeof(float) * U * kPartsCap * G * 2},
+      {(void**)&h->d_part_acc, sizeof(float) * U * kPartsCap * G * p->rank_r},
+      {(void**)&h->d_counters, sizeof(uint32_t) * 2 * U},
+      {(void**)&h->d_status, sizeof(uint32_t)},
+      {(void**)&h->d_q_stage, h->elem * B * Hkv * G * p->head_dim},
+      {(void**)&h->d_out_stage, sizeof(float) * B * Hkv * G * p->head_dim},
+      {(void**)&h->d_sel_stage, sizeof(int32_t) * U * p->max_topk},
+  };
+  for (auto& a : allocs) {
+    if (cudaMalloc(a.ptr, a.bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return cleanup_fail(BASISKV_ERR_OOM, "device allocation failed");
+    }
+  }
+  if (cudaMemset(h->d_page_table, 0, sizeof(int32_t) * B * p->max_pages_per_seq) != cudaSuccess ||
+      cudaMemset(h->d_seq_lens, 0, sizeof(int32_t) * B) != cudaSuccess ||
+      cudaMemset(h->d_counters, 0, sizeof(uint32_t) * 2 * U) != cudaSuccess ||
+      cudaMemset(h->d_status, 0, sizeof(uint32_t)) != cudaSuccess)
+    return cleanup_fail(BASISKV_ERR_CUDA, "cudaMemset failed");
+  h->h_table.assign(B * p->max_pages_per_seq, 0);
+  h->h_lens.assign(B, 0);
+  h->h_npages.assign(B, 0);
+
+  choose_kernels(h);
+  int arc = h->route_fn ? set_smem_attr((const void*)h->route_fn, h->route_smem) : BASISKV_OK;
+  if (!arc && h->attn_fn) arc = set_smem_attr((const void*)h->attn_fn, h->attn_smem);
+  if (!arc)
+    arc = p->dtype == BASISKV_DTYPE_BF16 ? set_generic_attrs<__nv_bfloat16>(*p) : set_generic_attrs<float>(*p);
+  if (arc) {
+    std::string msg = g_last_error;
+    basiskv_destroy(h);
+    return fail(arc, "%s", msg.c_str());
+  }
+  if (cudaDeviceSynchronize() != cudaSuccess) return cleanup_fail(BASISKV_ERR_CUDA, "device synchronize failed");
+  *out = h;
+  return BASISKV_OK;
+}
+
+int basiskv_destroy(basiskv_handle* h) {
+  if (!h) return BASISKV_OK;
+  cudaDeviceSynchronize();
+  void* ptrs[] = {h->d_page_table, h->d_seq_lens, h->d_scores, h->d_sel, h->d_part_ml, h->d_part_acc,
+                  h->d_counters, h->d_status, h->d_q_stage, h->d_out_stage, h->d_sel_stage};
+  for (void* q : ptrs)
+    if (q) cudaFree(q);
+  for (cudaEvent_t e : h->events) cudaEventDestroy(e);
+  delete h;
+  return BASISKV_OK;
+}
+
+int basiskv_append_page(basiskv_handle* h, int seq, int slot, int n_tokens, basiskv_stream_t stream) {
+  int rc = check_handle(h);
+  if (rc) return rc;
+  const basiskv_params& p = h->p;
+  if (seq < 0 || seq >= p.max_batch) return fail(BASISKV_ERR_INVALID_ARG, "seq %d outside [0, %d)", seq, p.max_batch);
+  if (slot < 0 || slot >= p.num_slots) return fail(BASISKV_ERR_INVALID_ARG, "slot %d outside [0, %d)", slot, p.num_slots);
+  if (n_tokens < 1 || n_tokens > p.page_size)
+    return fail(BASISKV_ERR_INVALID_ARG, "n_tokens %d outside [1, %d]", n_tokens, p.page_size);
+  const int n = h->h_npages[seq];
+  if (n > 0 && h->h_lens[seq] != n * p.page_size)
+    return fail(BASISKV_ERR_STATE, "sequence %d ends in a partial page", seq);
+  if (n >= p.max_pages_per_seq) return fail(BASISKV_ERR_CAPACITY, "sequence %d already has %d pages", seq, n);
+  const int idx = seq * p.max_pages_per_seq + n;
+  const int len = h->h_lens[seq] + n_tokens;
+  set_entry_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(h->d_page_table, h->d_seq_lens + seq, idx, slot, len);
+  CUDA_TRY(cudaGetLastError());
+  h->h_table[idx] = slot;
+  h->h_lens[seq] = len;
+  h->h_npages[seq] = n + 1;
+  return BASISKV_OK;
+}
+
+int basiskv_append_tokens(basiskv_handle* h, int seq, int n_tokens, basiskv_stream_t stream) {
+  int rc = check_handle(h);
+  if (rc) return rc;
+  const basiskv_params& p = h->p;
+  if (seq < 0 || seq >= p.max_batch) return fail(BASISKV_ERR_INVALID_ARG, "seq %d outside [0, %d)", seq, p.max_batch);
+  if (n_tokens < 1) return fail(BASISKV_ERR_INVALID_ARG, "n_tokens must be >= 1");
+  const int n = h->h_npages[seq];
+  if (n == 0) return fail(BASISKV_ERR_STATE, "sequence %d has no page", seq);
+  const int len = h->h_lens[seq] + n_tokens;
+  if (len > n * p.page_size) return fail(BASISKV_ERR_STATE, "last page of sequence %d would overflow", seq);
+  set_entry_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(h->d_page_table, h->d_seq_lens + seq, -1, 0, len);
+  CUDA_TRY(cudaGetLastError());
+  h->h_lens[seq] = len;
+  return BASISKV_OK;
+}
+
+int basiskv_reset_seq(basiskv_handle* h, int seq, basiskv_stream_t stream) {
+  int rc = check_handle(h);
+  if (rc) return rc;
+  if (seq < 0 || seq >= h->p.max_batch) return fail(BASISKV_ERR_INVALID_ARG, "seq %d outside [0, %d)", seq, h->p.max_batch);
+  set_entry_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(h->d_page_table, h->d_seq_lens + seq, -1, 0, 0);
+  CUDA_TRY(cudaGetLastError());
+  h->h_lens[seq] = 0;
+  h->h_npages[seq] = 0;
+  return BASISKV_OK;
+}
+
+int basiskv_load_page_table(basiskv_handle* h, int batch, const int32_t* page_table, int ld,
+                            const int32_t* seq_lens, basiskv_stream_t stream) {
+  int rc = check_handle(h);
+  if (rc) return rc;
+  const basiskv_params& p = h->p;
+  if (batch < 0 || batch > p.max_batch) return fail(BASISKV_ERR_INVALID_ARG, "batch %d outside [0, %d]", batch, p.max_batch);
+  if (batch > 0 && (!page_table || !seq_lens || ld <= 0)) return fail(BASISKV_ERR_INVALID_ARG, "NULL table or lens");
+  std::vector<int32_t> tab((size_t)batch * p.max_pages_per_seq, 0), lens(batch), np(batch);
+  for (int b = 0; b < batch; ++b) {
+    const int L = seq_lens[b];
+    if (L < 0) return fail(BASISKV_ERR_INVALID_ARG, "seq_lens[%d] = %d", b, L);
+    const int n = (L + p.page_size - 1) / p.page_size;
+    if (n > p.max_pages_per_seq || n > ld)
+      return fail(BASISKV_ERR_CAPACITY, "sequence %d needs %d pages (max %d, ld %d)", b, n, p.max_pages_per_seq, ld);
+    for (int j = 0; j < n; ++j) {
+      const int s = page_table[(size_t)b * ld + j];
+      if (s < 0 || s >= p.num_slots) return fail(BASISKV_ERR_INVALID_ARG, "page_table[%d][%d] = %d outside [0, %d)", b, j, s, p.num_slots);
+      tab[(size_t)b * p.max_pages_per_seq + j] = s;
+    }
+    lens[b] = L;
+    np[b] = n;
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  if (batch > 0) {
+    CUDA_TRY(cudaMemcpyAsync(h->d_page_table, tab.data(), sizeof(int32_t) * tab.size(), cudaMemcpyHostToDevice, st));
+    CUDA_TRY(cudaMemcpyAsync(h->d_seq_lens, lens.data(), sizeof(int32_t) * batch, cudaMemcpyHostToDevice, st));
+  }
+  CUDA_TRY(cudaStreamSynchronize(st));
+  std::copy(tab.begin(), tab.end(), h->h_table.begin());
+  std::copy(lens.begin(), lens.end(), h->h_lens.begin());
+  std::copy(np.begin(), np.end(), h->h_npages.begin());
+  return BASISKV_OK;
+}
+
+int basiskv_decode_attn(basiskv_handle* h, int batch, const void* q, int topk, float softmax_scale,
+                        float* out, int32_t* sel_out, basiskv_stream_t stream) {
+  int rc = check_call(h, batch, q, topk);
+  if (rc) return rc;
+  if (!out) return fail(BASISKV_ERR_INVALID_ARG, "out is NULL");
+  if (!std::isfinite(softmax_scale)) return fail(BASISKV_ERR_INVALID_ARG, "softmax_scale must be finite");
+  if (batch == 0) return BASISKV_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  const LaunchPlan lp = plan(h, batch, topk, false);
+  const bool prof = h->prof_calls < h->prof_cap;
+  cudaEvent_t* ev = prof ? &h->events[3 * h->prof_calls] : nullptr;
+  if (prof) CUDA_TRY(cudaEventRecord(ev[0], st));
+  if (lp.any_routed) {
+    RouteArgs ra = route_args(h, batch, q, topk, h->d_scores, sel_out, 0, lp.route_ppc, 0);
+    rc = launch_route(h, lp, ra, st);
+    if (rc) return rc;
+  }
+  if (prof) CUDA_TRY(cudaEventRecord(ev[1], st));
+  rc = launch_attn(h, lp, q, topk, softmax_scale, out, sel_out, lp.any_routed && !prof, st);
+  if (rc) return rc;
+  if (prof) {
+    CUDA_TRY(cudaEventRecord(ev[2], st));
+    ++h->prof_calls;
+  }
+  h->last_launch[0] = lp.any_routed ? lp.route_ppc : 0;
+  h->last_launch[1] = lp.any_routed ? lp.route_chunks * h->p.num_kv_heads * batch : 0;
+  h->last_launch[2] = lp.attn_splits;
+  h->last_launch[3] = lp.attn_splits * h->p.num_kv_heads * batch;
+  h->last_launch[4] = h->route_fn != nullptr;
+  h->last_launch[5] = h->attn_fn != nullptr;
+  return BASISKV_OK;
+}
+
+int basiskv_decode_attn_host(basiskv_handle* h, int batch, const void* q_host, int topk, float softmax_scale,
+                             float* out_host, int32_t* sel_host, basiskv_stream_t stream) {
+  int rc = check_handle(h);
+  if (rc) return rc;
+  if (!q_host || !out_host) return fail(BASISKV_ERR_INVALID_ARG, "q_host or out_host is NULL");
+  if (batch < 0 || batch > h->p.max_batch) return fail(BASISKV_ERR_INVALID_ARG, "batch %d outside [0, %d]", batch, h->p.max_batch);
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t rows = (size_t)batch * h->p.num_kv_heads * h->p.gqa_group;
+  CUDA_TRY(cudaMemcpyAsync(h->d_q_stage, q_host, h->elem * rows * h->p.head_dim, cudaMemcpyHostToDevice, st));
+  rc = basiskv_decode_attn(h, batch, h->d_q_stage, topk, softmax_scale, h->d_out_stage,
+                           sel_host ? h->d_sel_stage : nullptr, stream);
+  if (rc) return rc;
+  CUDA_TRY(cudaMemcpyAsync(out_host, h->d_out_stage, sizeof(float) * rows * h->p.head_dim, cudaMemcpyDeviceToHost, st));
+  if (sel_host)
+    CUDA_TRY(cudaMemcpyAsync(sel_host, h->d_sel_stage, sizeof(int32_t) * batch * h->p.num_kv_heads * topk,
+                             cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(cudaStreamSynchronize(st));
+  return BASISKV_OK;
+}
+
+int basiskv_route(basiskv_handle* h, int batch, const void* q, int topk, float* scores_out, int32_t* sel_out,
+                  basiskv_stream_t stream) {
+  int rc = check_call(h, batch, q, topk);
+  if (rc) return rc;
+  if (batch == 0) return BASISKV_OK;
+  const LaunchPlan lp = plan(h, batch, topk, true);
+  if (!lp.any_routed) {
+    if (scores_out || sel_out) {
+      // no sequence has a page: scores all -inf, selections all -1
+      if (scores_out) {
+        std::vector<float> ninf((size_t)batch * h->p.num_kv_heads * h->p.max_pages_per_seq, -INFINITY);
+        CUDA_TRY(cudaMemcpyAsync(scores_out, ninf.data(), sizeof(float) * ninf.size(), cudaMemcpyHostToDevice, (cudaStream_t)stream));
+        CUDA_TRY(cudaStreamSynchronize((cudaStream_t)stream));
+      }
+      if (sel_out) CUDA_TRY(cudaMemsetAsync(sel_out, 0xff, sizeof(int32_t) * batch * h->p.num_kv_heads * topk, (cudaStream_t)stream));
+    }
+    return BASISKV_OK;
+  }
+  RouteArgs ra = route_args(h, batch, q, topk, scores_out ? scores_out : h->d_scores, sel_out, 1, lp.route_ppc, 0);
+  return launch_route(h, lp, ra, (cudaStream_t)stream);
+}
+
+int basiskv_get_status(basiskv_handle* h, uint32_t* status, int clear) {
+  int rc = check_handle(h);
+  if (rc) return rc;
+  if (!status) return fail(BASISKV_ERR_INVALID_ARG, "status is NULL");
+  CUDA_TRY(cudaDeviceSynchronize());
+  CUDA_TRY(cudaMemcpy(status, h->d_status, sizeof(uint32_t), cudaMemcpyDeviceToHost));
+  if (clear) CUDA_TRY(cudaMemset(h->d_status, 0, sizeof(uint32_t)));
+  return BASISKV_OK;
+}
+
+int basiskv_profile_begin(basiskv_handle* h, int max_calls) {
+  int rc = check_handle(h);
+  if (rc) return rc;
+  if (max_calls < 0) return fail(BASISKV_ERR_INVALID_ARG, "max_calls < 0");
+  while ((int)h->events.size() < 3 * max_calls) {
+    cudaEvent_t e;
+    CUDA_TRY(cudaEventCreate(&e));
+    h->events.push_back(e);
+  }
+  h->prof_cap = max_calls;
+  h->prof_calls = 0;
+  return BASISKV_OK;
+}
+
+int basiskv_profile_end(basiskv_handle* h, float* route_ms, float* attn_ms, float* total_ms, int* ncalls) {
+  int rc = check_handle(h);
+  if (rc) return rc;
+  for (int i = 0; i < h->prof_calls; ++i) {
+    cudaEvent_t* ev = &h->events[3 * i];
+    CUDA_TRY(cudaEventSynchronize(ev[2]));
+    float a = 0.f, b = 0.f, c = 0.f;
+    CUDA_TRY(cudaEventElapsedTime(&a, ev[0], ev[1]));
+    CUDA_TRY(cudaEventElapsedTime(&b, ev[1], ev[2]));
+    CUDA_TRY(cudaEventElapsedTime(&c, ev[0], ev[2]));
+    if (route_ms) route_ms[i] = a;
+    if (attn_ms) attn_ms[i] = b;
+    if (total_ms) total_ms[i] = c;
+  }
+  if (ncalls) *ncalls = h->prof_calls;
+  h->prof_cap = 0;
+  h->prof_calls = 0;
+  return BASISKV_OK;
+}
+
+int basiskv_last_launch(basiskv_handle* h, int info[6]) {
+  int rc = check_handle(h);
+  if (rc) return rc;
+  if (!info) return fail(BASISKV_ERR_INVALID_ARG, "info is NULL");
+  for (int i = 0; i < 6; ++i) info[i] = h->last_launch[i];
+  return BASISKV_OK;
+}
+
+}  // extern "C"

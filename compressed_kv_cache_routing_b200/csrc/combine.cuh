@@ -1,0 +1,72 @@
+// Merge of split-K attention partials and expansion through B_v (BasisKV:
+// the attention result is a weighted latent; the per-KV-head basis B_v turns
+// it into a value, "Value compression associated with the output
+// projection").
+//
+// Partial j of query head h holds (m_j, l_j, acc_j[r]) with m_j a running
+// max in log2 units, l_j = sum 2^(s - m_j), acc_j = sum 2^(s - m_j) Z_t.
+// With M = max_j m_j:  l = sum_j l_j 2^(m_j - M),
+//                      zbar = sum_j acc_j 2^(m_j - M) / l,
+//                      out_h = zbar . B_v  (fp32, d wide).
+// A head with no token at all (M = -inf) gets out = 0.
+#pragma once
+
+#include "common.cuh"
+
+namespace basiskv {
+
+struct CombineArgs {
+  const float* part_ml;   // [NP][G][2] of this unit
+  const float* part_acc;  // [NP][G][r] of this unit
+  const float* b_v;       // [r][d] of this KV head
+  float* out;             // [G][d] of this unit (row stride d)
+  int np, g, r, d;
+};
+
+// smem: np*g + 2*g + g*r floats.  All NT threads must call it.
+template <int NT>
+__device__ void combine_unit(const CombineArgs& c, float* smem) {
+  const int tid = threadIdx.x;
+  float* w = smem;                 // [np][g] merge weights
+  float* lsum = w + c.np * c.g;    // [g]
+  float* zbar = lsum + c.g;        // [g][r]
+  float* mmax = zbar + c.g * c.r;  // [g]
+  for (int h = tid; h < c.g; h += NT) {
+    float M = -INFINITY;
+    for (int j = 0; j < c.np; ++j) M = fmaxf(M, __ldcg(c.part_ml + (j * c.g + h) * 2));
+    mmax[h] = M;
+  }
+  __syncthreads();
+  for (int i = tid; i < c.np * c.g; i += NT) {
+    const int h = i % c.g;
+    const float mj = __ldcg(c.part_ml + i * 2);
+    w[i] = (mj == -INFINITY) ? 0.f : exp2f(mj - mmax[h]);
+  }
+  __syncthreads();
+  for (int h = tid; h < c.g; h += NT) {
+    float l = 0.f;
+    for (int j = 0; j < c.np; ++j) l += w[j * c.g + h] * __ldcg(c.part_ml + (j * c.g + h) * 2 + 1);
+    lsum[h] = l;
+  }
+  __syncthreads();
+  for (int i = tid; i < c.g * c.r; i += NT) {
+    const int h = i / c.r, a = i % c.r;
+    float acc = 0.f;
+    for (int j = 0; j < c.np; ++j) {
+      const float wj = w[j * c.g + h];
+      if (wj != 0.f) acc += wj * __ldcg(c.part_acc + (j * c.g + h) * c.r + a);
+    }
+    const float l = lsum[h];
+    zbar[i] = l > 0.f ? acc / l : 0.f;
+  }
+  __syncthreads();
+  for (int i = tid; i < c.g * c.d; i += NT) {
+    const int h = i / c.d, col = i % c.d;
+    const float* z = zbar + h * c.r;
+    float o = 0.f;
+    for (int a = 0; a < c.r; ++a) o = fmaf(z[a], __ldg(c.b_v + a * c.d + col), o);
+    c.out[h * c.d + col] = o;
+  }
+}
+
+}  // namespace basiskv

@@ -1,0 +1,136 @@
+// Deterministic block-wide top-k page selection (BasisKV routing, "selected
+// pages": the k pages of largest routing score per (sequence, KV head);
+// equal scores go to the lower page index; the result is listed ascending).
+//
+// Scores are mapped to order-preserving unsigned keys; an MSB-first radix
+// select (four 8-bit digits) finds the k-th largest key T and how many keys
+// equal to T must be taken; a block scan in page order then takes every key
+// above T plus the lowest-index keys equal to T.  The scores are read from
+// global memory (L2) on every pass, so no shared buffer bounds the page count.
+#pragma once
+
+#include "common.cuh"
+
+namespace basiskv {
+
+// Order-preserving map float -> uint32 (larger float -> larger key).  -inf
+// maps below every finite score; a NaN with the sign bit clear ranks above
+// +inf.
+__device__ __forceinline__ uint32_t score_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+struct TopkSmem {
+  int hist[256];
+  int scan_tmp[32];
+  int digit;
+  int remaining;
+};
+
+// Select min(k, n) of the n scores at `scores` (global, written by other
+// CTAs of this grid: read through L2).  Writes the ascending page list to
+// sel[0 .. min(k,n)) and, when sel_out is not null, the same list padded with
+// -1 to sel_out[0 .. out_len).  All NT threads of the block must call it.
+template <int NT>
+__device__ void block_topk(const float* scores, int n, int k, int32_t* sel, int32_t* sel_out,
+                           int out_len, TopkSmem& sm) {
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int kb = k < n ? k : n;
+
+  uint32_t thr = 0u;      // the kb-th largest key
+  int need = 0;           // keys equal to thr to take, lowest page first
+  if (kb < n) {
+    uint32_t prefix = 0u, mask = 0u;
+    int remaining = kb;
+#pragma unroll 1
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += NT) sm.hist[i] = 0;
+      __syncthreads();
+      for (int i = tid; i < n; i += NT) {
+        const uint32_t key = score_key(__ldcg(scores + i));
+        if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 255u], 1);
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // lane l owns digits [8l, 8l+8); count keys in higher digits
+        int local = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) local += sm.hist[8 * lane + q];
+        int incl = local;  // keys in digits >= 8l
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_down_sync(0xffffffffu, incl, o);
+          if (lane + o < 32) incl += y;
+        }
+        const int above = incl - local;
+        if (above < remaining && remaining <= incl) {
+          int acc = above;
+          for (int q = 7; q >= 0; --q) {
+            const int c = sm.hist[8 * lane + q];
+            if (acc + c >= remaining) {
+              sm.digit = 8 * lane + q;
+              sm.remaining = remaining - acc;
+              break;
+            }
+            acc += c;
+          }
+        }
+      }
+      __syncthreads();
+      prefix |= static_cast<uint32_t>(sm.digit) << shift;
+      mask |= 0xFFu << shift;
+      remaining = sm.remaining;
+      __syncthreads();
+    }
+    thr = prefix;
+    need = remaining;
+  }
+
+  // each thread owns a contiguous run of pages, so scans follow page order
+  const int per = (n + NT - 1) / NT;
+  const int i0 = min(n, tid * per), i1 = min(n, i0 + per);
+  int total;
+  int eq_before = 0;
+  if (kb < n) {
+    int eq = 0;
+    for (int i = i0; i < i1; ++i) eq += score_key(__ldcg(scores + i)) == thr;
+    eq_before = block_exclusive_scan<NT>(eq, sm.scan_tmp, &total);
+  }
+  int taken = 0;
+  {
+    int e = eq_before;
+    for (int i = i0; i < i1; ++i) {
+      bool take = true;
+      if (kb < n) {
+        const uint32_t key = score_key(__ldcg(scores + i));
+        take = key > thr || (key == thr && e < need);
+        e += key == thr;
+      }
+      taken += take;
+    }
+  }
+  int pos = block_exclusive_scan<NT>(taken, sm.scan_tmp, &total);
+  {
+    int e = eq_before;
+    for (int i = i0; i < i1; ++i) {
+      bool take = true;
+      if (kb < n) {
+        const uint32_t key = score_key(__ldcg(scores + i));
+        take = key > thr || (key == thr && e < need);
+        e += key == thr;
+      }
+      if (take) {
+        sel[pos] = i;
+        if (sel_out) sel_out[pos] = i;
+        ++pos;
+      }
+    }
+  }
+  if (sel_out)
+    for (int i = kb + tid; i < out_len; i += NT) sel_out[i] = -1;
+  (void)lane;
+}
+
+}  // namespace basiskv

@@ -1,0 +1,205 @@
+/*
+ * basiskv.h -- C ABI of the B200 (sm_100a) BasisKV decode-attention library.
+ *
+ * The operation: one decode step of attention over a compressed, paged KV
+ * cache in the form of "BasisKV: Value Latents for Communication and Key
+ * Routing" (English abstract):
+ *   - Values are stored only as rank-r latents Z; a per-KV-head basis B_v
+ *     expands a latent back to a value (V ~ Z.B_v).
+ *   - Routing: the Value latents predict part of each key and a rank-s
+ *     Key-specific residual R holds what they cannot, so the routing key is
+ *     Khat = Z.W_zk + R.B_r.  A page's score is the largest q_h.Khat_t over
+ *     the G query heads of the KV head's group and the page's valid tokens.
+ *   - Selection: the k pages of largest score per (sequence, KV head); equal
+ *     scores go to the lower page index.
+ *   - Exact attention: the original keys K are read only for the selected
+ *     pages; softmax(scale * q_h.K_t) over their valid tokens weights the
+ *     latents, and the weighted latent is expanded by B_v.
+ *
+ * Layouts (row-major, element type = the pool dtype unless stated):
+ *   z_pool [num_slots][Hkv][P][r]     value latents Z
+ *   r_pool [num_slots][Hkv][P][s]     key residuals R (NULL when s = 0)
+ *   k_pool [num_slots][Hkv][P][d]     original keys K
+ *   w_zk   [Hkv][r][d]  fp32          latent-to-key basis
+ *   b_r    [Hkv][s][d]  fp32          residual-to-key basis (NULL when s = 0)
+ *   b_v    [Hkv][r][d]  fp32          latent-to-value basis
+ *   q      [batch][Hkv*G][d]          query; head h of KV head kvh is kvh*G + h
+ *   out    [batch][Hkv*G][d] fp32
+ *   sel    [batch][Hkv][topk] int32   selected pages, ascending, -1 padded
+ * A "slot" holds one page (P tokens) of every KV head.  Logical page j of
+ * sequence b (tokens j*P .. j*P+P-1) lives in slot page_table[b][j].  Rows
+ * past a sequence's length in its last page are never read into a result
+ * (their contents are ignored, whatever they hold).
+ *
+ * Pointers are DEVICE pointers unless a comment says "host".  The library
+ * never frees or writes caller memory other than the outputs named in each
+ * call.  Every call returns BASISKV_OK (0) or a negative error code and, on
+ * error, leaves a message for basiskv_last_error().  Calls taking a stream
+ * enqueue on it and return without waiting unless the comment says otherwise.
+ * A handle is not thread-safe: one host thread (or external locking) per
+ * handle.
+ */
+#ifndef BASISKV_H
+#define BASISKV_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BASISKV_API __attribute__((visibility("default")))
+#else
+#define BASISKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                          /* cudaStream_t is CUstream_st* */
+typedef struct CUstream_st *basiskv_stream_t;
+
+enum {
+    BASISKV_OK = 0,
+    BASISKV_ERR_INVALID_ARG = -1, /* bad argument, shape or alignment      */
+    BASISKV_ERR_OOM = -2,         /* device allocation failed (create)      */
+    BASISKV_ERR_CUDA = -3,        /* a CUDA runtime call failed             */
+    BASISKV_ERR_UNSUPPORTED = -4, /* no sm_100 device, or unsupported shape */
+    BASISKV_ERR_CAPACITY = -5,    /* page table row full                    */
+    BASISKV_ERR_STATE = -6        /* e.g. appending a page after a partial  */
+};
+
+/* Device-side status bits (basiskv_get_status).  Kernels never trap: a
+ * detected fault sets a bit and the kernel completes with garbage output for
+ * the affected unit. */
+enum {
+    BASISKV_STATUS_BAD_SLOT = 1u,   /* a page-table entry outside [0, num_slots) */
+    BASISKV_STATUS_TIMEOUT = 2u,    /* a bounded wait on a copy expired          */
+    BASISKV_STATUS_BAD_PAGE = 4u    /* a selected page outside [0, n_b)          */
+};
+
+enum { BASISKV_DTYPE_BF16 = 0, BASISKV_DTYPE_F32 = 1 };
+
+/* Creation parameters.  Shapes: Hkv = num_kv_heads, G = gqa_group (1..8),
+ * d = head_dim, P = page_size, r = rank_r (1..d), s = rank_s (0 allowed).
+ * The fast bf16 path needs d % 32 == 0, P % 16 == 0, r % 8 == 0,
+ * s % 8 == 0 and (G, d, r, s) among the compiled shapes; every other shape
+ * runs the generic CUDA-core kernels (also the fp32 path).  All pools and
+ * bases must be 16-byte aligned; pool row strides follow from the shapes. */
+typedef struct basiskv_params {
+    int32_t max_batch;          /* sequences addressable by the page table   */
+    int32_t num_kv_heads;
+    int32_t gqa_group;
+    int32_t head_dim;
+    int32_t page_size;
+    int32_t rank_r;
+    int32_t rank_s;
+    int32_t max_pages_per_seq;  /* page-table row length                     */
+    int32_t max_topk;           /* largest topk a decode call may ask for    */
+    int32_t num_slots;          /* pages the pools hold                      */
+    int32_t dtype;              /* BASISKV_DTYPE_*                           */
+    int32_t reserved;           /* must be 0                                 */
+    const void *z_pool;         /* caller-owned, read-only during calls      */
+    const void *r_pool;
+    const void *k_pool;
+    const float *w_zk;
+    const float *b_r;
+    const float *b_v;
+} basiskv_params;
+
+typedef struct basiskv_handle basiskv_handle;
+
+/* Validate *p and allocate the library-owned state on the current device:
+ * the device page table [max_batch][max_pages_per_seq], sequence lengths, and
+ * the decode workspace (page scores, selection, split partials, arrival
+ * counters, status word).  Pools and bases stay caller-owned and must outlive
+ * the handle.  Errors: INVALID_ARG (shape, null or misaligned pointer),
+ * UNSUPPORTED (device is not compute capability 10.x), OOM, CUDA. */
+BASISKV_API int basiskv_create(const basiskv_params *p, basiskv_handle **out);
+
+/* Free the library-owned state (never the caller's pools).  Synchronises the
+ * device first.  NULL is accepted. */
+BASISKV_API int basiskv_destroy(basiskv_handle *h);
+
+/* Append pool slot `slot`, holding n_tokens (1..P) valid tokens, as the next
+ * logical page of sequence `seq`.  Only a sequence's last page may be
+ * partial, so appending after a partial page is STATE.  Stream-ordered
+ * (a one-thread kernel writes the entry); the host mirror used for launch
+ * sizing is updated immediately.  Errors: INVALID_ARG, CAPACITY, STATE. */
+BASISKV_API int basiskv_append_page(basiskv_handle *h, int seq, int slot, int n_tokens,
+                        basiskv_stream_t stream);
+
+/* Grow the last (partial) page of `seq` by n_tokens; the new rows must
+ * already be written in its slot.  Errors: INVALID_ARG, STATE (no page, or
+ * the page would overflow P). */
+BASISKV_API int basiskv_append_tokens(basiskv_handle *h, int seq, int n_tokens,
+                          basiskv_stream_t stream);
+
+/* Forget every page of `seq` (length 0).  Stream-ordered. */
+BASISKV_API int basiskv_reset_seq(basiskv_handle *h, int seq, basiskv_stream_t stream);
+
+/* Replace the page table of sequences [0, batch) from HOST arrays:
+ * page_table [batch][ld] (entries past ceil(seq_lens[b]/P) ignored) and
+ * seq_lens [batch].  Validates every entry, then copies and waits for the
+ * copy (synchronous w.r.t. the host: a set-up call, not for the decode
+ * loop).  Errors: INVALID_ARG, CAPACITY, CUDA. */
+BASISKV_API int basiskv_load_page_table(basiskv_handle *h, int batch, const int32_t *page_table,
+                            int ld, const int32_t *seq_lens, basiskv_stream_t stream);
+
+/* One decode step for sequences [0, batch):
+ *   q        [batch][Hkv*G][d] in the pool dtype (device)
+ *   topk     pages kept per (sequence, KV head), 1..max_topk; when
+ *            topk >= n_b every page of sequence b is used and its routing
+ *            is skipped
+ *   out      [batch][Hkv*G][d] fp32 (device)
+ *   sel_out  [batch][Hkv][topk] int32 or NULL (device)
+ * Enqueues the routing kernel (scores, fused top-k) and the attention
+ * kernel (split exact QK + softmax + latent sum, fused combine and B_v) on
+ * `stream`; no allocation, no host synchronisation.  A sequence of length 0
+ * gets out = 0 and sel = -1.  Device-detected faults set status bits.
+ * Errors: INVALID_ARG. */
+BASISKV_API int basiskv_decode_attn(basiskv_handle *h, int batch, const void *q, int topk,
+                        float softmax_scale, float *out, int32_t *sel_out,
+                        basiskv_stream_t stream);
+
+/* The same step with HOST buffers: copies q_host (pinned or pageable) to a
+ * library-owned device buffer, runs basiskv_decode_attn, copies out (and
+ * sel when sel_host is not NULL) back, and waits for the stream. */
+BASISKV_API int basiskv_decode_attn_host(basiskv_handle *h, int batch, const void *q_host, int topk,
+                             float softmax_scale, float *out_host, int32_t *sel_host,
+                             basiskv_stream_t stream);
+
+/* Routing alone (steps route-prep, route-score, top-k) for every sequence
+ * with at least one page, whether or not topk >= n_b.  scores_out
+ * [batch][Hkv][max_pages_per_seq] fp32 (device, nullable) receives the page
+ * scores (-inf past n_b); sel_out [batch][Hkv][topk] (device, nullable). */
+BASISKV_API int basiskv_route(basiskv_handle *h, int batch, const void *q, int topk,
+                  float *scores_out, int32_t *sel_out, basiskv_stream_t stream);
+
+/* Read (and optionally clear) the device status bits.  Synchronises the
+ * device. */
+BASISKV_API int basiskv_get_status(basiskv_handle *h, uint32_t *status, int clear);
+
+/* Kernel timing: after basiskv_profile_begin(h, n), the next n decode calls
+ * record CUDA events on their stream around the routing and the attention
+ * kernel.  basiskv_profile_end waits for them and writes per-call
+ * milliseconds into route_ms[i] / attn_ms[i] / total_ms[i] (host arrays of
+ * length >= n, nullable) and the number of recorded calls into *ncalls. */
+BASISKV_API int basiskv_profile_begin(basiskv_handle *h, int max_calls);
+BASISKV_API int basiskv_profile_end(basiskv_handle *h, float *route_ms, float *attn_ms,
+                        float *total_ms, int *ncalls);
+
+/* Launch shape chosen for the last decode call (for reports): routing pages
+ * per CTA and CTA count, attention splits per unit and CTA count, and
+ * whether the tensor-core kernels ran (1) or the generic ones (0). */
+BASISKV_API int basiskv_last_launch(basiskv_handle *h, int info[6]);
+
+/* Thread-local message for the last non-zero return of this thread. */
+BASISKV_API const char *basiskv_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+BASISKV_API int basiskv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BASISKV_H */

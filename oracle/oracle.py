@@ -190,8 +190,8 @@ def route(prob: Problem, units=None, library=None):
     scores = np.full((prob.batch, prob.num_kv_heads, prob.page_table.shape[1]), -np.inf)
     sel = np.full((prob.batch, prob.num_kv_heads, prob.topk), -1, dtype=np.int32)
     gap = np.full((prob.batch, prob.num_kv_heads), np.nan)
-    m = _mask(prob, units)
-    st = prob._struct(m)
+    mask = _mask(prob, units)  # must outlive the call: the struct holds its address
+    st = prob._struct(mask)
     l = library if library is not None else lib()
     rc = l.oracle_route(ctypes.byref(st), scores.ctypes.data, sel.ctypes.data, gap.ctypes.data)
     if rc:
@@ -204,7 +204,8 @@ def attend(prob: Problem, sel: np.ndarray, units=None, library=None):
     """Exact attention over the pages in ``sel``; out [B][Hkv*G][d] float64."""
     sel = np.ascontiguousarray(sel, dtype=np.int32)
     out = np.zeros((prob.batch, prob.num_kv_heads * prob.gqa_group, prob.head_dim))
-    st = prob._struct(_mask(prob, units))
+    mask = _mask(prob, units)  # must outlive the call: the struct holds its address
+    st = prob._struct(mask)
     l = library if library is not None else lib()
     rc = l.oracle_attend(ctypes.byref(st), sel.ctypes.data, out.ctypes.data)
     if rc:
@@ -218,7 +219,8 @@ def decode(prob: Problem, units=None, want_scores=False, library=None):
     sel = np.full((prob.batch, prob.num_kv_heads, prob.topk), -1, dtype=np.int32)
     gap = np.full((prob.batch, prob.num_kv_heads), np.nan)
     out = np.zeros((prob.batch, prob.num_kv_heads * prob.gqa_group, prob.head_dim))
-    st = prob._struct(_mask(prob, units))
+    mask = _mask(prob, units)  # must outlive the call: the struct holds its address
+    st = prob._struct(mask)
     l = library if library is not None else lib()
     rc = l.oracle_decode(ctypes.byref(st), int(bool(want_scores)), scores.ctypes.data,
                          sel.ctypes.data, gap.ctypes.data, out.ctypes.data)

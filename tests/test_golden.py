@@ -32,3 +32,19 @@ def test_tiny_golden():
     n = len(doc["page_scores"])
     assert np.array_equal(scores[0, 0, :n], np.array(doc["page_scores"]))
     assert np.array_equal(out[0], np.array(doc["out"]))
+
+
+def test_unit_sampling_matches_full_run():
+    """Oracle on a subset of units equals the full run on those units."""
+    spec = W.shrink("high_concurrency", batch=6, len_lo=700, len_hi=1500, topk=8)
+    w = W.generate(spec)
+    prob = to_problem(w)
+    full = oracle.decode(prob)
+    units = [1, 7, 30, 47]
+    part = oracle.decode(prob, units=units)
+    for u in units:
+        b, kvh = divmod(u, spec.num_kv_heads)
+        G = spec.gqa_group
+        assert np.array_equal(part[1][b, kvh], full[1][b, kvh])
+        assert np.array_equal(part[0][b, kvh * G:(kvh + 1) * G], full[0][b, kvh * G:(kvh + 1) * G])
+    assert (part[1][0, 0] == -1).all()  # unit 0 not computed

@@ -1,0 +1,259 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle.
+
+Selections must match bit for bit; outputs within a row-normalised max
+relative error of 2e-3 (max over (b, h) of |y - y*|_inf / |y*|_inf), the
+bound for bf16 storage with fp32 accumulation.  Page scores from the routing
+kernel are compared too (relative 1e-3).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from compressed_kv_cache_routing_b200 import basiskv as bk
+from compressed_kv_cache_routing_b200 import workloads as W
+from oracle import oracle
+from helpers import to_problem
+
+pytestmark = pytest.mark.gpu
+
+OUT_TOL = 2e-3
+SCORE_TOL = 1e-3
+
+
+def setup_module():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    from compressed_kv_cache_routing_b200 import build
+    build.build()
+
+
+def gpu_decode(w, topk=None, scale=None, kv=None, max_topk=None):
+    s = w.spec
+    topk = s.topk if topk is None else topk
+    scale = s.softmax_scale if scale is None else scale
+    own = kv is None
+    if own:
+        kv = bk.BasisKV.for_workload(w, max_topk=max(topk, max_topk or 0))
+    B = len(w.seq_lens)
+    out = torch.full((B, s.num_q_heads, s.head_dim), float("nan"), device="cuda")
+    sel = torch.full((B, s.num_kv_heads, topk), -7, device="cuda", dtype=torch.int32)
+    bk.basiskv_decode_attn(kv.handle, w.q[:B], topk, scale, out, sel)
+    torch.cuda.synchronize()
+    assert bk.basiskv_get_status(kv.handle, clear=True) == 0
+    res = out.cpu().numpy(), sel.cpu().numpy()
+    if own:
+        kv.close()
+    return res
+
+
+def gpu_scores(w, topk=None):
+    s = w.spec
+    topk = s.topk if topk is None else topk
+    kv = bk.BasisKV.for_workload(w, max_topk=topk)
+    B = len(w.seq_lens)
+    sc = torch.zeros((B, s.num_kv_heads, w.page_table.shape[1]), device="cuda")
+    sel = torch.zeros((B, s.num_kv_heads, topk), device="cuda", dtype=torch.int32)
+    bk.basiskv_route(kv.handle, w.q[:B], topk, sc, sel)
+    torch.cuda.synchronize()
+    assert bk.basiskv_get_status(kv.handle) == 0
+    kv.close()
+    return sc.cpu().numpy(), sel.cpu().numpy()
+
+
+def out_error(out, ref, mask=None):
+    """Max over rows of |y - y*|_inf / |y*|_inf; rows with y* == 0 must be 0."""
+    worst = 0.0
+    for idx in np.ndindex(ref.shape[:2]):
+        if mask is not None and not mask[idx]:
+            continue
+        y, ys = out[idx].astype(np.float64), ref[idx]
+        den = np.abs(ys).max()
+        if den == 0:
+            assert np.abs(y).max() == 0, idx
+            continue
+        worst = max(worst, np.abs(y - ys).max() / den)
+    return worst
+
+
+def unit_rows(w, units):
+    m = np.zeros((len(w.seq_lens), w.spec.num_q_heads), bool)
+    for u in units:
+        b, kvh = divmod(u, w.spec.num_kv_heads)
+        m[b, kvh * w.spec.gqa_group:(kvh + 1) * w.spec.gqa_group] = True
+    return m
+
+
+SMALL = {
+    "tiny": W.SPECS["tiny"],
+    "llama3_8b_decode": W.shrink("llama3_8b_decode", batch=3, len_lo=2500, len_hi=5000, topk=16),
+    "long_context": W.shrink("long_context", batch=2, len_lo=6000, len_hi=9000, topk=32),
+    "high_concurrency": W.shrink("high_concurrency", batch=6, len_lo=700, len_hi=1500, topk=8),
+    "dense_limit": W.shrink("dense_limit", batch=2, len_lo=900, len_hi=1100, topk=32),
+    # shapes outside the compiled tensor-core set run the generic kernels
+    "generic_bf16": W.WorkloadSpec("generic_bf16", 2, 3, 3, 96, 24, 20, 12, 4, 300, 500, "bf16",
+                                   1 / math.sqrt(96), 0.5, False, 7),
+    "gqa8": W.shrink("llama3_8b_decode", batch=2, len_lo=3000, len_hi=4000, topk=12, gqa_group=8,
+                     num_kv_heads=4),
+    "gqa2": W.shrink("llama3_8b_decode", batch=2, len_lo=3000, len_hi=4000, topk=12, gqa_group=2),
+    "fp32_llama_shape": W.shrink("llama3_8b_decode", batch=2, len_lo=1000, len_hi=2000, topk=8,
+                                 dtype="f32"),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_parity(name):
+    w = W.generate(SMALL[name], device="cuda")
+    prob = to_problem(w)
+    ref_out, ref_sel, ref_sc, gap = oracle.decode(prob, want_scores=True)
+    out, sel = gpu_decode(w)
+    assert np.array_equal(sel, ref_sel), name
+    err = out_error(out, ref_out)
+    print(f"{name}: max row rel err {err:.3e}")
+    assert err <= OUT_TOL
+    # routing scores of every unit (routing forced even where k >= n_b)
+    sc, sel_r = gpu_scores(w)
+    _, _, full_sc, _ = oracle.decode(to_problem(w, topk=1), want_scores=True)
+    n = w.num_pages
+    for b in range(len(n)):
+        a, r = sc[b, :, :n[b]], full_sc[b, :, :n[b]]
+        assert np.all(np.abs(a - r) <= SCORE_TOL * np.maximum(1.0, np.abs(r))), name
+        assert np.all(np.isneginf(sc[b, :, n[b]:]))
+
+
+FULL = ["tiny", "llama3_8b_decode", "long_context", "high_concurrency", "dense_limit"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled(name):
+    """Full workload sizes in the benchmark's launch configuration; the oracle
+    checks a sample of units one by one, and every routed unit must pick its
+    planted pages (the unique top-k once the margin holds)."""
+    w = W.generate(name, device="cuda")
+    out, sel = gpu_decode(w)
+    s = w.spec
+    U = s.batch * s.num_kv_heads
+    rng = np.random.default_rng(123)
+    units = sorted(set([0, U - 1] + rng.choice(U, size=min(U, 4), replace=False).tolist()))
+    prob = to_problem(w)
+    ref_out, ref_sel, _, gap = oracle.decode(prob, units=units)
+    for u in units:
+        b, kvh = divmod(u, s.num_kv_heads)
+        assert np.array_equal(sel[b, kvh], ref_sel[b, kvh]), (name, u)
+        if min(s.topk, w.num_pages[b]) < w.num_pages[b]:
+            assert gap[b, kvh] >= 1e-2
+    err = out_error(out, ref_out, unit_rows(w, units))
+    print(f"{name}: sampled units {units}: max row rel err {err:.3e}")
+    assert err <= OUT_TOL
+    for (b, kvh), pages in w.planted.items():
+        got = sel[b, kvh][sel[b, kvh] >= 0]
+        assert np.array_equal(got, pages), (name, b, kvh)
+    assert np.isfinite(out).all()
+
+
+def _with_lengths(spec, lens, **kw):
+    w = W.generate(spec, device="cuda")
+    w.seq_lens = np.asarray(lens, np.int32)
+    for k, v in kw.items():
+        setattr(w, k, v)
+    return w
+
+
+def test_edge_lengths_and_mixed_routing():
+    """Empty sequence, one token, exactly one page, one page plus one token,
+    and sequences with fewer pages than k next to routed ones."""
+    spec = W.shrink("llama3_8b_decode", batch=7, len_lo=4000, len_hi=4000, topk=8)
+    w = _with_lengths(spec, [0, 1, 64, 65, 4000, 8 * 64, 8 * 64 + 1])
+    prob = to_problem(w)
+    ref_out, ref_sel, _, _ = oracle.decode(prob)
+    out, sel = gpu_decode(w)
+    assert np.array_equal(sel, ref_sel)
+    assert (sel[0] == -1).all() and (out[0] == 0).all()
+    assert out_error(out, ref_out) <= OUT_TOL
+
+
+def test_topk_one_and_max():
+    spec = W.shrink("high_concurrency", batch=3, len_lo=900, len_hi=1400, topk=1)
+    w = W.generate(spec, device="cuda")
+    for k in (1, 2, 45):
+        ref_out, ref_sel, _, _ = oracle.decode(to_problem(w, topk=k))
+        out, sel = gpu_decode(w, topk=k)
+        assert np.array_equal(sel, ref_sel), k
+        assert out_error(out, ref_out) <= OUT_TOL
+
+
+def test_exact_ties_go_to_lower_page():
+    """Logical pages sharing a physical slot score exactly the same."""
+    spec = W.shrink("llama3_8b_decode", batch=2, len_lo=64 * 40, len_hi=64 * 40, topk=6)
+    w = W.generate(spec, device="cuda")
+    pt = w.page_table.copy()
+    pt[0, :] = pt[0, 0]                              # every page identical
+    pt[1, :] = pt[1, np.arange(pt.shape[1]) % 3]     # three distinct pages, repeated
+    w.page_table = pt
+    prob = to_problem(w)
+    ref_out, ref_sel, sc, gap = oracle.decode(prob, want_scores=True)
+    assert (ref_sel[0] == np.arange(6)).all()
+    out, sel = gpu_decode(w)
+    assert np.array_equal(sel, ref_sel)
+    assert out_error(out, ref_out) <= OUT_TOL
+
+
+def test_deterministic_and_host_entry_point():
+    w = W.generate(SMALL["llama3_8b_decode"], device="cuda")
+    s = w.spec
+    kv = bk.BasisKV.for_workload(w)
+    o1, s1 = gpu_decode(w, kv=kv)
+    o2, s2 = gpu_decode(w, kv=kv)
+    assert np.array_equal(o1, o2) and np.array_equal(s1, s2)
+    qh = w.q.cpu().pin_memory()
+    oh = torch.empty((s.batch, s.num_q_heads, s.head_dim), dtype=torch.float32).pin_memory()
+    sh = torch.empty((s.batch, s.num_kv_heads, s.topk), dtype=torch.int32).pin_memory()
+    bk.basiskv_decode_attn_host(kv.handle, qh, s.topk, s.softmax_scale, oh, sh)
+    assert np.array_equal(oh.numpy(), o1) and np.array_equal(sh.numpy(), s1)
+    kv.close()
+
+
+def test_incremental_page_table_matches_bulk_load():
+    w = W.generate(SMALL["high_concurrency"], device="cuda")
+    s = w.spec
+    ref_out, ref_sel = gpu_decode(w)
+    kv = bk.BasisKV(z_pool=w.z_pool, r_pool=w.r_pool, k_pool=w.k_pool, w_zk=w.w_zk, b_r=w.b_r,
+                    b_v=w.b_v, gqa_group=s.gqa_group, max_batch=s.batch,
+                    max_pages_per_seq=w.page_table.shape[1], max_topk=s.topk)
+    P = s.page_size
+    for b, L in enumerate(w.seq_lens.tolist()):
+        n = -(-L // P)
+        for j in range(n):
+            if j == n - 1 and L - j * P < P:
+                first = max(1, (L - j * P) // 2)  # partial page: append, then grow it
+                bk.basiskv_append_page(kv.handle, b, int(w.page_table[b, j]), first)
+                if L - j * P > first:
+                    bk.basiskv_append_tokens(kv.handle, b, L - j * P - first)
+            else:
+                bk.basiskv_append_page(kv.handle, b, int(w.page_table[b, j]), P)
+    out, sel = gpu_decode(w, kv=kv)
+    assert np.array_equal(out, ref_out) and np.array_equal(sel, ref_sel)
+    partial = [b for b, L in enumerate(w.seq_lens.tolist()) if L % P]
+    assert partial, "the workload should have a sequence ending in a partial page"
+    with pytest.raises(bk.BasisKVError) as e:
+        bk.basiskv_append_page(kv.handle, partial[0], 0, 1)
+    assert e.value.code == bk.BASISKV_ERR_STATE
+    bk.basiskv_reset_seq(kv.handle, 0)
+    out2, sel2 = gpu_decode(w, kv=kv)
+    assert (sel2[0] == -1).all() and (out2[0] == 0).all()
+    assert np.array_equal(out2[1:], ref_out[1:]) and np.array_equal(sel2[1:], ref_sel[1:])
+    kv.close()
+
+
+def test_invalid_calls_rejected():
+    w = W.generate(SMALL["tiny"], device="cuda")
+    kv = bk.BasisKV.for_workload(w)
+    out = torch.empty((1, 4, 64), device="cuda")
+    for topk in (0, -1, w.spec.topk + 1):
+        with pytest.raises(bk.BasisKVError) as e:
+            bk.basiskv_decode_attn(kv.handle, w.q, topk, 0.1, out)
+        assert e.value.code == bk.BASISKV_ERR_INVALID_ARG
+    with pytest.raises(bk.BasisKVError):
+        bk.basiskv_load_page_table(kv.handle, np.full((1, 64), 10 ** 6), np.array([1024]))
+    kv.close()
