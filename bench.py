@@ -35,10 +35,12 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama3_8b_decode")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (smaller profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     return ap.parse_args()
@@ -102,7 +104,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -261,6 +263,8 @@ def run_ours(args, rank, world, local):
     init_dist(world, "nccl")
     build.build()
     spec = W.SPECS[args.workload]
+    if args.batch:
+        spec = spec.with_(batch=args.batch)
     if rank:
         spec = spec.with_(seed=spec.seed + 1000 * rank)
     w = W.generate(spec, device=dev)
@@ -284,6 +288,7 @@ def run_ours(args, rank, world, local):
 
     K = args.steps
     with ClockSampler(local) as clk:
+        time.sleep(0.3)  # let the sampler start before the timed loop
         barrier(world, dev)
         torch.cuda.synchronize(dev)
         bk.basiskv_profile_begin(kv.handle, K)
@@ -347,7 +352,8 @@ def run_ours(args, rank, world, local):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_step_max, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": s.dtype, "data": "synthetic",
-            "config": {"workload": args.workload, "batch": s.batch, "kv_heads": s.num_kv_heads,
+            "config": {"workload": args.workload if not args.batch else f"{args.workload}[batch={s.batch}]",
+                       "batch": s.batch, "kv_heads": s.num_kv_heads,
                        "q_heads": s.num_q_heads, "head_dim": s.head_dim, "page": s.page_size,
                        "rank_r": s.rank_r, "rank_s": s.rank_s, "topk": s.topk,
                        "context_tokens": tokens, "algorithmic_bytes": nbytes["total"],

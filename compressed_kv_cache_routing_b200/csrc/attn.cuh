@@ -32,6 +32,11 @@ struct AttnArgs {
   int ld_pt, ld_sel, num_slots, num_kv_heads, head_dim, page_size, rank_r, gqa_group;
   int topk, pages_per_split, stages, np_cap;
   float scale_log2;          // softmax_scale * log2(e)
+  // persistent tensor-core kernel only
+  int batch;
+  const int32_t* attn_off;   // [B+1] prefix of attention items x Hkv (from the prep grid)
+  int plan_n;                // >= 0: plan_off holds attn_off (batch <= kPlanMax)
+  int32_t plan_off[kPlanMax + 1];
 };
 
 constexpr int kAttnThreads = 128;
@@ -101,7 +106,9 @@ __device__ __forceinline__ void attn_finish(const AttnArgs& a, const AttnUnit& a
 }
 
 // ---------------------------------------------------------------------------
-// Tensor-core attention for bf16 pools.
+// Tensor-core attention for bf16 pools, persistent over the flat list of
+// attention items (sequence-major, then KV head, selected entry, stage of
+// the page); every warp streams one contiguous share of it.
 //
 // QK: S(16 x 8 tokens) = Qg(16 x d) . K^T, rows 0..G-1 of Qg hold the group's
 // queries (rows G..15 zero), K rows come from shared memory; the k index is
@@ -114,9 +121,66 @@ __device__ __forceinline__ void attn_finish(const AttnArgs& a, const AttnUnit& a
 // acc[g] + acc[g+8] is the latent sum with ~16-bit weights; Z fragments come
 // from ldmatrix.trans.
 // Each stage carries TPS tokens of one selected page (K then Z), staged by
-// bulk copies into a per-warp ring.
+// bulk copies into a per-warp ring.  At the end of its segment of a unit a
+// warp writes one partial (m, l, acc); the warp that completes the unit
+// merges the partials and applies B_v.
+struct AttnCursor {
+  int b, kvh, jj, ts, n, kb, L;
+  int uoff;            // flat index of the unit's first item
+  const int32_t* off;  // prefix of attention items x Hkv over sequences
+  __device__ __forceinline__ void load(const AttnArgs& a) {
+    L = a.seq_lens[b];
+    n = (L + a.page_size - 1) / a.page_size;
+    kb = min(a.topk, n);
+    uoff = off[b];
+  }
+  __device__ void seek(const AttnArgs& a, const int32_t* offsets, int f, int sub) {
+    off = offsets;
+    int lo = 0, hi = a.batch;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (off[mid] <= f) lo = mid + 1;
+      else hi = mid;
+    }
+    b = lo - 1;
+    load(a);
+    const int per_unit = kb * sub;
+    const int rel = f - uoff;
+    kvh = rel / per_unit;
+    const int r2 = rel % per_unit;
+    jj = r2 / sub;
+    ts = r2 % sub;
+    uoff += kvh * per_unit;
+  }
+  __device__ __forceinline__ void advance(const AttnArgs& a, int sub) {
+    if (++ts < sub) return;
+    ts = 0;
+    if (++jj < kb) return;
+    jj = 0;
+    if (++kvh < a.num_kv_heads) {
+      uoff += kb * sub;
+      return;
+    }
+    kvh = 0;
+    for (++b; b < a.batch; ++b) {
+      load(a);
+      if (kb > 0) return;
+    }
+  }
+  __device__ __forceinline__ int unit(const AttnArgs& a) const { return b * a.num_kv_heads + kvh; }
+  __device__ __forceinline__ int page(const AttnArgs& a) const {
+    if (a.topk >= n) return jj;
+    int p = __ldcg(a.sel + (size_t)unit(a) * a.ld_sel + jj);
+    if (p < 0 || p >= n) {
+      atomicOr(a.status, kStatusBadPage);
+      p = 0;
+    }
+    return p;
+  }
+};
+
 template <int G, int D, int RR, int TPS>
-__global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_constant__ AttnArgs a) {
   static_assert(G >= 1 && G <= 8, "GQA group must be 1..8");
   static_assert(D % 32 == 0 && RR % 8 == 0 && TPS % 16 == 0, "shape");
   constexpr int DS = D / 32;     // 32-wide spans of the head dim
@@ -126,24 +190,38 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const AttnArgs a
   constexpr uint32_t kbytes = TPS * D * 2, zbytes = TPS * RR * 2;
   constexpr uint32_t stage_bytes = kbytes + zbytes;
 
-  const AttnUnit au = attn_unit(a);
   const int P = a.page_size, S = a.stages;
+  const int sub = P / TPS;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
-  const int sub = P / TPS;
-  const int items = max(0, au.j1 - au.j0) * sub;
-  const int mine = items > warp ? (items - warp + kAttnWarps - 1) / kAttnWarps : 0;
 
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t bars[kAttnWarps][8];
-  __shared__ int flag;
+  __shared__ int tok0s[kAttnWarps][8];
   uint8_t* ring = smem + (size_t)warp * S * stage_bytes;
+  float* zbar = reinterpret_cast<float*>(smem + (size_t)kAttnWarps * S * stage_bytes) + warp * G * RR;
+  if (lane == 0) {
+    for (int i = 0; i < S; ++i) mbar_init(&bars[warp][i], 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
 
-  // query fragments (A operand), rows >= G are zero
+  // the plan comes in the parameters, or from the prep grid, which finished
+  // before the routing grid let this one launch
+  const int32_t* offsets = a.plan_n >= 0 ? a.plan_off : a.attn_off;
+  const long long W = (long long)gridDim.x * kAttnWarps;
+  const int wg = blockIdx.x * kAttnWarps + warp;
+  const long long T = offsets[a.batch];
+  const int f0 = (int)(T * wg / W), f1 = (int)(T * (wg + 1) / W);
+  const int count = f1 - f0;
+  AttnCursor ic;
+  if (count > 0) ic.seek(a, offsets, f0, sub);
+  (void)f1;
+  AttnCursor cc = ic;
+
   uint32_t qa[DS][2][2];
-  {
-    const __nv_bfloat16* qrow =
-        static_cast<const __nv_bfloat16*>(a.q) + ((size_t)au.u * G + (g < G ? g : 0)) * D;
+  auto load_q = [&](int u) {
+    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)u * G + (g < G ? g : 0)) * D;
 #pragma unroll
     for (int s = 0; s < DS; ++s) {
       uint4 v = make_uint4(0, 0, 0, 0);
@@ -153,45 +231,144 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const AttnArgs a
       qa[s][1][0] = v.z;
       qa[s][1][1] = v.w;
     }
+  };
+  int cur_u = -1;
+  if (count > 0) {
+    cur_u = cc.unit(a);
+    load_q(cur_u);
   }
-  if (lane == 0) {
-    for (int i = 0; i < S; ++i) mbar_init(&bars[warp][i], 1);
-    mbar_init_fence();
-  }
-  __syncwarp();
   pdl_wait_primary();  // the selection is written by the routing grid
+  if (count <= 0) return;
 
   const __nv_bfloat16* kpool = static_cast<const __nv_bfloat16*>(a.k_pool);
   const __nv_bfloat16* zpool = static_cast<const __nv_bfloat16*>(a.z_pool);
   const uint64_t pol = policy_evict_first();
-  auto issue = [&](int i) {  // lane 0: my i-th item into stage i % S
-    const int item = warp + i * kAttnWarps;
-    const int page = selected_page(a, au, au.j0 + item / sub);
-    const int slot = page_slot(a, au, page);
-    const size_t row0 = ((size_t)slot * a.num_kv_heads + au.kvh) * P + (size_t)(item % sub) * TPS;
+  // lane 0 issues item i of this warp into stage i % S; the selection and
+  // page-table reads for an item are made one iteration before its issue so
+  // they overlap the arithmetic of the current stage
+  auto slot_of = [&](int page) { return __ldg(a.page_table + (size_t)ic.b * a.ld_pt + page); };
+  auto issue = [&](int i, int page, int slot) {
+    if (slot < 0 || slot >= a.num_slots) {
+      atomicOr(a.status, kStatusBadSlot);
+      slot = 0;
+    }
+    const size_t row0 = ((size_t)slot * a.num_kv_heads + ic.kvh) * P + (size_t)ic.ts * TPS;
+    tok0s[warp][i % S] = page * P + ic.ts * TPS;
     uint64_t* bar = &bars[warp][i % S];
     uint8_t* dst = ring + (size_t)(i % S) * stage_bytes;
     mbar_arrive_expect_tx(bar, stage_bytes);
     bulk_load(dst, kpool + row0 * D, kbytes, bar, pol);
     bulk_load(dst + kbytes, zpool + row0 * RR, zbytes, bar, pol);
+    ic.advance(a, sub);
   };
-  if (lane == 0)
-    for (int i = 0; i < S && i < mine; ++i) issue(i);
+  AttnCursor ia;       // lane 0: the item after the next one to issue
+  int next_page = 0;   // lane 0: page of the next item to issue
+  {
+    // the first S items: lane j looks item j up (all lookups in parallel),
+    // lane 0 issues them in order
+    const int first = min(S, count);
+    int pg = 0, sl = 0;
+    if (lane < first) {
+      AttnCursor c = ic;
+      for (int k = 0; k < lane; ++k) c.advance(a, sub);
+      pg = c.page(a);
+      sl = __ldg(a.page_table + (size_t)c.b * a.ld_pt + pg);
+    }
+    for (int i = 0; i < first; ++i) {
+      const int pgi = __shfl_sync(0xffffffffu, pg, i), sli = __shfl_sync(0xffffffffu, sl, i);
+      if (lane == 0) issue(i, pgi, sli);
+    }
+  }
+  if (lane == 0) {
+    if (S < count) {
+      next_page = ic.page(a);
+      ia = ic;
+      ia.advance(a, sub);
+    }
+  }
 
   float m_run = -INFINITY, l_run = 0.f;
   float acc[RT][4];
 #pragma unroll
   for (int c = 0; c < RT; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.f;
+  int seg = 0;
+  AttnCursor prev = cc;
+
+  // end of this warp's segment of unit u: write its partial, count the
+  // items; the warp completing the unit merges everything and applies B_v
+  // Warp w streams items [floor(T*w/W), floor(T*(w+1)/W)); the warp holding
+  // item o is ceil((o+1)*W/T) - 1.  A unit's partial slot is the warp's rank
+  // among the warps holding its items, so the merge order never changes.
+  auto owner = [&](long long o) { return (int)(((o + 1) * W + T - 1) / T) - 1; };
+  // end of this warp's segment of unit u: write its partial, count the
+  // items; the warp completing the unit merges everything and applies B_v
+  auto flush = [&](const AttnCursor& at) {
+    const int u = cur_u;
+    float l = l_run;
+    l += __shfl_xor_sync(0xffffffffu, l, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    const int items = at.kb * sub;
+    const int w_first = owner(at.uoff);
+    const int np = owner((long long)at.uoff + items - 1) - w_first + 1;
+    const int slot = wg - w_first;
+    if (slot < a.np_cap) {
+      if (g < G) {
+        const size_t part = ((size_t)u * a.np_cap + slot) * G + g;
+        if (t == 0) {
+          a.part_ml[part * 2] = m_run;
+          a.part_ml[part * 2 + 1] = l;
+        }
+        float* pa = a.part_acc + part * RR;
+#pragma unroll
+        for (int c = 0; c < RT; ++c) {
+          pa[8 * c + 2 * t] = acc[c][0] + acc[c][2];
+          pa[8 * c + 2 * t + 1] = acc[c][1] + acc[c][3];
+        }
+      }
+    } else if (lane == 0) {
+      atomicOr(a.status, kStatusTimeout);  // more partials than slots: result invalid
+    }
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+      __threadfence();
+      const uint32_t prevc = atomicAdd(a.counters + u, (uint32_t)seg);
+      last = prevc + seg == (uint32_t)items;
+      __threadfence();
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) {
+      warp_combine<G, RR, D>(a.part_ml + (size_t)u * a.np_cap * G * 2,
+                             a.part_acc + (size_t)u * a.np_cap * G * RR, min(np, a.np_cap),
+                             a.b_v + (size_t)at.kvh * RR * D, a.out + (size_t)u * G * D, zbar);
+      if (lane == 0) a.counters[u] = 0u;
+    }
+  };
 
   bool ok = true;
   int i = 0;
-  for (; i < mine; ++i) {
+  const int trow = (lane & 7) + 8 * ((lane >> 3) & 1);
+  for (; i < count; ++i) {
+    int next_slot = 0, page_after = 0;
+    if (lane == 0) {
+      if (i + S < count) next_slot = slot_of(next_page);
+      if (i + S + 1 < count) page_after = ia.page(a);
+    }
+    const int u = cc.unit(a);
+    if (u != cur_u) {
+      flush(prev);
+      cur_u = u;
+      seg = 0;
+      m_run = -INFINITY;
+      l_run = 0.f;
+#pragma unroll
+      for (int c = 0; c < RT; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.f;
+      load_q(u);
+    }
     ok = mbar_wait(&bars[warp][i % S], (uint32_t)((i / S) & 1), a.status);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;
-    const int item = warp + i * kAttnWarps;
-    const int page = selected_page(a, au, au.j0 + item / sub);
-    const int valid = au.L - (page * P + (item % sub) * TPS);  // tokens of this stage in range
+    const int valid = cc.L - tok0s[warp][i % S];  // tokens of this stage inside the sequence
     const __nv_bfloat16* ks = reinterpret_cast<const __nv_bfloat16*>(ring + (size_t)(i % S) * stage_bytes);
     const __nv_bfloat16* zs = ks + TPS * D;
 
@@ -237,7 +414,6 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const AttnArgs a
       acc[c][3] *= corr;
     }
     // latent sum P.Z
-    const int trow = (lane & 7) + 8 * ((lane >> 3) & 1);
 #pragma unroll
     for (int kb = 0; kb < KBS; ++kb) {
       float h0, l0, h1, l1, h2, l2, h3, l3;
@@ -261,36 +437,29 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const AttnArgs a
         mma_k16(acc[RT - 1], a0, a1, a2, a3, b0, b1);
       }
     }
+    ++seg;
     __syncwarp();
-    if (lane == 0 && i + S < mine) issue(i + S);
-  }
-  if (!ok && lane == 0)
-    for (int j = i; j < mine && j < i + S; ++j)
-      mbar_wait(&bars[warp][j % S], (uint32_t)((j / S) & 1), a.status);
-
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-  if (g < G) {
-    const size_t part = ((size_t)au.u * a.np_cap + blockIdx.x * kAttnWarps + warp) * G + g;
-    if (t == 0) {
-      a.part_ml[part * 2] = m_run;
-      a.part_ml[part * 2 + 1] = l_run;
+    if (lane == 0 && i + S < count) {
+      issue(i + S, next_page, next_slot);
+      next_page = page_after;
+      ia.advance(a, sub);
     }
-    float* pa = a.part_acc + part * RR;
-#pragma unroll
-    for (int c = 0; c < RT; ++c) {
-      pa[8 * c + 2 * t] = acc[c][0] + acc[c][2];
-      pa[8 * c + 2 * t + 1] = acc[c][1] + acc[c][3];
-    }
+    prev = cc;
+    cc.advance(a, sub);
   }
-  write_identity_selection(a, au);
-  attn_finish<kAttnThreads>(a, au, kAttnWarps, reinterpret_cast<float*>(smem), &flag);
+  if (!ok) {
+    if (lane == 0)
+      for (int j = i; j < count && j < i + S; ++j)
+        mbar_wait(&bars[warp][j % S], (uint32_t)((j / S) & 1), a.status);
+    return;
+  }
+  flush(prev);
 }
 
 // ---------------------------------------------------------------------------
 // CUDA-core attention for any shape and for fp32 pools: one partial per CTA.
 template <typename T>
-__global__ void __launch_bounds__(kAttnThreads) attn_generic_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(kAttnThreads) attn_generic_kernel(const __grid_constant__ AttnArgs a) {
   const AttnUnit au = attn_unit(a);
   const int G = a.gqa_group, D = a.head_dim, RR = a.rank_r, P = a.page_size;
   extern __shared__ __align__(128) uint8_t smem[];

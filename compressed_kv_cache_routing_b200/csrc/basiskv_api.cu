@@ -14,6 +14,7 @@
 
 #include "../../include/basiskv.h"
 #include "attn.cuh"
+#include "plan.cuh"
 #include "route.cuh"
 
 using namespace basiskv;
@@ -40,16 +41,18 @@ int fail(int code, const char* fmt, ...) {
 
 constexpr int kMaxSplits = 16;
 constexpr int kPartsCap = kMaxSplits * kAttnWarps;  // partials per unit
-constexpr size_t kRouteSmemBudget = 96 * 1024;       // ring bytes per routing CTA
-constexpr size_t kAttnSmemBudget = 200 * 1024;       // ring bytes per attention CTA
+// Ring bytes per CTA: small rings let several CTAs (and so many warps, each
+// with copies in flight) share an SM.
+constexpr size_t kRouteSmemBudget = 48 * 1024;
+constexpr size_t kAttnSmemBudget = 100 * 1024;
 
 using KernelFn = void (*)(const RouteArgs);
 using AttnFn = void (*)(const AttnArgs);
 
 // ---- compiled tensor-core shapes ------------------------------------------
 struct RouteKey {
-  int g, r, s;
-  bool operator<(const RouteKey& o) const { return std::tie(g, r, s) < std::tie(o.g, o.r, o.s); }
+  int g, r, s, p;
+  bool operator<(const RouteKey& o) const { return std::tie(g, r, s, p) < std::tie(o.g, o.r, o.s, o.p); }
 };
 struct AttnKey {
   int g, d, r, tps;
@@ -60,10 +63,13 @@ struct AttnKey {
 
 const std::map<RouteKey, KernelFn>& route_table() {
   static const std::map<RouteKey, KernelFn> t = {
-#define RK(G, R, S) {RouteKey{G, R, S}, &route_mma_kernel<G, R, S>}
-      RK(4, 16, 8),  RK(4, 24, 8),  RK(4, 32, 8),  RK(4, 32, 16), RK(4, 64, 16),
-      RK(4, 64, 32), RK(4, 128, 0), RK(4, 32, 0),  RK(8, 32, 16), RK(8, 24, 8),
-      RK(8, 64, 32), RK(2, 32, 16), RK(1, 32, 16),
+#define RK(G, R, S, P) {RouteKey{G, R, S, P}, &route_mma_kernel<G, R, S, P>}
+#define RK2(G, R, S) RK(G, R, S, 32), RK(G, R, S, 64)
+      RK2(4, 16, 8),  RK2(4, 24, 8),  RK2(4, 32, 8),  RK2(4, 32, 16), RK2(4, 64, 16),
+      RK2(4, 64, 32), RK2(4, 128, 0), RK2(4, 32, 0),  RK2(8, 32, 16), RK2(8, 24, 8),
+      RK2(8, 64, 32), RK2(2, 32, 16), RK2(1, 32, 16), RK(4, 32, 16, 16), RK(4, 32, 16, 128),
+      RK(4, 24, 8, 16),
+#undef RK2
 #undef RK
   };
   return t;
@@ -97,8 +103,12 @@ struct basiskv_handle {
   int32_t* d_sel = nullptr;         // [max_batch][Hkv][max_topk]
   float* d_part_ml = nullptr;       // [max_batch*Hkv][kPartsCap][G][2]
   float* d_part_acc = nullptr;      // [max_batch*Hkv][kPartsCap][G][r]
-  uint32_t* d_counters = nullptr;   // [2][max_batch*Hkv]
+  uint32_t* d_counters = nullptr;   // [3][max_batch*Hkv]: route, attention, partial count
   uint32_t* d_status = nullptr;
+  int32_t* d_route_off = nullptr;   // [max_batch+1]
+  int32_t* d_attn_off = nullptr;    // [max_batch+1]
+  uint32_t* d_qfrag = nullptr;      // [max_batch*Hkv][frag_words][32]
+  int frag_words = 0;
   // host-buffer entry point staging
   void* d_q_stage = nullptr;
   float* d_out_stage = nullptr;
@@ -112,7 +122,9 @@ struct basiskv_handle {
   AttnFn attn_fn = nullptr;
   int attn_tps = 0;
   int route_stages = 0, attn_stages = 0;
-  size_t route_smem = 0, attn_smem = 0;
+  size_t route_smem = 0, attn_smem = 0, prep_smem = 0;
+  int topk_keys = 0;  // scores staged in shared memory by the selection kernel
+  int route_occ = 1, attn_occ = 1;  // resident CTAs per SM of the persistent kernels
   // profiling
   std::vector<cudaEvent_t> events;  // 3 per recorded call
   int prof_cap = 0, prof_calls = 0;
@@ -148,8 +160,9 @@ int validate_params(const basiskv_params* p) {
     if (!aligned16(q)) return fail(BASISKV_ERR_INVALID_ARG, "pools and bases must be 16-byte aligned");
   if (p->rank_s > 0 && (!aligned16(p->r_pool) || !aligned16(p->b_r)))
     return fail(BASISKV_ERR_INVALID_ARG, "pools and bases must be 16-byte aligned");
-  if ((size_t)p->max_batch * p->max_pages_per_seq > (size_t)1 << 31)
-    return fail(BASISKV_ERR_INVALID_ARG, "page table too large");
+  if ((size_t)p->max_batch * p->max_pages_per_seq * p->num_kv_heads * (p->page_size / 16 + 1) >=
+      ((size_t)1 << 31))
+    return fail(BASISKV_ERR_INVALID_ARG, "page table too large (work lists must index in 32 bits)");
   return BASISKV_OK;
 }
 
@@ -158,15 +171,14 @@ void choose_kernels(basiskv_handle* h) {
   const basiskv_params& p = h->p;
   if (p.dtype != BASISKV_DTYPE_BF16) return;
   const size_t es = 2;
-  auto rit = route_table().find(RouteKey{p.gqa_group, p.rank_r, p.rank_s});
+  auto rit = route_table().find(RouteKey{p.gqa_group, p.rank_r, p.rank_s, p.page_size});
   if (rit != route_table().end() && p.page_size % 16 == 0 && p.head_dim % 32 == 0) {
     const size_t stage = (size_t)p.page_size * (p.rank_r + p.rank_s) * es;
-    int st = (int)std::min<size_t>(kMaxStages, kRouteSmemBudget / (kRouteWarps * stage));
+    int st = (int)std::min<size_t>(4, kRouteSmemBudget / (kRouteWarps * stage));
     if (st >= 2) {
       h->route_fn = rit->second;
       h->route_stages = st;
-      h->route_smem = kRouteWarps * st * stage +
-                      sizeof(float) * (size_t)p.gqa_group * (p.head_dim + p.rank_r + p.rank_s);
+      h->route_smem = kRouteWarps * st * stage;
     }
   }
   for (int tps : {64, 32, 16}) {
@@ -180,8 +192,7 @@ void choose_kernels(basiskv_handle* h) {
     h->attn_fn = ait->second;
     h->attn_tps = tps;
     h->attn_stages = st;
-    h->attn_smem = std::max(kAttnWarps * st * stage,
-                            sizeof(float) * combine_smem_floats(kPartsCap, p.gqa_group, p.rank_r));
+    h->attn_smem = kAttnWarps * st * stage + sizeof(float) * kAttnWarps * p.gqa_group * p.rank_r;
     break;
   }
 }
@@ -210,15 +221,25 @@ int set_generic_attrs(const basiskv_params& p) {
 struct LaunchPlan {
   int batch = 0;
   bool any_routed = false;
+  long long route_pages = 0;  // routed pages x Hkv (persistent routing work list)
+  long long attn_items = 0;   // selected pages x stages x Hkv (persistent attention work list)
+  int max_unit_items = 0;
+  int sub = 1;                // attention stages per page
+  // generic kernels
   int route_ppc = 0, route_chunks = 0;
   int attn_pps = 0, attn_splits = 0;
+  // persistent kernels
+  int route_ctas = 0, attn_ctas = 0;
+  // work plans (prefix over sequences), when batch <= kPlanMax
+  std::vector<int32_t> route_off, attn_off;
 };
 
 LaunchPlan plan(const basiskv_handle* h, int batch, int topk, bool force_route) {
   LaunchPlan lp;
   lp.batch = batch;
   const basiskv_params& p = h->p;
-  long long route_pages = 0;
+  lp.sub = h->attn_fn ? p.page_size / h->attn_tps : 1;
+  long long route_pages = 0, items = 0;
   int max_routed = 0, max_kb = 0;
   for (int b = 0; b < batch; ++b) {
     const int n = h->h_npages[b];
@@ -226,16 +247,32 @@ LaunchPlan plan(const basiskv_handle* h, int batch, int topk, bool force_route) 
       route_pages += n;
       max_routed = std::max(max_routed, n);
     }
-    max_kb = std::max(max_kb, std::min(topk, n));
+    const int kb = std::min(topk, n);
+    max_kb = std::max(max_kb, kb);
+    items += (long long)kb * lp.sub;
   }
-  route_pages *= p.num_kv_heads;
+  lp.route_pages = route_pages * p.num_kv_heads;
+  lp.attn_items = items * p.num_kv_heads;
+  if (batch <= kPlanMax) {
+    lp.route_off.assign(batch + 1, 0);
+    lp.attn_off.assign(batch + 1, 0);
+    for (int b = 0; b < batch; ++b) {
+      const int n = h->h_npages[b];
+      const bool routed = n > 0 && (force_route || topk < n);
+      lp.route_off[b + 1] = lp.route_off[b] + (routed ? n : 0) * p.num_kv_heads;
+      lp.attn_off[b + 1] = lp.attn_off[b] + std::min(topk, n) * lp.sub * p.num_kv_heads;
+    }
+  }
+  lp.max_unit_items = max_kb * lp.sub;
   lp.any_routed = max_routed > 0;
+
+  // generic kernels: a grid of (chunk | split, Hkv, batch)
   if (lp.any_routed) {
-    const long long target = (long long)h->num_sms * 8;  // about four waves of two CTAs
-    long long ppc = (route_pages + target - 1) / target;
+    const long long target = (long long)h->num_sms * 8;
+    long long ppc = (lp.route_pages + target - 1) / target;
     ppc = std::max<long long>(kRouteWarps * 2, std::min<long long>(ppc, 512));
     const int chunks = (int)((max_routed + ppc - 1) / ppc);
-    lp.route_ppc = (max_routed + chunks - 1) / chunks;  // even chunks for the longest sequence
+    lp.route_ppc = (max_routed + chunks - 1) / chunks;
     lp.route_chunks = (max_routed + lp.route_ppc - 1) / lp.route_ppc;
   }
   const long long units = (long long)batch * p.num_kv_heads;
@@ -244,11 +281,62 @@ LaunchPlan plan(const basiskv_handle* h, int batch, int topk, bool force_route) 
   splits = std::max(1, std::min(splits, std::max(1, max_kb)));
   lp.attn_pps = std::max(1, (max_kb + splits - 1) / splits);
   lp.attn_splits = std::max(1, (max_kb + lp.attn_pps - 1) / lp.attn_pps);
+
+  // persistent kernels: every warp streams an equal contiguous share
+  const long long min_per_warp = 4;
+  lp.route_ctas = (int)std::max<long long>(1, std::min<long long>(
+      (long long)h->num_sms * h->route_occ, (lp.route_pages + kRouteWarps * min_per_warp - 1) /
+                                                (kRouteWarps * min_per_warp)));
+  long long attn_warps = std::min<long long>((long long)h->num_sms * h->attn_occ * kAttnWarps,
+                                             std::max<long long>(1, lp.attn_items));
+  if (lp.max_unit_items > 0) {
+    // a unit must meet at most kPartsCap - 2 warps: each warp gets at least
+    // ceil(max_unit_items / (kPartsCap - 2)) items
+    const long long per = (lp.max_unit_items + kPartsCap - 3) / (kPartsCap - 2);
+    attn_warps = std::min<long long>(attn_warps, std::max<long long>(1, lp.attn_items / per));
+  }
+  lp.attn_ctas = (int)std::max<long long>(1, (attn_warps + kAttnWarps - 1) / kAttnWarps);
   return lp;
 }
 
-RouteArgs route_args(basiskv_handle* h, int batch, const void* q, int topk, float* scores,
-                     int32_t* sel_out, int force, int ppc, int stages) {
+int launch_prep(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk, int force, float* out,
+                int32_t* sel_out, float* fill_scores, cudaStream_t stream) {
+  const basiskv_params& p = h->p;
+  PrepArgs a;
+  a.q = q;
+  a.w_zk = p.w_zk;
+  a.b_r = p.b_r;
+  a.seq_lens = h->d_seq_lens;
+  a.route_off = h->d_route_off;
+  a.attn_off = h->d_attn_off;
+  a.qfrag = h->d_qfrag;
+  a.sel_out = sel_out;
+  a.out = out;
+  a.scores = fill_scores;
+  a.batch = lp.batch;
+  a.num_kv_heads = p.num_kv_heads;
+  a.gqa_group = p.gqa_group;
+  a.head_dim = p.head_dim;
+  a.page_size = p.page_size;
+  a.rank_r = p.rank_r;
+  a.rank_s = p.rank_s;
+  a.topk = topk;
+  a.force = force;
+  a.attn_sub = lp.sub;
+  a.ld_pt = p.max_pages_per_seq;
+  a.fr = h->frag_words;
+  a.fill_scores = fill_scores != nullptr;
+  dim3 grid(p.num_kv_heads, lp.batch);
+  if (p.dtype == BASISKV_DTYPE_BF16)
+    prep_kernel<__nv_bfloat16><<<grid, kPrepThreads, h->prep_smem, stream>>>(a);
+  else
+    prep_kernel<float><<<grid, kPrepThreads, h->prep_smem, stream>>>(a);
+  CUDA_TRY(cudaGetLastError());
+  return BASISKV_OK;
+}
+
+RouteArgs route_args(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk, float* scores,
+                     int32_t* sel_out, int force) {
   const basiskv_params& p = h->p;
   RouteArgs a;
   a.q = q;
@@ -273,33 +361,79 @@ RouteArgs route_args(basiskv_handle* h, int batch, const void* q, int topk, floa
   a.rank_s = p.rank_s;
   a.gqa_group = p.gqa_group;
   a.topk = topk;
-  a.pages_per_cta = ppc;
-  a.stages = stages;
+  a.pages_per_cta = lp.route_ppc;
+  a.stages = h->route_stages;
   a.force = force;
   a.fill_tail = force;
-  (void)batch;
+  a.batch = lp.batch;
+  a.route_off = h->d_route_off;
+  a.qfrag = h->d_qfrag;
+  a.frag_words = h->frag_words;
+  a.plan_n = lp.route_off.empty() ? -1 : lp.batch;
+  for (size_t i = 0; i < lp.route_off.size(); ++i) a.plan_off[i] = lp.route_off[i];
   return a;
 }
 
-int launch_route(basiskv_handle* h, const LaunchPlan& lp, const RouteArgs& a, cudaStream_t stream) {
+cudaLaunchConfig_t launch_cfg(dim3 grid, int threads, size_t smem, cudaStream_t stream, bool pdl,
+                              cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cfg;
+}
+
+// Routing after the prep grid: the persistent tensor-core kernel (PDL: it
+// waits for the prep grid before reading the plan), else the generic one.
+int launch_route(basiskv_handle* h, const LaunchPlan& lp, const RouteArgs& a, bool pdl, cudaStream_t stream) {
   const basiskv_params& p = h->p;
-  dim3 grid(lp.route_chunks, p.num_kv_heads, lp.batch);
+  cudaLaunchAttribute attr[1];
   if (h->route_fn) {
-    RouteArgs ra = a;
-    ra.stages = h->route_stages;
-    h->route_fn<<<grid, kRouteThreads, h->route_smem, stream>>>(ra);
-  } else if (p.dtype == BASISKV_DTYPE_BF16) {
-    route_generic_kernel<__nv_bfloat16><<<grid, kRouteThreads, generic_route_smem(p), stream>>>(a);
-  } else {
-    route_generic_kernel<float><<<grid, kRouteThreads, generic_route_smem(p), stream>>>(a);
+    cudaLaunchConfig_t cfg = launch_cfg(dim3(lp.route_ctas), kRouteThreads, h->route_smem, stream, pdl, attr);
+    CUDA_TRY(cudaLaunchKernelEx(&cfg, h->route_fn, a));
+    return BASISKV_OK;
   }
+  dim3 grid(lp.route_chunks, p.num_kv_heads, lp.batch);
+  if (p.dtype == BASISKV_DTYPE_BF16)
+    route_generic_kernel<__nv_bfloat16><<<grid, kRouteThreads, generic_route_smem(p), stream>>>(a);
+  else
+    route_generic_kernel<float><<<grid, kRouteThreads, generic_route_smem(p), stream>>>(a);
   CUDA_TRY(cudaGetLastError());
+  return BASISKV_OK;
+}
+
+// Selection for the persistent routing kernel (PDL behind it).
+int launch_topk(basiskv_handle* h, const LaunchPlan& lp, int topk, const float* scores, int32_t* sel_out,
+                int force, bool pdl, cudaStream_t stream) {
+  const basiskv_params& p = h->p;
+  TopkArgs a;
+  a.scores = scores;
+  a.seq_lens = h->d_seq_lens;
+  a.sel = h->d_sel;
+  a.sel_out = sel_out;
+  a.num_kv_heads = p.num_kv_heads;
+  a.page_size = p.page_size;
+  a.ld_pt = p.max_pages_per_seq;
+  a.ld_sel = p.max_topk;
+  a.topk = topk;
+  a.force = force;
+  a.keys_cap = h->topk_keys;
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = launch_cfg(dim3(p.num_kv_heads, lp.batch), kTopkThreads,
+                                      sizeof(uint32_t) * (size_t)h->topk_keys, stream, pdl, attr);
+  CUDA_TRY(cudaLaunchKernelEx(&cfg, &topk_kernel, a));
   return BASISKV_OK;
 }
 
 int launch_attn(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk, float scale,
                 float* out, int32_t* sel_out, bool pdl, cudaStream_t stream) {
   const basiskv_params& p = h->p;
+  const size_t U = (size_t)p.max_batch * p.num_kv_heads;
   AttnArgs a;
   a.q = q;
   a.k_pool = p.k_pool;
@@ -311,7 +445,7 @@ int launch_attn(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk
   a.sel_out = sel_out;
   a.part_ml = h->d_part_ml;
   a.part_acc = h->d_part_acc;
-  a.counters = h->d_counters + (size_t)p.max_batch * p.num_kv_heads;
+  a.counters = h->d_counters + U;
   a.status = h->d_status;
   a.out = out;
   a.ld_pt = p.max_pages_per_seq;
@@ -327,26 +461,23 @@ int launch_attn(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk
   a.stages = h->attn_stages;
   a.np_cap = kPartsCap;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.batch = lp.batch;
+  a.attn_off = h->d_attn_off;
+  a.plan_n = lp.attn_off.empty() ? -1 : lp.batch;
+  for (size_t i = 0; i < lp.attn_off.size(); ++i) a.plan_off[i] = lp.attn_off[i];
 
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(lp.attn_splits, p.num_kv_heads, lp.batch);
-  cfg.blockDim = dim3(kAttnThreads);
-  cfg.stream = stream;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
   if (h->attn_fn) {
-    cfg.dynamicSmemBytes = h->attn_smem;
+    cudaLaunchConfig_t cfg = launch_cfg(dim3(lp.attn_ctas), kAttnThreads, h->attn_smem, stream, pdl, attr);
     CUDA_TRY(cudaLaunchKernelEx(&cfg, h->attn_fn, a));
-  } else if (p.dtype == BASISKV_DTYPE_BF16) {
-    cfg.dynamicSmemBytes = generic_attn_smem(p);
-    CUDA_TRY(cudaLaunchKernelEx(&cfg, &attn_generic_kernel<__nv_bfloat16>, a));
-  } else {
-    cfg.dynamicSmemBytes = generic_attn_smem(p);
-    CUDA_TRY(cudaLaunchKernelEx(&cfg, &attn_generic_kernel<float>, a));
+    return BASISKV_OK;
   }
+  cudaLaunchConfig_t cfg = launch_cfg(dim3(lp.attn_splits, p.num_kv_heads, lp.batch), kAttnThreads,
+                                      generic_attn_smem(p), stream, false, attr);
+  if (p.dtype == BASISKV_DTYPE_BF16)
+    CUDA_TRY(cudaLaunchKernelEx(&cfg, &attn_generic_kernel<__nv_bfloat16>, a));
+  else
+    CUDA_TRY(cudaLaunchKernelEx(&cfg, &attn_generic_kernel<float>, a));
   return BASISKV_OK;
 }
 
@@ -408,8 +539,12 @@ int basiskv_create(const basiskv_params* p, basiskv_handle** out) {
       {(void**)&h->d_sel, sizeof(int32_t) * U * p->max_topk},
       {(void**)&h->d_part_ml, sizeof(float) * U * kPartsCap * G * 2},
       {(void**)&h->d_part_acc, sizeof(float) * U * kPartsCap * G * p->rank_r},
-      {(void**)&h->d_counters, sizeof(uint32_t) * 2 * U},
+      {(void**)&h->d_counters, sizeof(uint32_t) * 3 * U},
       {(void**)&h->d_status, sizeof(uint32_t)},
+      {(void**)&h->d_route_off, sizeof(int32_t) * (B + 1)},
+      {(void**)&h->d_attn_off, sizeof(int32_t) * (B + 1)},
+      {(void**)&h->d_qfrag, sizeof(uint32_t) * U * 32 *
+                                (size_t)FragGeom(p->gqa_group, p->rank_r, p->rank_s).words()},
       {(void**)&h->d_q_stage, h->elem * B * Hkv * G * p->head_dim},
       {(void**)&h->d_out_stage, sizeof(float) * B * Hkv * G * p->head_dim},
       {(void**)&h->d_sel_stage, sizeof(int32_t) * U * p->max_topk},
@@ -422,16 +557,31 @@ int basiskv_create(const basiskv_params* p, basiskv_handle** out) {
   }
   if (cudaMemset(h->d_page_table, 0, sizeof(int32_t) * B * p->max_pages_per_seq) != cudaSuccess ||
       cudaMemset(h->d_seq_lens, 0, sizeof(int32_t) * B) != cudaSuccess ||
-      cudaMemset(h->d_counters, 0, sizeof(uint32_t) * 2 * U) != cudaSuccess ||
+      cudaMemset(h->d_counters, 0, sizeof(uint32_t) * 3 * U) != cudaSuccess ||
       cudaMemset(h->d_status, 0, sizeof(uint32_t)) != cudaSuccess)
     return cleanup_fail(BASISKV_ERR_CUDA, "cudaMemset failed");
   h->h_table.assign(B * p->max_pages_per_seq, 0);
   h->h_lens.assign(B, 0);
   h->h_npages.assign(B, 0);
 
+  h->frag_words = FragGeom(p->gqa_group, p->rank_r, p->rank_s).words();
+  h->topk_keys = std::min(p->max_pages_per_seq, 16384);
+  h->prep_smem = sizeof(float) * (size_t)p->gqa_group * (p->head_dim + p->rank_r + p->rank_s);
   choose_kernels(h);
   int arc = h->route_fn ? set_smem_attr((const void*)h->route_fn, h->route_smem) : BASISKV_OK;
   if (!arc && h->attn_fn) arc = set_smem_attr((const void*)h->attn_fn, h->attn_smem);
+  if (!arc)
+    arc = p->dtype == BASISKV_DTYPE_BF16 ? set_smem_attr((const void*)&prep_kernel<__nv_bfloat16>, h->prep_smem)
+                                         : set_smem_attr((const void*)&prep_kernel<float>, h->prep_smem);
+  if (!arc) arc = set_smem_attr((const void*)&topk_kernel, sizeof(uint32_t) * (size_t)h->topk_keys);
+  if (!arc && h->route_fn &&
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&h->route_occ, h->route_fn, kRouteThreads, h->route_smem) != cudaSuccess)
+    arc = fail(BASISKV_ERR_CUDA, "occupancy query failed");
+  if (!arc && h->attn_fn &&
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&h->attn_occ, h->attn_fn, kAttnThreads, h->attn_smem) != cudaSuccess)
+    arc = fail(BASISKV_ERR_CUDA, "occupancy query failed");
+  h->route_occ = std::max(1, h->route_occ);
+  h->attn_occ = std::max(1, h->attn_occ);
   if (!arc)
     arc = p->dtype == BASISKV_DTYPE_BF16 ? set_generic_attrs<__nv_bfloat16>(*p) : set_generic_attrs<float>(*p);
   if (arc) {
@@ -448,7 +598,8 @@ int basiskv_destroy(basiskv_handle* h) {
   if (!h) return BASISKV_OK;
   cudaDeviceSynchronize();
   void* ptrs[] = {h->d_page_table, h->d_seq_lens, h->d_scores, h->d_sel, h->d_part_ml, h->d_part_acc,
-                  h->d_counters, h->d_status, h->d_q_stage, h->d_out_stage, h->d_sel_stage};
+                  h->d_counters, h->d_status, h->d_q_stage, h->d_out_stage, h->d_sel_stage,
+                  h->d_route_off, h->d_attn_off, h->d_qfrag};
   for (void* q : ptrs)
     if (q) cudaFree(q);
   for (cudaEvent_t e : h->events) cudaEventDestroy(e);
@@ -551,22 +702,36 @@ int basiskv_decode_attn(basiskv_handle* h, int batch, const void* q, int topk, f
   const bool prof = h->prof_calls < h->prof_cap;
   cudaEvent_t* ev = prof ? &h->events[3 * h->prof_calls] : nullptr;
   if (prof) CUDA_TRY(cudaEventRecord(ev[0], st));
-  if (lp.any_routed) {
-    RouteArgs ra = route_args(h, batch, q, topk, h->d_scores, sel_out, 0, lp.route_ppc, 0);
-    rc = launch_route(h, lp, ra, st);
+  const bool route_tc = lp.any_routed && h->route_fn;
+  const bool use_prep = route_tc || h->attn_fn;
+  if (use_prep) {
+    rc = launch_prep(h, lp, q, topk, 0, out, sel_out, nullptr, st);
     if (rc) return rc;
   }
+  if (lp.any_routed) {
+    RouteArgs ra = route_args(h, lp, q, topk, h->d_scores, sel_out, 0);
+    rc = launch_route(h, lp, ra, !prof, st);
+    if (rc) return rc;
+    if (h->route_fn) {
+      rc = launch_topk(h, lp, topk, h->d_scores, sel_out, 0, !prof, st);
+      if (rc) return rc;
+    }
+  }
   if (prof) CUDA_TRY(cudaEventRecord(ev[1], st));
-  rc = launch_attn(h, lp, q, topk, softmax_scale, out, sel_out, lp.any_routed && !prof, st);
+  // PDL needs the plan complete when this grid starts: it is in the
+  // parameters, or a routing grid (which signals only after the prep grid
+  // finished) precedes this one
+  rc = launch_attn(h, lp, q, topk, softmax_scale, out, sel_out,
+                   use_prep && (!lp.attn_off.empty() || lp.any_routed) && !prof, st);
   if (rc) return rc;
   if (prof) {
     CUDA_TRY(cudaEventRecord(ev[2], st));
     ++h->prof_calls;
   }
-  h->last_launch[0] = lp.any_routed ? lp.route_ppc : 0;
-  h->last_launch[1] = lp.any_routed ? lp.route_chunks * h->p.num_kv_heads * batch : 0;
-  h->last_launch[2] = lp.attn_splits;
-  h->last_launch[3] = lp.attn_splits * h->p.num_kv_heads * batch;
+  h->last_launch[0] = lp.any_routed ? (h->route_fn ? 0 : lp.route_ppc) : 0;
+  h->last_launch[1] = lp.any_routed ? (h->route_fn ? lp.route_ctas : lp.route_chunks * h->p.num_kv_heads * batch) : 0;
+  h->last_launch[2] = h->attn_fn ? 0 : lp.attn_splits;
+  h->last_launch[3] = h->attn_fn ? lp.attn_ctas : lp.attn_splits * h->p.num_kv_heads * batch;
   h->last_launch[4] = h->route_fn != nullptr;
   h->last_launch[5] = h->attn_fn != nullptr;
   return BASISKV_OK;
@@ -597,21 +762,17 @@ int basiskv_route(basiskv_handle* h, int batch, const void* q, int topk, float* 
   int rc = check_call(h, batch, q, topk);
   if (rc) return rc;
   if (batch == 0) return BASISKV_OK;
+  cudaStream_t st = (cudaStream_t)stream;
   const LaunchPlan lp = plan(h, batch, topk, true);
-  if (!lp.any_routed) {
-    if (scores_out || sel_out) {
-      // no sequence has a page: scores all -inf, selections all -1
-      if (scores_out) {
-        std::vector<float> ninf((size_t)batch * h->p.num_kv_heads * h->p.max_pages_per_seq, -INFINITY);
-        CUDA_TRY(cudaMemcpyAsync(scores_out, ninf.data(), sizeof(float) * ninf.size(), cudaMemcpyHostToDevice, (cudaStream_t)stream));
-        CUDA_TRY(cudaStreamSynchronize((cudaStream_t)stream));
-      }
-      if (sel_out) CUDA_TRY(cudaMemsetAsync(sel_out, 0xff, sizeof(int32_t) * batch * h->p.num_kv_heads * topk, (cudaStream_t)stream));
-    }
-    return BASISKV_OK;
-  }
-  RouteArgs ra = route_args(h, batch, q, topk, scores_out ? scores_out : h->d_scores, sel_out, 1, lp.route_ppc, 0);
-  return launch_route(h, lp, ra, (cudaStream_t)stream);
+  float* scores = scores_out ? scores_out : h->d_scores;
+  // the prep grid writes -inf past n_b and the -1 rows of empty sequences
+  rc = launch_prep(h, lp, q, topk, 1, nullptr, sel_out, scores, st);
+  if (rc) return rc;
+  if (!lp.any_routed) return BASISKV_OK;
+  RouteArgs ra = route_args(h, lp, q, topk, scores, sel_out, 1);
+  rc = launch_route(h, lp, ra, true, st);
+  if (rc || !h->route_fn) return rc;
+  return launch_topk(h, lp, topk, scores, sel_out, 1, true, st);
 }
 
 int basiskv_get_status(basiskv_handle* h, uint32_t* status, int clear) {

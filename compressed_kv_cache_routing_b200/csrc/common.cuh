@@ -13,6 +13,10 @@ constexpr uint32_t kStatusBadSlot = 1u;
 constexpr uint32_t kStatusTimeout = 2u;
 constexpr uint32_t kStatusBadPage = 4u;
 
+// Largest batch whose work plan travels in the kernel parameters; larger
+// batches read the plan the prep grid writes to global memory.
+constexpr int kPlanMax = 512;
+
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 

@@ -16,6 +16,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "plan.cuh"
 #include "topk.cuh"
 
 namespace basiskv {
@@ -38,6 +39,13 @@ struct RouteArgs {
   int topk, pages_per_cta, stages;
   int force;                // route units whose every page would be selected
   int fill_tail;            // chunk 0 writes -inf to scores[n_b .. ld_pt)
+  // persistent tensor-core kernel only
+  int batch;
+  const int32_t* route_off; // [B+1] prefix of routed pages x Hkv (from the prep grid)
+  const uint32_t* qfrag;    // [B*Hkv][frag_words][32] query B fragments
+  int frag_words;
+  int plan_n;               // >= 0: plan_off holds route_off (batch <= kPlanMax)
+  int32_t plan_off[kPlanMax + 1];
 };
 
 constexpr int kRouteThreads = 128;
@@ -115,9 +123,11 @@ __device__ void route_finish(const RouteArgs& a, const RouteUnit& ru, TopkSmem& 
 // The B fragments use the same permutation, so every dot product is a sum
 // over the same index set.
 //
-// Pages stream through per-warp rings of `stages` shared buffers filled by
-// bulk copies (cp.async.bulk, L2 evict-first) completing on mbarriers; each
-// warp owns pages first+w, first+w+4, ... of the CTA.
+// Persistent: every warp streams one contiguous share of the flat list of
+// routed pages (sequence-major, then KV head, then page) through its own
+// ring of `stages` shared buffers filled by bulk copies (cp.async.bulk, L2
+// evict-first) completing on mbarriers, and writes one score per page.  The
+// selection runs in the next grid (topk_kernel).
 template <int G, int RR, int RS>
 struct RouteMma {
   static constexpr int NT = (2 * G + 7) / 8;  // n8 tiles of (hi, lo) columns
@@ -136,171 +146,186 @@ __device__ __forceinline__ int k16_phys(int blk, int t, int half) {
   return 32 * W32 + 4 * t + 2 * half;
 }
 
-template <int G, int RR, int RS>
-__global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const RouteArgs a) {
+// Position in the flat list of routed pages (sequence-major, then KV head,
+// then page), advanced one page at a time.
+struct RouteCursor {
+  int b, kvh, j, n, L;
+  const int32_t* off;  // prefix of routed pages x Hkv over sequences
+  __device__ __forceinline__ void load(const RouteArgs& a) {
+    L = a.seq_lens[b];
+    n = (L + a.page_size - 1) / a.page_size;
+  }
+  __device__ __forceinline__ bool routed(const RouteArgs& a) const {
+    return n > 0 && (a.force || a.topk < n);
+  }
+  // first page at or after flat index f (route_off[b] <= f < route_off[b+1])
+  __device__ void seek(const RouteArgs& a, const int32_t* offsets, int f) {
+    off = offsets;
+    int lo = 0, hi = a.batch;  // first b with off[b] > f, minus one
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (off[mid] <= f) lo = mid + 1;
+      else hi = mid;
+    }
+    b = lo - 1;
+    load(a);
+    const int rel = f - off[b];
+    kvh = rel / n;
+    j = rel % n;
+  }
+  __device__ __forceinline__ void advance(const RouteArgs& a) {
+    if (++j < n) return;
+    j = 0;
+    if (++kvh < a.num_kv_heads) return;
+    kvh = 0;
+    for (++b; b < a.batch; ++b) {
+      load(a);
+      if (routed(a)) return;
+    }
+  }
+  __device__ __forceinline__ int unit(const RouteArgs& a) const { return b * a.num_kv_heads + kvh; }
+};
+
+template <int G, int RR, int RS, int P>
+__global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_constant__ RouteArgs a) {
   using Shape = RouteMma<G, RR, RS>;
   constexpr int NT = Shape::NT;
-  pdl_launch_dependents();
-  const RouteUnit ru = route_unit(a);
-  if (a.fill_tail && blockIdx.x == 0)
-    for (int j = ru.n + threadIdx.x; j < a.ld_pt; j += blockDim.x)
-      a.scores[(size_t)ru.u * a.ld_pt + j] = -INFINITY;
-  if (!ru.active) return;
-
-  const int P = a.page_size;
+  static_assert(P % 16 == 0, "page size must be a multiple of 16");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
-  const uint32_t zbytes = (uint32_t)P * RR * 2, rbytes = (uint32_t)P * RS * 2;
-  const uint32_t stage_bytes = zbytes + rbytes;
+  constexpr uint32_t zbytes = P * RR * 2, rbytes = P * RS * 2;
+  constexpr uint32_t stage_bytes = zbytes + rbytes;
   const int S = a.stages;
 
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t bars[kRouteWarps][kMaxStages];
-  __shared__ TopkSmem tk;
-  __shared__ int flag;
   uint8_t* ring = smem + (size_t)warp * S * stage_bytes;
-  float* qs = reinterpret_cast<float*>(smem + (size_t)kRouteWarps * S * stage_bytes);
-  float* qz = qs + G * a.head_dim;
-  float* qr = qz + G * RR;
+  if (lane == 0) {
+    for (int i = 0; i < S; ++i) mbar_init(&bars[warp][i], 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
+  // The plan comes in the parameters (small batches) or from the prep grid.
+  // With the plan in hand the first copies go out before the prep grid has
+  // finished folding the query.
+  const int32_t* offsets = a.plan_n >= 0 ? a.plan_off : a.route_off;
+  if (a.plan_n < 0) pdl_wait_primary();
 
-  const int npg = ru.last - ru.first;
-  const int mine = npg > warp ? (npg - warp + kRouteWarps - 1) / kRouteWarps : 0;
+  // this warp's contiguous share of the flat routed-page list
+  const int W = gridDim.x * kRouteWarps, wg = blockIdx.x * kRouteWarps + warp;
+  const long long T = offsets[a.batch];
+  const int f0 = (int)(T * wg / W), f1 = (int)(T * (wg + 1) / W);
+  const int count = f1 - f0;
+
   const __nv_bfloat16* zpool = static_cast<const __nv_bfloat16*>(a.z_pool);
   const __nv_bfloat16* rpool = static_cast<const __nv_bfloat16*>(a.r_pool);
-  const int32_t* ptab = a.page_table + (size_t)ru.b * a.ld_pt;
-  uint64_t pol = policy_evict_first();
-
-  auto issue = [&](int i) {  // lane 0 only: my i-th page into stage i % S
-    const int p = ru.first + warp + i * kRouteWarps;
-    int slot = ptab[p];
+  const uint64_t pol = policy_evict_first();
+  RouteCursor ic;  // issue cursor (lane 0), runs S pages ahead
+  if (count > 0) ic.seek(a, offsets, f0);
+  RouteCursor cc = ic;  // compute cursor
+  // lane 0 looks the next slot up one iteration early, so the page-table
+  // read overlaps the current page's arithmetic
+  auto lookup = [&]() { return __ldg(a.page_table + (size_t)ic.b * a.ld_pt + ic.j); };
+  auto issue = [&](int i, int slot) {
     if (slot < 0 || slot >= a.num_slots) {
       atomicOr(a.status, kStatusBadSlot);
       slot = 0;
     }
-    const size_t row0 = ((size_t)slot * a.num_kv_heads + ru.kvh) * P;
+    const size_t row0 = ((size_t)slot * a.num_kv_heads + ic.kvh) * P;
     uint64_t* bar = &bars[warp][i % S];
     uint8_t* dst = ring + (size_t)(i % S) * stage_bytes;
     mbar_arrive_expect_tx(bar, stage_bytes);
     bulk_load(dst, zpool + row0 * RR, zbytes, bar, pol);
     if (RS > 0) bulk_load(dst + zbytes, rpool + row0 * RS, rbytes, bar, pol);
+    ic.advance(a);
   };
-
-  if (lane == 0) {
-    for (int i = 0; i < S; ++i) mbar_init(&bars[warp][i], 1);
-    mbar_init_fence();
-    for (int i = 0; i < S && i < mine; ++i) issue(i);
-  }
-  __syncwarp();
-
-  route_prep<__nv_bfloat16>(a, ru, qs, qz, qr);
-
-  // B fragments of the split query: column n = 8j + g -> head 4j + g/2,
-  // hi (g even) or lo (g odd) half.
-  uint32_t bz[NT][Shape::ZB > 0 ? Shape::ZB : 1][2];
-  uint32_t bz8[NT];
-  uint32_t bs[NT][Shape::SB > 0 ? Shape::SB : 1][2];
-  uint32_t bs8[NT];
-#pragma unroll
-  for (int j = 0; j < NT; ++j) {
-    const int h = 4 * j + (g >> 1);
-    const bool lo = g & 1;
-    auto part = [&](const float* v, int idx) {
-      if (h >= G) return 0.f;
-      float hi, lw;
-      split_bf16(v[idx], hi, lw);
-      return lo ? lw : hi;
-    };
-    const float* qzh = qz + h * RR;
-    const float* qrh = qr + h * RS;
-#pragma unroll
-    for (int blk = 0; blk < Shape::ZB; ++blk) {
-      const int e0 = k16_phys<Shape::Z32, Shape::Z16>(blk, t, 0);
-      const int e1 = k16_phys<Shape::Z32, Shape::Z16>(blk, t, 1);
-      bz[j][blk][0] = pack_bf16(part(qzh, e0), part(qzh, e0 + 1));
-      bz[j][blk][1] = pack_bf16(part(qzh, e1), part(qzh, e1 + 1));
+  {
+    // the first S pages: lane j looks page j up (in parallel), lane 0 issues
+    const int first = min(S, count);
+    int sl = 0;
+    if (lane < first) {
+      RouteCursor c = ic;
+      for (int k = 0; k < lane; ++k) c.advance(a);
+      sl = __ldg(a.page_table + (size_t)c.b * a.ld_pt + c.j);
     }
-    if (Shape::Z8) {
-      const int e = 32 * Shape::Z32 + 16 * Shape::Z16 + 2 * t;
-      bz8[j] = pack_bf16(part(qzh, e), part(qzh, e + 1));
-    }
-#pragma unroll
-    for (int blk = 0; blk < Shape::SB; ++blk) {
-      const int e0 = k16_phys<Shape::S32, Shape::S16>(blk, t, 0);
-      const int e1 = k16_phys<Shape::S32, Shape::S16>(blk, t, 1);
-      bs[j][blk][0] = pack_bf16(part(qrh, e0), part(qrh, e0 + 1));
-      bs[j][blk][1] = pack_bf16(part(qrh, e1), part(qrh, e1 + 1));
-    }
-    if (Shape::S8) {
-      const int e = 32 * Shape::S32 + 16 * Shape::S16 + 2 * t;
-      bs8[j] = pack_bf16(part(qrh, e), part(qrh, e + 1));
+    for (int i = 0; i < first; ++i) {
+      const int sli = __shfl_sync(0xffffffffu, sl, i);
+      if (lane == 0) issue(i, sli);
     }
   }
+  if (a.plan_n >= 0) pdl_wait_primary();  // query fragments
+  pdl_launch_dependents();
+  if (count <= 0) return;
 
-  float* scores = a.scores + (size_t)ru.u * a.ld_pt;
+  constexpr int FR = NT * (2 * Shape::ZB + Shape::Z8 + 2 * Shape::SB + Shape::S8);
+  uint32_t fr[FR];
+  int cur_u = -1;
+
   bool ok = true;
   int i = 0;
-  for (; i < mine; ++i) {
-    const int p = ru.first + warp + i * kRouteWarps;
+  for (; i < count; ++i) {
+    int next_slot = 0;
+    if (lane == 0 && i + S < count) next_slot = lookup();
+    const int u = cc.unit(a);
+    if (u != cur_u) {
+      cur_u = u;
+      const uint32_t* src = a.qfrag + (size_t)u * a.frag_words * 32 + lane;
+#pragma unroll
+      for (int w = 0; w < FR; ++w) fr[w] = __ldcg(src + w * 32);
+    }
     ok = mbar_wait(&bars[warp][i % S], (uint32_t)((i / S) & 1), a.status);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;
     const __nv_bfloat16* zs = reinterpret_cast<const __nv_bfloat16*>(ring + (size_t)(i % S) * stage_bytes);
     const __nv_bfloat16* rs = zs + P * RR;
-    const int valid = min(P, ru.L - p * P);
+    const int valid = min(P, cc.L - cc.j * P);
     float best = -INFINITY;
-    for (int mt = 0; mt * 16 < valid; ++mt) {
+#pragma unroll
+    for (int mt = 0; mt < P / 16; ++mt) {
       float acc[NT][4];
 #pragma unroll
       for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
       const __nv_bfloat16* z0 = zs + (mt * 16 + g) * RR;
       const __nv_bfloat16* z1 = z0 + 8 * RR;
 #pragma unroll
-      for (int sp = 0; sp < Shape::Z32; ++sp) {
-        const uint4 v0 = lds128(z0 + 32 * sp + 8 * t), v1 = lds128(z1 + 32 * sp + 8 * t);
+      for (int j = 0; j < NT; ++j) {
+        const uint32_t* f = fr + j * (2 * Shape::ZB + Shape::Z8 + 2 * Shape::SB + Shape::S8);
 #pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          mma_k16(acc[j], v0.x, v1.x, v0.y, v1.y, bz[j][2 * sp][0], bz[j][2 * sp][1]);
-          mma_k16(acc[j], v0.z, v1.z, v0.w, v1.w, bz[j][2 * sp + 1][0], bz[j][2 * sp + 1][1]);
+        for (int sp = 0; sp < Shape::Z32; ++sp) {
+          const uint4 v0 = lds128(z0 + 32 * sp + 8 * t), v1 = lds128(z1 + 32 * sp + 8 * t);
+          mma_k16(acc[j], v0.x, v1.x, v0.y, v1.y, f[4 * sp + 0], f[4 * sp + 1]);
+          mma_k16(acc[j], v0.z, v1.z, v0.w, v1.w, f[4 * sp + 2], f[4 * sp + 3]);
         }
-      }
-      if (Shape::Z16) {
-        const uint2 v0 = lds64(z0 + 32 * Shape::Z32 + 4 * t), v1 = lds64(z1 + 32 * Shape::Z32 + 4 * t);
+        if (Shape::Z16) {
+          const uint2 v0 = lds64(z0 + 32 * Shape::Z32 + 4 * t), v1 = lds64(z1 + 32 * Shape::Z32 + 4 * t);
+          mma_k16(acc[j], v0.x, v1.x, v0.y, v1.y, f[2 * Shape::ZB - 2], f[2 * Shape::ZB - 1]);
+        }
+        if (Shape::Z8) {
+          const int o = 32 * Shape::Z32 + 16 * Shape::Z16 + 2 * t;
+          mma_k8(acc[j], lds32(z0 + o), lds32(z1 + o), f[2 * Shape::ZB]);
+        }
+        if (RS > 0) {
+          const uint32_t* fs = f + 2 * Shape::ZB + Shape::Z8;
+          const __nv_bfloat16* r0 = rs + (mt * 16 + g) * RS;
+          const __nv_bfloat16* r1 = r0 + 8 * RS;
 #pragma unroll
-        for (int j = 0; j < NT; ++j)
-          mma_k16(acc[j], v0.x, v1.x, v0.y, v1.y, bz[j][Shape::ZB - 1][0], bz[j][Shape::ZB - 1][1]);
-      }
-      if (Shape::Z8) {
-        const int o = 32 * Shape::Z32 + 16 * Shape::Z16 + 2 * t;
-        const uint32_t v0 = lds32(z0 + o), v1 = lds32(z1 + o);
-#pragma unroll
-        for (int j = 0; j < NT; ++j) mma_k8(acc[j], v0, v1, bz8[j]);
-      }
-      if (RS > 0) {
-        const __nv_bfloat16* r0 = rs + (mt * 16 + g) * RS;
-        const __nv_bfloat16* r1 = r0 + 8 * RS;
-#pragma unroll
-        for (int sp = 0; sp < Shape::S32; ++sp) {
-          const uint4 v0 = lds128(r0 + 32 * sp + 8 * t), v1 = lds128(r1 + 32 * sp + 8 * t);
-#pragma unroll
-          for (int j = 0; j < NT; ++j) {
-            mma_k16(acc[j], v0.x, v1.x, v0.y, v1.y, bs[j][2 * sp][0], bs[j][2 * sp][1]);
-            mma_k16(acc[j], v0.z, v1.z, v0.w, v1.w, bs[j][2 * sp + 1][0], bs[j][2 * sp + 1][1]);
+          for (int sp = 0; sp < Shape::S32; ++sp) {
+            const uint4 v0 = lds128(r0 + 32 * sp + 8 * t), v1 = lds128(r1 + 32 * sp + 8 * t);
+            mma_k16(acc[j], v0.x, v1.x, v0.y, v1.y, fs[4 * sp + 0], fs[4 * sp + 1]);
+            mma_k16(acc[j], v0.z, v1.z, v0.w, v1.w, fs[4 * sp + 2], fs[4 * sp + 3]);
+          }
+          if (Shape::S16) {
+            const uint2 v0 = lds64(r0 + 32 * Shape::S32 + 4 * t), v1 = lds64(r1 + 32 * Shape::S32 + 4 * t);
+            mma_k16(acc[j], v0.x, v1.x, v0.y, v1.y, fs[2 * Shape::SB - 2], fs[2 * Shape::SB - 1]);
+          }
+          if (Shape::S8) {
+            const int o = 32 * Shape::S32 + 16 * Shape::S16 + 2 * t;
+            mma_k8(acc[j], lds32(r0 + o), lds32(r1 + o), fs[2 * Shape::SB]);
           }
         }
-        if (Shape::S16) {
-          const uint2 v0 = lds64(r0 + 32 * Shape::S32 + 4 * t), v1 = lds64(r1 + 32 * Shape::S32 + 4 * t);
-#pragma unroll
-          for (int j = 0; j < NT; ++j)
-            mma_k16(acc[j], v0.x, v1.x, v0.y, v1.y, bs[j][Shape::SB - 1][0], bs[j][Shape::SB - 1][1]);
-        }
-        if (Shape::S8) {
-          const int o = 32 * Shape::S32 + 16 * Shape::S16 + 2 * t;
-          const uint32_t v0 = lds32(r0 + o), v1 = lds32(r1 + o);
-#pragma unroll
-          for (int j = 0; j < NT; ++j) mma_k8(acc[j], v0, v1, bs8[j]);
-        }
       }
-      // D fragment: rows g, g+8 = tokens; columns 2t, 2t+1 = (hi, lo) of head 4j + t
+      // D fragment: rows g, g+8 = tokens; columns 2t, 2t+1 = (hi, lo) of head 4j + t.
+      // Rows past the sequence end are dropped by selection, never by arithmetic.
       const int tok0 = mt * 16 + g, tok1 = tok0 + 8;
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
@@ -313,24 +338,23 @@ __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const RouteArg
     best = warp_max(best);
     __syncwarp();
     if (lane == 0) {
-      scores[p] = best;
-      if (i + S < mine) issue(i + S);
+      a.scores[(size_t)cur_u * a.ld_pt + cc.j] = best;
+      if (i + S < count) issue(i + S, next_slot);
     }
+    cc.advance(a);
   }
-  if (!ok && lane == 0) {
-    // a copy never completed: wait (bounded) for the pages still in flight,
-    // [i, min(i + S, mine)), before the CTA's shared memory is released
-    for (int j = i; j < mine && j < i + S; ++j)
-      mbar_wait(&bars[warp][j % S], (uint32_t)((j / S) & 1), a.status);
+  if (!ok) {
+    if (lane == 0)  // drain the copies still in flight, [i, min(i + S, count))
+      for (int j = i; j < count && j < i + S; ++j)
+        mbar_wait(&bars[warp][j % S], (uint32_t)((j / S) & 1), a.status);
   }
-  route_finish<kRouteThreads>(a, ru, tk, &flag);
 }
 
 // ---------------------------------------------------------------------------
 // CUDA-core routing for any shape and for fp32 pools: thread per (token,
 // head) pair, rows read straight from global memory.
 template <typename T>
-__global__ void __launch_bounds__(kRouteThreads) route_generic_kernel(const RouteArgs a) {
+__global__ void __launch_bounds__(kRouteThreads) route_generic_kernel(const __grid_constant__ RouteArgs a) {
   pdl_launch_dependents();
   const RouteUnit ru = route_unit(a);
   if (a.fill_tail && blockIdx.x == 0)

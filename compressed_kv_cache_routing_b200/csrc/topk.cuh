@@ -134,3 +134,223 @@ __device__ void block_topk(const float* scores, int n, int k, int32_t* sel, int3
 }
 
 }  // namespace basiskv
+
+namespace basiskv {
+
+// One-warp version of block_topk for the warp that completes a unit:
+// same ordering and output.  hist: 256 ints of this warp's shared memory.
+__device__ void warp_topk(const float* scores, int n, int k, int32_t* sel, int32_t* sel_out,
+                          int out_len, int* hist) {
+  const int lane = threadIdx.x & 31;
+  const int kb = k < n ? k : n;
+  uint32_t thr = 0u;
+  int need = 0;
+  if (kb < n) {
+    uint32_t prefix = 0u, mask = 0u;
+    int remaining = kb;
+#pragma unroll 1
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = lane; i < 256; i += 32) hist[i] = 0;
+      __syncwarp();
+      for (int base = 0; base < n; base += 32) {
+        const int i = base + lane;
+        const uint32_t key = i < n ? score_key(__ldcg(scores + i)) : 0u;
+        const bool in = i < n && (key & mask) == prefix;
+        const uint32_t act = __ballot_sync(0xffffffffu, in);
+        if (in) {
+          // one shared atomic per distinct digit: lanes holding equal digits
+          // (the common case in the top byte) would otherwise serialise
+          const uint32_t digit = (key >> shift) & 255u;
+          const uint32_t grp = __match_any_sync(act, digit);
+          if ((int)(__ffs(grp) - 1) == lane) atomicAdd(&hist[digit], __popc(grp));
+        }
+      }
+      __syncwarp();
+      int local = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) local += hist[8 * lane + q];
+      int incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_down_sync(0xffffffffu, incl, o);
+        if (lane + o < 32) incl += y;
+      }
+      const int above = incl - local;
+      const bool mine = above < remaining && remaining <= incl;
+      int digit = 0, rem = 0;
+      if (mine) {
+        int acc = above;
+        for (int q = 7; q >= 0; --q) {
+          const int c = hist[8 * lane + q];
+          if (acc + c >= remaining) {
+            digit = 8 * lane + q;
+            rem = remaining - acc;
+            break;
+          }
+          acc += c;
+        }
+      }
+      const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+      digit = __shfl_sync(0xffffffffu, digit, src);
+      remaining = __shfl_sync(0xffffffffu, rem, src);
+      prefix |= static_cast<uint32_t>(digit) << shift;
+      mask |= 0xFFu << shift;
+      __syncwarp();
+    }
+    thr = prefix;
+    need = remaining;
+  }
+  const uint32_t lt = (1u << lane) - 1u;
+  int eq_before = 0, taken = 0;
+  for (int base = 0; base < n; base += 32) {
+    const int i = base + lane;
+    bool take = false, eq = false;
+    if (i < n) {
+      if (kb < n) {
+        const uint32_t key = score_key(__ldcg(scores + i));
+        eq = key == thr;
+        take = key > thr;
+      } else {
+        take = true;
+      }
+    }
+    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+    if (eq && eq_before + __popc(eqm & lt) < need) take = true;
+    const uint32_t tm = __ballot_sync(0xffffffffu, take);
+    if (take) {
+      const int pos = taken + __popc(tm & lt);
+      sel[pos] = i;
+      if (sel_out) sel_out[pos] = i;
+    }
+    taken += __popc(tm);
+    eq_before += __popc(eqm);
+  }
+  if (sel_out)
+    for (int i = kb + lane; i < out_len; i += 32) sel_out[i] = -1;
+}
+
+}  // namespace basiskv
+
+namespace basiskv {
+
+// ---------------------------------------------------------------------------
+// Selection kernel: one CTA per (sequence, KV head) whose pages are routed.
+// The scores are staged once in shared memory (kTopkKeysMax of them), the
+// radix passes and the page-ordered compaction run there; units with more
+// pages read the scores from L2 on every pass (block_topk).
+struct TopkArgs {
+  const float* scores;     // [B][Hkv][ld_pt]
+  const int32_t* seq_lens; // [B]
+  int32_t* sel;            // [B][Hkv][ld_sel]
+  int32_t* sel_out;        // [B][Hkv][topk] or null
+  int num_kv_heads, page_size, ld_pt, ld_sel, topk, force, keys_cap;
+};
+
+constexpr int kTopkThreads = 256;
+
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkArgs a) {
+  pdl_launch_dependents();  // the attention grid waits for this one anyway
+  __shared__ TopkSmem sm;
+  extern __shared__ uint32_t keys[];
+  const int b = blockIdx.y, kvh = blockIdx.x, u = b * a.num_kv_heads + kvh;
+  const int n = (a.seq_lens[b] + a.page_size - 1) / a.page_size;
+  if (n == 0 || !(a.force || a.topk < n)) return;
+  pdl_wait_primary();  // the scores come from the routing grid
+  const float* sc = a.scores + (size_t)u * a.ld_pt;
+  int32_t* sel = a.sel + (size_t)u * a.ld_sel;
+  int32_t* so = a.sel_out ? a.sel_out + (size_t)u * a.topk : nullptr;
+  if (n > a.keys_cap) {
+    block_topk<kTopkThreads>(sc, n, a.topk, sel, so, a.topk, sm);
+    return;
+  }
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < n; i += kTopkThreads) keys[i] = score_key(__ldcg(sc + i));
+  __syncthreads();
+  const int kb = a.topk < n ? a.topk : n;
+  uint32_t thr = 0u;
+  int need = 0;
+  if (kb < n) {
+    uint32_t prefix = 0u, mask = 0u;
+    int remaining = kb;
+#pragma unroll 1
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += kTopkThreads) sm.hist[i] = 0;
+      __syncthreads();
+      for (int base = 0; base < n; base += kTopkThreads) {
+        const int i = base + tid;
+        const uint32_t key = i < n ? keys[i] : 0u;
+        const bool in = i < n && (key & mask) == prefix;
+        const uint32_t act = __ballot_sync(0xffffffffu, in);
+        if (in) {
+          const uint32_t digit = (key >> shift) & 255u;
+          const uint32_t grp = __match_any_sync(act, digit);
+          if ((int)(__ffs(grp) - 1) == lane) atomicAdd(&sm.hist[digit], __popc(grp));
+        }
+      }
+      __syncthreads();
+      if (warp == 0) {
+        int local = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) local += sm.hist[8 * lane + q];
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_down_sync(0xffffffffu, incl, o);
+          if (lane + o < 32) incl += y;
+        }
+        const int above = incl - local;
+        if (above < remaining && remaining <= incl) {
+          int acc = above;
+          for (int q = 7; q >= 0; --q) {
+            const int c = sm.hist[8 * lane + q];
+            if (acc + c >= remaining) {
+              sm.digit = 8 * lane + q;
+              sm.remaining = remaining - acc;
+              break;
+            }
+            acc += c;
+          }
+        }
+      }
+      __syncthreads();
+      prefix |= static_cast<uint32_t>(sm.digit) << shift;
+      mask |= 0xFFu << shift;
+      remaining = sm.remaining;
+      __syncthreads();
+    }
+    thr = prefix;
+    need = remaining;
+  }
+  // page-ordered compaction: each thread owns a contiguous run
+  const int per = (n + kTopkThreads - 1) / kTopkThreads;
+  const int i0 = min(n, tid * per), i1 = min(n, i0 + per);
+  int total;
+  int eq = 0, take = 0;
+  for (int i = i0; i < i1; ++i) eq += keys[i] == thr;
+  const int eq_before = kb < n ? block_exclusive_scan<kTopkThreads>(eq, sm.scan_tmp, &total) : 0;
+  {
+    int e = eq_before;
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t key = keys[i];
+      take += kb >= n || key > thr || (key == thr && e < need);
+      e += key == thr;
+    }
+  }
+  int pos = block_exclusive_scan<kTopkThreads>(take, sm.scan_tmp, &total);
+  {
+    int e = eq_before;
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t key = keys[i];
+      if (kb >= n || key > thr || (key == thr && e < need)) {
+        sel[pos] = i;
+        if (so) so[pos] = i;
+        ++pos;
+      }
+      e += key == thr;
+    }
+  }
+  if (so)
+    for (int i = kb + tid; i < a.topk; i += kTopkThreads) so[i] = -1;
+}
+
+}  // namespace basiskv
