@@ -36,6 +36,7 @@ EXPORTED = (
     "basiskv_reset_seq", "basiskv_load_page_table", "basiskv_decode_attn",
     "basiskv_decode_attn_host", "basiskv_route", "basiskv_get_status", "basiskv_profile_begin",
     "basiskv_profile_end", "basiskv_last_launch", "basiskv_last_error", "basiskv_version",
+    "basiskv_decode_attn_noalloc",
 )
 
 
@@ -87,6 +88,8 @@ def load(path: str = LIB_PATH):
         "basiskv_profile_end": [H, vp, vp, vp, ctypes.POINTER(ctypes.c_int)],
         "basiskv_last_launch": [H, ctypes.POINTER(ctypes.c_int * 6)],
         "basiskv_version": [],
+        "basiskv_decode_attn_noalloc": [ctypes.POINTER(basiskv_params), i32, vp, vp, vp, i32, f32, vp,
+                                        vp, vp],
     }
     for name, args in sigs.items():
         f = getattr(lib, name)
@@ -190,6 +193,18 @@ def basiskv_last_launch(h):
     keys = ("route_pages_per_cta", "route_ctas", "attn_splits", "attn_ctas", "route_tensor_core",
             "attn_tensor_core")
     return dict(zip(keys, list(info)))
+
+
+def basiskv_decode_attn_noalloc(params, page_table, seq_lens, q, topk, softmax_scale, out,
+                                sel_out=None, stream=None):
+    """Decode step without a handle or any device allocation (see basiskv.h):
+    for callers that may not allocate device memory.  ``page_table`` and
+    ``seq_lens`` are device int32 tensors; the library's fixed scratch array
+    is shared by all calls, so calls must not overlap on the GPU."""
+    _check(load().basiskv_decode_attn_noalloc(ctypes.byref(params), int(seq_lens.shape[0]),
+                                              _ptr(page_table), _ptr(seq_lens), _ptr(q), topk,
+                                              float(softmax_scale), _ptr(out), _ptr(sel_out),
+                                              _stream(stream)))
 
 
 def basiskv_version() -> int:

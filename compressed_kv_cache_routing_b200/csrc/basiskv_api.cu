@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <cstring>
 #include <map>
+#include <mutex>
 #include <string>
 #include <tuple>
 #include <vector>
@@ -828,3 +829,162 @@ int basiskv_last_launch(basiskv_handle* h, int info[6]) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free decode.  Some callers may not allocate device memory at
+// all: code running inside a framework that owns every allocation, or code
+// inside a region where cudaMalloc is not allowed.  This entry point runs
+// the decode step without a handle and without allocating: its scratch
+// (page scores, selection, split partials, arrival counters, a status word)
+// is one fixed-size __device__ array in this file, which every GPU that
+// loads the library keeps until the process exits.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 16u << 20;  // 16 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Device address of the scratch array on the current device.  The symbol's
+// host-side name is not a device address, so it is resolved here once per
+// device with cudaGetSymbolAddress.
+int noalloc_scratch(int dev, void** out) {
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(BASISKV_ERR_UNSUPPORTED, "device %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(BASISKV_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return BASISKV_OK;
+}
+
+}  // namespace
+
+extern "C" int basiskv_decode_attn_noalloc(const basiskv_params* p, int batch, const int32_t* page_table,
+                                           const int32_t* seq_lens, const void* q, int topk,
+                                           float softmax_scale, float* out, int32_t* sel_out,
+                                           basiskv_stream_t stream) {
+  int rc = validate_params(p);
+  if (rc) return rc;
+  if (batch < 0 || batch > p->max_batch) return fail(BASISKV_ERR_INVALID_ARG, "batch %d outside [0, %d]", batch, p->max_batch);
+  if (topk <= 0 || topk > p->max_topk) return fail(BASISKV_ERR_INVALID_ARG, "topk %d outside [1, %d]", topk, p->max_topk);
+  if (!q || !aligned16(q) || !out || !page_table || !seq_lens)
+    return fail(BASISKV_ERR_INVALID_ARG, "q (16-byte aligned), out, page_table and seq_lens are required");
+  if (!std::isfinite(softmax_scale)) return fail(BASISKV_ERR_INVALID_ARG, "softmax_scale must be finite");
+  if (batch == 0) return BASISKV_OK;
+
+  // scratch layout: counters | status | scores | selection | partial (m, l) | partial acc
+  const size_t U = (size_t)batch * p->num_kv_heads, G = p->gqa_group;
+  const int splits = std::min(kMaxSplits, std::max(1, topk));
+  const size_t off_counters = 0;
+  const size_t off_status = align256(off_counters + sizeof(uint32_t) * 2 * U);
+  const size_t off_scores = align256(off_status + sizeof(uint32_t));
+  const size_t off_sel = align256(off_scores + sizeof(float) * U * p->max_pages_per_seq);
+  const size_t off_ml = align256(off_sel + sizeof(int32_t) * U * topk);
+  const size_t off_acc = align256(off_ml + sizeof(float) * U * splits * G * 2);
+  const size_t need = align256(off_acc + sizeof(float) * U * splits * G * p->rank_r);
+  if (need > kNoAllocScratchBytes)
+    return fail(BASISKV_ERR_CAPACITY,
+                "this call needs %zu bytes of scratch; the allocation-free path has %zu (reduce batch, "
+                "pages per sequence or top-k, or use basiskv_create)", need, kNoAllocScratchBytes);
+
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  unsigned char* scratch = nullptr;
+  rc = noalloc_scratch(dev, reinterpret_cast<void**>(&scratch));
+  if (rc) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  // the arrival counters and the status word must start at zero
+  CUDA_TRY(cudaMemsetAsync(scratch, 0, off_scores, st));
+
+  // routing: a grid of (page chunk, KV head, sequence) sized by the table's
+  // row length; chunks past a sequence's pages exit at once
+  const int ppc = std::max(kRouteWarps * 2, std::min(64, p->max_pages_per_seq));
+  RouteArgs ra{};
+  ra.q = q;
+  ra.z_pool = p->z_pool;
+  ra.r_pool = p->r_pool;
+  ra.w_zk = p->w_zk;
+  ra.b_r = p->b_r;
+  ra.page_table = page_table;
+  ra.seq_lens = seq_lens;
+  ra.scores = reinterpret_cast<float*>(scratch + off_scores);
+  ra.sel = reinterpret_cast<int32_t*>(scratch + off_sel);
+  ra.sel_out = sel_out;
+  ra.counters = reinterpret_cast<uint32_t*>(scratch + off_counters);
+  ra.status = reinterpret_cast<uint32_t*>(scratch + off_status);
+  ra.ld_pt = p->max_pages_per_seq;
+  ra.ld_sel = topk;
+  ra.num_slots = p->num_slots;
+  ra.num_kv_heads = p->num_kv_heads;
+  ra.head_dim = p->head_dim;
+  ra.page_size = p->page_size;
+  ra.rank_r = p->rank_r;
+  ra.rank_s = p->rank_s;
+  ra.gqa_group = p->gqa_group;
+  ra.topk = topk;
+  ra.pages_per_cta = ppc;
+  ra.batch = batch;
+  ra.plan_n = -1;
+  const dim3 rgrid((p->max_pages_per_seq + ppc - 1) / ppc, p->num_kv_heads, batch);
+  const size_t rsmem = generic_route_smem(*p);
+  if (p->dtype == BASISKV_DTYPE_BF16) {
+    CUDA_TRY(cudaFuncSetAttribute(&route_generic_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
+    route_generic_kernel<__nv_bfloat16><<<rgrid, kRouteThreads, rsmem, st>>>(ra);
+  } else {
+    CUDA_TRY(cudaFuncSetAttribute(&route_generic_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
+    route_generic_kernel<float><<<rgrid, kRouteThreads, rsmem, st>>>(ra);
+  }
+  CUDA_TRY(cudaGetLastError());
+
+  // attention: (split, KV head, sequence), one partial per CTA
+  AttnArgs aa{};
+  aa.q = q;
+  aa.k_pool = p->k_pool;
+  aa.z_pool = p->z_pool;
+  aa.b_v = p->b_v;
+  aa.page_table = page_table;
+  aa.seq_lens = seq_lens;
+  aa.sel = ra.sel;
+  aa.sel_out = sel_out;
+  aa.part_ml = reinterpret_cast<float*>(scratch + off_ml);
+  aa.part_acc = reinterpret_cast<float*>(scratch + off_acc);
+  aa.counters = ra.counters + U;
+  aa.status = ra.status;
+  aa.out = out;
+  aa.ld_pt = p->max_pages_per_seq;
+  aa.ld_sel = topk;
+  aa.num_slots = p->num_slots;
+  aa.num_kv_heads = p->num_kv_heads;
+  aa.head_dim = p->head_dim;
+  aa.page_size = p->page_size;
+  aa.rank_r = p->rank_r;
+  aa.gqa_group = p->gqa_group;
+  aa.topk = topk;
+  aa.pages_per_split = (topk + splits - 1) / splits;
+  aa.np_cap = splits;
+  aa.scale_log2 = softmax_scale * 1.4426950408889634f;
+  aa.batch = batch;
+  aa.plan_n = -1;
+  const dim3 agrid((topk + aa.pages_per_split - 1) / aa.pages_per_split, p->num_kv_heads, batch);
+  const size_t g = p->gqa_group;
+  const size_t asmem = sizeof(float) * std::max(g * (p->head_dim + p->page_size + p->rank_r) + 3 * g,
+                                                combine_smem_floats(splits, p->gqa_group, p->rank_r));
+  if (p->dtype == BASISKV_DTYPE_BF16) {
+    CUDA_TRY(cudaFuncSetAttribute(&attn_generic_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asmem));
+    attn_generic_kernel<__nv_bfloat16><<<agrid, kAttnThreads, asmem, st>>>(aa);
+  } else {
+    CUDA_TRY(cudaFuncSetAttribute(&attn_generic_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asmem));
+    attn_generic_kernel<float><<<agrid, kAttnThreads, asmem, st>>>(aa);
+  }
+  CUDA_TRY(cudaGetLastError());
+  return BASISKV_OK;
+}

@@ -192,6 +192,37 @@ BASISKV_API int basiskv_profile_end(basiskv_handle *h, float *route_ms, float *a
  * whether the tensor-core kernels ran (1) or the generic ones (0). */
 BASISKV_API int basiskv_last_launch(basiskv_handle *h, int info[6]);
 
+/* Allocation-free decode step.  The BasisKV paper has no counterpart to
+ * this call: it exists for callers that must not allocate device memory,
+ * for instance code running under a framework that owns every device
+ * allocation, or inside a region where cudaMalloc is not permitted (and so
+ * cannot call basiskv_create).  It computes the same step as
+ * basiskv_decode_attn, without a handle:
+ *   p           pools, bases and shapes (host struct, as for basiskv_create);
+ *               p->max_batch bounds batch, p->max_pages_per_seq is the row
+ *               length of page_table, p->max_topk bounds topk
+ *   page_table  [batch][p->max_pages_per_seq] int32 (device), seq_lens
+ *               [batch] int32 (device); q, topk, softmax_scale, out, sel_out
+ *               as for basiskv_decode_attn
+ * It allocates nothing.  Its scratch (page scores, selection, split
+ * partials, arrival counters) lives in one 16 MiB __device__ array inside
+ * the library, held by every GPU that loads the library until the process
+ * exits.  A call whose scratch would exceed 16 MiB
+ * (about batch * Hkv * (4 * max_pages_per_seq + 4 * topk + 32 * G * (r + 2))
+ * bytes) is rejected with BASISKV_ERR_CAPACITY and a message naming the
+ * size.  The first call on each device resolves the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  Every call clears the counters it needs on
+ * `stream`, then reuses the same array, which keeps the last call's
+ * contents: calls that may overlap on the GPU (other streams, other host
+ * threads) race on it and must be serialised by the caller.  It runs the
+ * CUDA-core kernels, not the persistent tensor-core ones.  Errors:
+ * INVALID_ARG, CAPACITY, CUDA, UNSUPPORTED. */
+BASISKV_API int basiskv_decode_attn_noalloc(const basiskv_params *p, int batch,
+                                            const int32_t *page_table, const int32_t *seq_lens,
+                                            const void *q, int topk, float softmax_scale,
+                                            float *out, int32_t *sel_out, basiskv_stream_t stream);
+
 /* Thread-local message for the last non-zero return of this thread. */
 BASISKV_API const char *basiskv_last_error(void);
 
