@@ -85,7 +85,7 @@ def load(path: str = LIB_PATH):
         "basiskv_route": [H, i32, vp, i32, vp, vp, vp],
         "basiskv_get_status": [H, ctypes.POINTER(ctypes.c_uint32), i32],
         "basiskv_profile_begin": [H, i32],
-        "basiskv_profile_end": [H, vp, vp, vp, ctypes.POINTER(ctypes.c_int)],
+        "basiskv_profile_end": [H, vp, ctypes.POINTER(ctypes.c_int)],
         "basiskv_last_launch": [H, ctypes.POINTER(ctypes.c_int * 6)],
         "basiskv_version": [],
         "basiskv_decode_attn_noalloc": [ctypes.POINTER(basiskv_params), i32, vp, vp, vp, i32, f32, vp,
@@ -179,12 +179,13 @@ def basiskv_profile_begin(h, max_calls):
 
 
 def basiskv_profile_end(h, max_calls):
-    r = np.zeros(max(max_calls, 1), np.float32)
-    a = np.zeros_like(r)
-    t = np.zeros_like(r)
+    """Per recorded call: dict of arrays (ms) for the prep, routing,
+    selection and attention grids and the whole call."""
+    ms = np.zeros((max(max_calls, 1), 5), np.float32)
     n = ctypes.c_int()
-    _check(load().basiskv_profile_end(h, r.ctypes.data, a.ctypes.data, t.ctypes.data, ctypes.byref(n)))
-    return r[:n.value], a[:n.value], t[:n.value]
+    _check(load().basiskv_profile_end(h, ms.ctypes.data, ctypes.byref(n)))
+    ms = ms[:n.value]
+    return {"prep": ms[:, 0], "route": ms[:, 1], "select": ms[:, 2], "attn": ms[:, 3], "total": ms[:, 4]}
 
 
 def basiskv_last_launch(h):

@@ -198,6 +198,15 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t bars[kAttnWarps][8];
   __shared__ int tok0s[kAttnWarps][8];
+  // sequences no warp visits: without pages they get out = 0 and a -1
+  // selection; with every page used (no routing) the identity selection
+  for (int u = blockIdx.x; u < a.batch * a.num_kv_heads; u += gridDim.x) {
+    const int n = (a.seq_lens[u / a.num_kv_heads] + a.page_size - 1) / a.page_size;
+    if (n == 0)
+      for (int i = threadIdx.x; i < G * D; i += blockDim.x) a.out[(size_t)u * G * D + i] = 0.f;
+    if (a.sel_out && a.topk >= n)
+      for (int i = threadIdx.x; i < a.topk; i += blockDim.x) a.sel_out[(size_t)u * a.topk + i] = i < n ? i : -1;
+  }
   uint8_t* ring = smem + (size_t)warp * S * stage_bytes;
   float* zbar = reinterpret_cast<float*>(smem + (size_t)kAttnWarps * S * stage_bytes) + warp * G * RR;
   if (lane == 0) {
@@ -237,7 +246,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
     cur_u = cc.unit(a);
     load_q(cur_u);
   }
-  pdl_wait_primary();  // the selection is written by the routing grid
+  pdl_wait_primary();  // the selection is written by the previous grid
   if (count <= 0) return;
 
   const __nv_bfloat16* kpool = static_cast<const __nv_bfloat16*>(a.k_pool);

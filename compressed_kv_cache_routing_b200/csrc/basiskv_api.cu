@@ -41,6 +41,7 @@ int fail(int code, const char* fmt, ...) {
   } while (0)
 
 constexpr int kMaxSplits = 16;
+constexpr int kProfEvents = 5;  // start, after prep, after routing, after selection, after attention
 constexpr int kPartsCap = kMaxSplits * kAttnWarps;  // partials per unit
 // Ring bytes per CTA: small rings let several CTAs (and so many warps, each
 // with copies in flight) share an SM.
@@ -127,7 +128,7 @@ struct basiskv_handle {
   int topk_keys = 0;  // scores staged in shared memory by the selection kernel
   int route_occ = 1, attn_occ = 1;  // resident CTAs per SM of the persistent kernels
   // profiling
-  std::vector<cudaEvent_t> events;  // 3 per recorded call
+  std::vector<cudaEvent_t> events;  // kProfEvents per recorded call
   int prof_cap = 0, prof_calls = 0;
   int last_launch[6] = {0, 0, 0, 0, 0, 0};
 };
@@ -173,7 +174,7 @@ void choose_kernels(basiskv_handle* h) {
   if (p.dtype != BASISKV_DTYPE_BF16) return;
   const size_t es = 2;
   auto rit = route_table().find(RouteKey{p.gqa_group, p.rank_r, p.rank_s, p.page_size});
-  if (rit != route_table().end() && p.page_size % 16 == 0 && p.head_dim % 32 == 0) {
+  if (rit != route_table().end() && p.page_size % 16 == 0 && (p.head_dim == 128 || p.head_dim == 64)) {
     const size_t stage = (size_t)p.page_size * (p.rank_r + p.rank_s) * es;
     int st = (int)std::min<size_t>(4, kRouteSmemBudget / (kRouteWarps * stage));
     if (st >= 2) {
@@ -207,8 +208,13 @@ size_t generic_attn_smem(const basiskv_params& p) {
   return sizeof(float) * std::max(own, combine_smem_floats(kMaxSplits, p.gqa_group, p.rank_r));
 }
 
+// Dynamic shared memory limit, and the largest shared-memory carveout: SMs
+// then keep one L1/shared split for all of this library's grids, so a grid
+// launched early (programmatic dependent launch) can share SMs with the one
+// still finishing.
 int set_smem_attr(const void* fn, size_t bytes) {
   CUDA_TRY(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
+  CUDA_TRY(cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared));
   return BASISKV_OK;
 }
 
@@ -701,32 +707,35 @@ int basiskv_decode_attn(basiskv_handle* h, int batch, const void* q, int topk, f
   cudaStream_t st = (cudaStream_t)stream;
   const LaunchPlan lp = plan(h, batch, topk, false);
   const bool prof = h->prof_calls < h->prof_cap;
-  cudaEvent_t* ev = prof ? &h->events[3 * h->prof_calls] : nullptr;
+  cudaEvent_t* ev = prof ? &h->events[kProfEvents * h->prof_calls] : nullptr;
   if (prof) CUDA_TRY(cudaEventRecord(ev[0], st));
   const bool route_tc = lp.any_routed && h->route_fn;
-  const bool use_prep = route_tc || h->attn_fn;
+  // the persistent grids read the work plan from their parameters; only a
+  // batch too large for that needs the prep grid to write it
+  const bool use_prep = (route_tc || h->attn_fn) && lp.route_off.empty();
   if (use_prep) {
     rc = launch_prep(h, lp, q, topk, 0, out, sel_out, nullptr, st);
     if (rc) return rc;
   }
+  if (prof) CUDA_TRY(cudaEventRecord(ev[1], st));
+  // the first grid of a call never overlaps the caller's previous work
   if (lp.any_routed) {
     RouteArgs ra = route_args(h, lp, q, topk, h->d_scores, sel_out, 0);
-    rc = launch_route(h, lp, ra, !prof, st);
+    rc = launch_route(h, lp, ra, use_prep && !prof, st);
     if (rc) return rc;
-    if (h->route_fn) {
-      rc = launch_topk(h, lp, topk, h->d_scores, sel_out, 0, !prof, st);
-      if (rc) return rc;
-    }
   }
-  if (prof) CUDA_TRY(cudaEventRecord(ev[1], st));
-  // PDL needs the plan complete when this grid starts: it is in the
-  // parameters, or a routing grid (which signals only after the prep grid
-  // finished) precedes this one
-  rc = launch_attn(h, lp, q, topk, softmax_scale, out, sel_out,
-                   use_prep && (!lp.attn_off.empty() || lp.any_routed) && !prof, st);
+  if (prof) CUDA_TRY(cudaEventRecord(ev[2], st));
+  if (route_tc) {
+    rc = launch_topk(h, lp, topk, h->d_scores, sel_out, 0, !prof, st);
+    if (rc) return rc;
+  }
+  if (prof) CUDA_TRY(cudaEventRecord(ev[3], st));
+  // PDL only behind a routing grid (which signals after any prep grid has
+  // finished, so the plan is complete when this grid starts)
+  rc = launch_attn(h, lp, q, topk, softmax_scale, out, sel_out, lp.any_routed && !prof, st);
   if (rc) return rc;
   if (prof) {
-    CUDA_TRY(cudaEventRecord(ev[2], st));
+    CUDA_TRY(cudaEventRecord(ev[4], st));
     ++h->prof_calls;
   }
   h->last_launch[0] = lp.any_routed ? (h->route_fn ? 0 : lp.route_ppc) : 0;
@@ -766,7 +775,8 @@ int basiskv_route(basiskv_handle* h, int batch, const void* q, int topk, float* 
   cudaStream_t st = (cudaStream_t)stream;
   const LaunchPlan lp = plan(h, batch, topk, true);
   float* scores = scores_out ? scores_out : h->d_scores;
-  // the prep grid writes -inf past n_b and the -1 rows of empty sequences
+  // the prep grid writes -inf past n_b, the -1 rows of empty sequences and,
+  // for large batches, the plan
   rc = launch_prep(h, lp, q, topk, 1, nullptr, sel_out, scores, st);
   if (rc) return rc;
   if (!lp.any_routed) return BASISKV_OK;
@@ -790,7 +800,7 @@ int basiskv_profile_begin(basiskv_handle* h, int max_calls) {
   int rc = check_handle(h);
   if (rc) return rc;
   if (max_calls < 0) return fail(BASISKV_ERR_INVALID_ARG, "max_calls < 0");
-  while ((int)h->events.size() < 3 * max_calls) {
+  while ((int)h->events.size() < kProfEvents * max_calls) {
     cudaEvent_t e;
     CUDA_TRY(cudaEventCreate(&e));
     h->events.push_back(e);
@@ -800,19 +810,15 @@ int basiskv_profile_begin(basiskv_handle* h, int max_calls) {
   return BASISKV_OK;
 }
 
-int basiskv_profile_end(basiskv_handle* h, float* route_ms, float* attn_ms, float* total_ms, int* ncalls) {
+int basiskv_profile_end(basiskv_handle* h, float* ms, int* ncalls) {
   int rc = check_handle(h);
   if (rc) return rc;
   for (int i = 0; i < h->prof_calls; ++i) {
-    cudaEvent_t* ev = &h->events[3 * i];
-    CUDA_TRY(cudaEventSynchronize(ev[2]));
-    float a = 0.f, b = 0.f, c = 0.f;
-    CUDA_TRY(cudaEventElapsedTime(&a, ev[0], ev[1]));
-    CUDA_TRY(cudaEventElapsedTime(&b, ev[1], ev[2]));
-    CUDA_TRY(cudaEventElapsedTime(&c, ev[0], ev[2]));
-    if (route_ms) route_ms[i] = a;
-    if (attn_ms) attn_ms[i] = b;
-    if (total_ms) total_ms[i] = c;
+    cudaEvent_t* ev = &h->events[kProfEvents * i];
+    CUDA_TRY(cudaEventSynchronize(ev[kProfEvents - 1]));
+    for (int k = 0; k + 1 < kProfEvents && ms; ++k)
+      CUDA_TRY(cudaEventElapsedTime(&ms[i * kProfEvents + k], ev[k], ev[k + 1]));
+    if (ms) CUDA_TRY(cudaEventElapsedTime(&ms[i * kProfEvents + kProfEvents - 1], ev[0], ev[kProfEvents - 1]));
   }
   if (ncalls) *ncalls = h->prof_calls;
   h->prof_cap = 0;

@@ -186,6 +186,106 @@ struct RouteCursor {
   __device__ __forceinline__ int unit(const RouteArgs& a) const { return b * a.num_kv_heads + kvh; }
 };
 
+// Route-prep inside the routing warp: fold W_zk and B_r of KV head kvh into
+// the G queries of sequence b (qz_h = W_zk.q_h, qr_h = B_r.q_h, fp32) and
+// return this lane's B-fragment words of the split (hi, lo) folded query.
+// Lanes own d/32 consecutive channels; for each block of 32/G basis rows a
+// lane forms its 32 partial (row, head) dot products and a butterfly
+// reduce-scatter (31 shuffles) leaves the sum of (row, head) = (lane/G,
+// lane%G) in lane; the sums meet in the warp's shared scratch `qsm`
+// ([G][r] then [G][s]) to be regrouped into fragment order.
+template <int G, int RR, int RS, int FR, int CPL>
+__device__ void warp_fold_query(const RouteArgs& a, int b, int kvh, float* qsm, uint32_t (&fr)[FR]) {
+  static_assert(32 % G == 0, "G must divide 32");
+  static_assert(CPL == 2 || CPL == 4, "head_dim 64 or 128");
+  constexpr int RPB = 32 / G;
+  constexpr int ROWS = RR + RS;
+  constexpr int d = 32 * CPL;
+  const int lane = threadIdx.x & 31;
+  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.num_kv_heads + kvh) * G * d +
+                           lane * CPL;
+  float qv[G][CPL];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) qv[h][j] = __bfloat162float(q[h * d + j]);
+  const float* W = a.w_zk + (size_t)kvh * RR * d + lane * CPL;
+  const float* Br = a.b_r + (size_t)kvh * RS * d + lane * CPL;
+#pragma unroll 1
+  for (int row0 = 0; row0 < ROWS; row0 += RPB) {
+    float v[32];
+#pragma unroll
+    for (int rl = 0; rl < RPB; ++rl) {
+      const int row = row0 + rl;
+      const float* src = row < RR ? W + (size_t)row * d : Br + (size_t)(row - RR) * d;
+      float w[CPL];
+      if constexpr (CPL == 4) {
+        const float4 x = row < ROWS ? __ldg(reinterpret_cast<const float4*>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        w[0] = x.x;
+        w[1] = x.y;
+        w[2] = x.z;
+        w[3] = x.w;
+      } else {
+        const float2 x = row < ROWS ? __ldg(reinterpret_cast<const float2*>(src)) : make_float2(0.f, 0.f);
+        w[0] = x.x;
+        w[1] = x.y;
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float acc = 0.f;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) acc = fmaf(w[j], qv[h][j], acc);
+        v[rl * G + h] = acc;
+      }
+    }
+#pragma unroll
+    for (int step = 16, cnt = 32; step >= 1; step >>= 1, cnt >>= 1) {
+      const bool upper = (lane & step) != 0;
+#pragma unroll
+      for (int k = 0; k < cnt / 2; ++k) {
+        const float send = upper ? v[k] : v[k + cnt / 2];
+        const float keep = upper ? v[k + cnt / 2] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, step);
+      }
+    }
+    const int row = row0 + lane / G, h = lane % G;
+    if (row < RR) qsm[h * RR + row] = v[0];
+    else if (row < ROWS) qsm[G * RR + h * RS + (row - RR)] = v[0];
+  }
+  __syncwarp();
+  // regroup into this lane's fragment words (same order as the kernel reads)
+  using Shape = RouteMma<G, RR, RS>;
+  const int g = lane >> 2, t = lane & 3;
+  int w = 0;
+#pragma unroll
+  for (int j = 0; j < Shape::NT; ++j) {
+    const int hh = 4 * j + (g >> 1);
+    const bool lo = g & 1;
+    const float* qz = qsm + hh * RR;
+    const float* qr = qsm + G * RR + hh * RS;
+    auto word = [&](const float* src, int e) {
+      if (hh >= G) return 0u;
+      float h0, l0, h1, l1;
+      split_bf16(src[e], h0, l0);
+      split_bf16(src[e + 1], h1, l1);
+      return lo ? pack_bf16(l0, l1) : pack_bf16(h0, h1);
+    };
+#pragma unroll
+    for (int blk = 0; blk < Shape::ZB; ++blk) {
+      fr[w++] = word(qz, k16_phys<Shape::Z32, Shape::Z16>(blk, t, 0));
+      fr[w++] = word(qz, k16_phys<Shape::Z32, Shape::Z16>(blk, t, 1));
+    }
+    if (Shape::Z8) fr[w++] = word(qz, 32 * Shape::Z32 + 16 * Shape::Z16 + 2 * t);
+#pragma unroll
+    for (int blk = 0; blk < Shape::SB; ++blk) {
+      fr[w++] = word(qr, k16_phys<Shape::S32, Shape::S16>(blk, t, 0));
+      fr[w++] = word(qr, k16_phys<Shape::S32, Shape::S16>(blk, t, 1));
+    }
+    if (Shape::S8) fr[w++] = word(qr, 32 * Shape::S32 + 16 * Shape::S16 + 2 * t);
+  }
+  __syncwarp();
+}
+
 template <int G, int RR, int RS, int P>
 __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_constant__ RouteArgs a) {
   using Shape = RouteMma<G, RR, RS>;
@@ -199,15 +299,17 @@ __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_c
 
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t bars[kRouteWarps][kMaxStages];
+  __shared__ float qsm_all[kRouteWarps][G * (RR + RS)];
+  float* qsm = qsm_all[warp];
   uint8_t* ring = smem + (size_t)warp * S * stage_bytes;
   if (lane == 0) {
     for (int i = 0; i < S; ++i) mbar_init(&bars[warp][i], 1);
     mbar_init_fence();
   }
   __syncwarp();
-  // The plan comes in the parameters (small batches) or from the prep grid.
-  // With the plan in hand the first copies go out before the prep grid has
-  // finished folding the query.
+  // The plan comes in the parameters (small batches) or from the prep grid
+  // (then this grid waits for it first).  The query is folded by the warp
+  // itself once its first copies are in flight.
   const int32_t* offsets = a.plan_n >= 0 ? a.plan_off : a.route_off;
   if (a.plan_n < 0) pdl_wait_primary();
 
@@ -253,7 +355,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_c
       if (lane == 0) issue(i, sli);
     }
   }
-  if (a.plan_n >= 0) pdl_wait_primary();  // query fragments
   pdl_launch_dependents();
   if (count <= 0) return;
 
@@ -267,11 +368,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_c
     int next_slot = 0;
     if (lane == 0 && i + S < count) next_slot = lookup();
     const int u = cc.unit(a);
-    if (u != cur_u) {
+    if (u != cur_u) {  // fold this unit's query while its copies are in flight
       cur_u = u;
-      const uint32_t* src = a.qfrag + (size_t)u * a.frag_words * 32 + lane;
-#pragma unroll
-      for (int w = 0; w < FR; ++w) fr[w] = __ldcg(src + w * 32);
+      if (a.head_dim == 128) warp_fold_query<G, RR, RS, FR, 4>(a, cc.b, cc.kvh, qsm, fr);
+      else warp_fold_query<G, RR, RS, FR, 2>(a, cc.b, cc.kvh, qsm, fr);
     }
     ok = mbar_wait(&bars[warp][i % S], (uint32_t)((i / S) & 1), a.status);
     ok = __all_sync(0xffffffffu, ok);

@@ -179,13 +179,14 @@ BASISKV_API int basiskv_route(basiskv_handle *h, int batch, const void *q, int t
 BASISKV_API int basiskv_get_status(basiskv_handle *h, uint32_t *status, int clear);
 
 /* Kernel timing: after basiskv_profile_begin(h, n), the next n decode calls
- * record CUDA events on their stream around the routing and the attention
- * kernel.  basiskv_profile_end waits for them and writes per-call
- * milliseconds into route_ms[i] / attn_ms[i] / total_ms[i] (host arrays of
- * length >= n, nullable) and the number of recorded calls into *ncalls. */
+ * record CUDA events on their stream around each grid (the events keep the
+ * grids from overlapping, so profiled calls run a little slower).
+ * basiskv_profile_end waits for them and writes, per recorded call i,
+ * ms[5*i + 0..4] = prep grid, routing grid, selection grid, attention grid,
+ * whole call, in milliseconds (host array of >= 5*n floats, nullable), and
+ * the number of recorded calls into *ncalls. */
 BASISKV_API int basiskv_profile_begin(basiskv_handle *h, int max_calls);
-BASISKV_API int basiskv_profile_end(basiskv_handle *h, float *route_ms, float *attn_ms,
-                        float *total_ms, int *ncalls);
+BASISKV_API int basiskv_profile_end(basiskv_handle *h, float *ms, int *ncalls);
 
 /* Launch shape chosen for the last decode call (for reports): routing pages
  * per CTA and CTA count, attention splits per unit and CTA count, and
