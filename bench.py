@@ -81,6 +81,19 @@ def barrier(world, device=None):
             dist.barrier()
 
 
+def replica_spec(spec, rank: int):
+    """Rank r of a multi-GPU run processes its own replica of the workload
+    (weak scaling): same shapes, its own seed."""
+    return spec.with_(seed=spec.seed + 1000 * rank) if rank else spec
+
+
+def aggregate(tokens_per_rank: int, ms_per_step: float, world: int, device=None):
+    """Whole-job throughput: every rank's tokens over the slowest rank's step
+    time.  Returns (value, max ms per step)."""
+    ms_max = max_over_ranks(ms_per_step, world, device)
+    return tokens_per_rank * world / (ms_max * 1e-3), ms_max
+
+
 def peaks():
     try:
         with open(PEAKS_PATH) as f:
@@ -265,8 +278,7 @@ def run_ours(args, rank, world, local):
     spec = W.SPECS[args.workload]
     if args.batch:
         spec = spec.with_(batch=args.batch)
-    if rank:
-        spec = spec.with_(seed=spec.seed + 1000 * rank)
+    spec = replica_spec(spec, rank)
     w = W.generate(spec, device=dev)
     kv = bk.BasisKV.for_workload(w)
     s = w.spec
@@ -318,9 +330,8 @@ def run_ours(args, rank, world, local):
     launch = bk.basiskv_last_launch(kv.handle)
 
     ms_step = float(np.mean(step_ms))
-    ms_step_max = max_over_ranks(ms_step, world, dev)
     tokens = w.context_tokens
-    value = tokens * world / (ms_step_max * 1e-3)
+    value, ms_step_max = aggregate(tokens, ms_step, world, dev)
     nbytes = w.algorithmic_bytes()
     hbm_peak, peak_kind = peaks()
     route_mean = float(np.mean(prof["route"])) if launch["route_ctas"] else 0.0
