@@ -4,15 +4,17 @@
 // Key-specific residual stores what cannot be recovered from Value").
 //
 // Routing key  Khat_t = Z_t.W_zk + R_t.B_r  is never formed: the kernels fold
-// the bases into the query once per CTA (route-prep),
+// the bases into the query (route-prep),
 //     qz_h = W_zk.q_h  (r floats),   qr_h = B_r.q_h  (s floats),
 // so that  q_h.Khat_t = Z_t.qz_h + R_t.qr_h  costs r + s multiply-adds per
 // token and head and reads only the r + s stored values of each token.
-// Page score S_j = max over the G heads and page j's valid tokens; the last
-// CTA of each (sequence, KV head) runs the top-k over the page scores.
+// Page score S_j = max over the G heads and page j's valid tokens.
 //
-// Grid: (chunks of pages, Hkv, batch); each CTA owns pages
-// [chunk*ppc, min((chunk+1)*ppc, n_b)) of one (sequence, KV head).
+// Two kernels: route_mma_kernel (bf16 pools, tensor cores, persistent over a
+// flat page list, the fold done by each warp as it enters a (sequence, KV
+// head); the selection runs in the next grid) and route_generic_kernel (any
+// dtype, grid (chunks of pages, Hkv, batch), fold once per CTA, the last CTA
+// of each (sequence, KV head) runs the top-k).
 #pragma once
 
 #include "common.cuh"
