@@ -342,6 +342,9 @@ def run_ours(args, rank, world, local):
     else:
         dom_bytes, dom_ms = nbytes["attn"], attn_mean
         kname = "attn_mma_kernel" if launch["attn_tensor_core"] else "attn_generic_kernel"
+    # routing (+ its selection grid on the tensor-core path), attention, prep past 512 sequences
+    launches_per_step = (1 + launch["route_tensor_core"] if launch["route_ctas"] else 0) + 1 + \
+        (1 if s.batch > 512 else 0)
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     traffic = ncu_traffic(kname, args.workload)
 
@@ -396,7 +399,7 @@ def run_ours(args, rank, world, local):
             "kernels_ms_note": "second K-step loop, events between grids (no PDL overlap there)",
             "step_ms_p10_p50_p90": [float(np.percentile(step_ms, q)) for q in (10, 50, 90)],
             "launch": launch,
-            "gpu_launches": K * ((1 if launch["route_ctas"] else 0) + 1),
+            "gpu_launches": K * launches_per_step,
             "e2e": {"value": tokens * world / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_s * 1e3,
                     "how": "basiskv_decode_attn_host: pinned q H2D, decode, out+sel D2H, stream sync; host wall clock"},
