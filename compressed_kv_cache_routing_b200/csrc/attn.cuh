@@ -347,9 +347,10 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
     }
     last = __shfl_sync(0xffffffffu, last, 0);
     if (last) {
-      warp_combine<G, RR, D>(a.part_ml + (size_t)u * a.np_cap * G * 2,
-                             a.part_acc + (size_t)u * a.np_cap * G * RR, min(np, a.np_cap),
-                             a.b_v + (size_t)at.kvh * RR * D, a.out + (size_t)u * G * D, zbar);
+      MergeOut<G, RR> mo;
+      merge_all<G, RR>(a.part_ml + (size_t)u * a.np_cap * G * 2, a.part_acc + (size_t)u * a.np_cap * G * RR,
+                       min(np, a.np_cap), mo);
+      finish_unit<G, RR, D>(mo, a.b_v + (size_t)at.kvh * RR * D, a.out + (size_t)u * G * D, zbar);
       if (lane == 0) a.counters[u] = 0u;
     }
   };
