@@ -106,6 +106,9 @@ struct basiskv_handle {
   float* d_part_ml = nullptr;       // [max_batch*Hkv][kPartsCap][G][2]
   float* d_part_acc = nullptr;      // [max_batch*Hkv][kPartsCap][G][r]
   uint32_t* d_counters = nullptr;   // [3][max_batch*Hkv]: route, attention, partial count
+  float* d_qf = nullptr;            // [max_batch*Hkv][G][r+s] folded routing queries
+  uint32_t* d_fold_flag = nullptr;  // [max_batch*Hkv][32] tag of the call that wrote each fold slice
+  uint32_t route_tag = 0;           // tag of the last routing launch
   uint32_t* d_status = nullptr;
   int32_t* d_route_off = nullptr;   // [max_batch+1]
   int32_t* d_attn_off = nullptr;    // [max_batch+1]
@@ -376,6 +379,10 @@ RouteArgs route_args(basiskv_handle* h, const LaunchPlan& lp, const void* q, int
   a.route_off = h->d_route_off;
   a.qfrag = h->d_qfrag;
   a.frag_words = h->frag_words;
+  a.qf = h->d_qf;
+  a.fold_flag = h->d_fold_flag;
+  if (++h->route_tag == 0) h->route_tag = 1;  // 0 never matches: the flags start zeroed
+  a.tag = h->route_tag;
   a.plan_n = lp.route_off.empty() ? -1 : lp.batch;
   for (size_t i = 0; i < lp.route_off.size(); ++i) a.plan_off[i] = lp.route_off[i];
   return a;
@@ -547,6 +554,8 @@ int basiskv_create(const basiskv_params* p, basiskv_handle** out) {
       {(void**)&h->d_part_ml, sizeof(float) * U * kPartsCap * G * 2},
       {(void**)&h->d_part_acc, sizeof(float) * U * kPartsCap * G * p->rank_r},
       {(void**)&h->d_counters, sizeof(uint32_t) * 3 * U},
+      {(void**)&h->d_qf, sizeof(float) * U * G * (p->rank_r + p->rank_s)},
+      {(void**)&h->d_fold_flag, sizeof(uint32_t) * U * 32},
       {(void**)&h->d_status, sizeof(uint32_t)},
       {(void**)&h->d_route_off, sizeof(int32_t) * (B + 1)},
       {(void**)&h->d_attn_off, sizeof(int32_t) * (B + 1)},
@@ -565,6 +574,7 @@ int basiskv_create(const basiskv_params* p, basiskv_handle** out) {
   if (cudaMemset(h->d_page_table, 0, sizeof(int32_t) * B * p->max_pages_per_seq) != cudaSuccess ||
       cudaMemset(h->d_seq_lens, 0, sizeof(int32_t) * B) != cudaSuccess ||
       cudaMemset(h->d_counters, 0, sizeof(uint32_t) * 3 * U) != cudaSuccess ||
+      cudaMemset(h->d_fold_flag, 0, sizeof(uint32_t) * U * 32) != cudaSuccess ||
       cudaMemset(h->d_status, 0, sizeof(uint32_t)) != cudaSuccess)
     return cleanup_fail(BASISKV_ERR_CUDA, "cudaMemset failed");
   h->h_table.assign(B * p->max_pages_per_seq, 0);
@@ -606,7 +616,7 @@ int basiskv_destroy(basiskv_handle* h) {
   cudaDeviceSynchronize();
   void* ptrs[] = {h->d_page_table, h->d_seq_lens, h->d_scores, h->d_sel, h->d_part_ml, h->d_part_acc,
                   h->d_counters, h->d_status, h->d_q_stage, h->d_out_stage, h->d_sel_stage,
-                  h->d_route_off, h->d_attn_off, h->d_qfrag};
+                  h->d_route_off, h->d_attn_off, h->d_qfrag, h->d_qf, h->d_fold_flag};
   for (void* q : ptrs)
     if (q) cudaFree(q);
   for (cudaEvent_t e : h->events) cudaEventDestroy(e);

@@ -75,6 +75,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   }
 }
 
+// Wait (acquire) until *flag == tag, for at most limit_ns; false on expiry.
+// Polls back off so that many waiters do not flood one L2 line.
+constexpr uint64_t kFoldWaitNs = 50000ull;
+__device__ __forceinline__ bool wait_tag(const uint32_t* flag, uint32_t tag, uint64_t limit_ns) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+  if (v == tag) return true;
+  const uint64_t t0 = global_timer_ns();
+  uint32_t pause = 32;
+  for (;;) {
+    __nanosleep(pause);
+    pause = pause < 1024u ? 2 * pause : 1024u;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v == tag) return true;
+    if (global_timer_ns() - t0 > limit_ns) return false;
+  }
+}
+
 // ---- bulk copy global -> shared (TMA unit, non-tensor form) -----------------
 // dst, src 16-byte aligned, bytes a multiple of 16.  Completion is reported
 // as transaction bytes on `bar`.  `policy` is an L2 cache policy descriptor.

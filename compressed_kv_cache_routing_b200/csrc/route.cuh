@@ -46,6 +46,9 @@ struct RouteArgs {
   const int32_t* route_off; // [B+1] prefix of routed pages x Hkv (from the prep grid)
   const uint32_t* qfrag;    // [B*Hkv][frag_words][32] query B fragments
   int frag_words;
+  float* qf;                // [B*Hkv][G][r+s] folded queries (fp32)
+  uint32_t* fold_flag;      // [B*Hkv][32] per fold slice: the tag of the call that wrote it
+  uint32_t tag;             // this call's tag (never 0)
   int plan_n;               // >= 0: plan_off holds route_off (batch <= kPlanMax)
   int32_t plan_off[kPlanMax + 1];
 };
@@ -288,6 +291,101 @@ __device__ void warp_fold_query(const RouteArgs& a, int b, int kvh, float* qsm, 
   __syncwarp();
 }
 
+// Route-prep, spread over the routing warps: one fold slice each.
+// Rows [slice*32/G, +32/G) of [W_zk; B_r] of unit u's KV head times the G
+// queries: lanes own d/32 consecutive channels, each forms its 32 partial
+// (row, head) products and a butterfly reduce-scatter (31 shuffles) leaves
+// the full sum of (row, head) = (lane/G, lane%G) in the lane.
+template <int G, int RR, int RS, int CPL>
+__device__ void fold_slice(const RouteArgs& a, int u, int slice) {
+  constexpr int RPB = 32 / G, ROWS = RR + RS, d = 32 * CPL;
+  const int lane = threadIdx.x & 31;
+  const int kvh = u % a.num_kv_heads;
+  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q) + (size_t)u * G * d + lane * CPL;
+  float qv[G][CPL];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) qv[h][j] = __bfloat162float(q[h * d + j]);
+  const int row0 = slice * RPB;
+  float v[32];
+#pragma unroll
+  for (int rl = 0; rl < RPB; ++rl) {
+    const int row = row0 + rl;
+    const float* src = row < RR ? a.w_zk + ((size_t)kvh * RR + row) * d
+                                : a.b_r + ((size_t)kvh * RS + (row - RR)) * d;
+    src += lane * CPL;
+    float w[CPL];
+    if constexpr (CPL == 4) {
+      const float4 x = row < ROWS ? __ldg(reinterpret_cast<const float4*>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      w[0] = x.x;
+      w[1] = x.y;
+      w[2] = x.z;
+      w[3] = x.w;
+    } else {
+      const float2 x = row < ROWS ? __ldg(reinterpret_cast<const float2*>(src)) : make_float2(0.f, 0.f);
+      w[0] = x.x;
+      w[1] = x.y;
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float acc = 0.f;
+#pragma unroll
+      for (int j = 0; j < CPL; ++j) acc = fmaf(w[j], qv[h][j], acc);
+      v[rl * G + h] = acc;
+    }
+  }
+#pragma unroll
+  for (int step = 16, cnt = 32; step >= 1; step >>= 1, cnt >>= 1) {
+    const bool upper = (lane & step) != 0;
+#pragma unroll
+    for (int k = 0; k < cnt / 2; ++k) {
+      const float send = upper ? v[k] : v[k + cnt / 2];
+      const float keep = upper ? v[k + cnt / 2] : v[k];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, step);
+    }
+  }
+  const int row = row0 + lane / G, h = lane % G;
+  if (row < ROWS) a.qf[((size_t)u * G + h) * ROWS + row] = v[0];
+}
+
+// This lane's routing B-fragment words for unit u, from the folded query
+// (split into bf16 hi + lo columns; same order as route_mma_kernel), read
+// from global memory (written by other warps of this grid: read through L2).
+template <int G, int RR, int RS, int FR>
+__device__ void load_route_frags(const float* qfu, uint32_t (&fr)[FR]) {
+  using Shape = RouteMma<G, RR, RS>;
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  int w = 0;
+#pragma unroll
+  for (int j = 0; j < Shape::NT; ++j) {
+    const int hh = 4 * j + (g >> 1);
+    const bool lo = g & 1;
+    const float* qz = qfu + hh * (RR + RS);
+    const float* qr = qz + RR;
+    auto word = [&](const float* src, int e) {
+      if (hh >= G) return 0u;
+      const float2 x = __ldcg(reinterpret_cast<const float2*>(src + e));
+      float h0, l0, h1, l1;
+      split_bf16(x.x, h0, l0);
+      split_bf16(x.y, h1, l1);
+      return lo ? pack_bf16(l0, l1) : pack_bf16(h0, h1);
+    };
+#pragma unroll
+    for (int blk = 0; blk < Shape::ZB; ++blk) {
+      fr[w++] = word(qz, k16_phys<Shape::Z32, Shape::Z16>(blk, t, 0));
+      fr[w++] = word(qz, k16_phys<Shape::Z32, Shape::Z16>(blk, t, 1));
+    }
+    if (Shape::Z8) fr[w++] = word(qz, 32 * Shape::Z32 + 16 * Shape::Z16 + 2 * t);
+#pragma unroll
+    for (int blk = 0; blk < Shape::SB; ++blk) {
+      fr[w++] = word(qr, k16_phys<Shape::S32, Shape::S16>(blk, t, 0));
+      fr[w++] = word(qr, k16_phys<Shape::S32, Shape::S16>(blk, t, 1));
+    }
+    if (Shape::S8) fr[w++] = word(qr, 32 * Shape::S32 + 16 * Shape::S16 + 2 * t);
+  }
+}
+
 template <int G, int RR, int RS, int P>
 __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_constant__ RouteArgs a) {
   using Shape = RouteMma<G, RR, RS>;
@@ -358,6 +456,24 @@ __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_c
     }
   }
   pdl_launch_dependents();
+
+  // route-prep spread over the warps: task (unit, slice) -> warp task mod W;
+  // each writes its rows of the folded query and tags them with the call
+  constexpr int NSL = (RR + RS + 32 / G - 1) / (32 / G);
+  static_assert(NSL <= 32, "fold slices per unit must fit a warp");
+  const int U = a.batch * a.num_kv_heads;
+  for (int task = wg; task < U * NSL; task += W) {
+    const int u = task / NSL;
+    const int n = (a.seq_lens[u / a.num_kv_heads] + P - 1) / P;
+    if (n == 0 || !(a.force || a.topk < n)) continue;
+    if (a.head_dim == 128) fold_slice<G, RR, RS, 4>(a, u, task % NSL);
+    else fold_slice<G, RR, RS, 2>(a, u, task % NSL);
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence();
+      *reinterpret_cast<volatile uint32_t*>(a.fold_flag + (size_t)u * 32 + task % NSL) = a.tag;
+    }
+  }
   if (count <= 0) return;
 
   constexpr int FR = NT * (2 * Shape::ZB + Shape::Z8 + 2 * Shape::SB + Shape::S8);
@@ -370,10 +486,19 @@ __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_c
     int next_slot = 0;
     if (lane == 0 && i + S < count) next_slot = lookup();
     const int u = cc.unit(a);
-    if (u != cur_u) {  // fold this unit's query while its copies are in flight
+    if (u != cur_u) {
+      // this unit's folded query: its slices come from other warps; should
+      // they be late (their CTA not yet resident), fold it here instead
       cur_u = u;
-      if (a.head_dim == 128) warp_fold_query<G, RR, RS, FR, 4>(a, cc.b, cc.kvh, qsm, fr);
-      else warp_fold_query<G, RR, RS, FR, 2>(a, cc.b, cc.kvh, qsm, fr);
+      bool ready = true;
+      if (lane < NSL) ready = wait_tag(a.fold_flag + (size_t)u * 32 + lane, a.tag, kFoldWaitNs);
+      if (__all_sync(0xffffffffu, ready)) {
+        load_route_frags<G, RR, RS, FR>(a.qf + (size_t)u * G * (RR + RS), fr);
+      } else if (a.head_dim == 128) {
+        warp_fold_query<G, RR, RS, FR, 4>(a, cc.b, cc.kvh, qsm, fr);
+      } else {
+        warp_fold_query<G, RR, RS, FR, 2>(a, cc.b, cc.kvh, qsm, fr);
+      }
     }
     ok = mbar_wait(&bars[warp][i % S], (uint32_t)((i / S) & 1), a.status);
     ok = __all_sync(0xffffffffu, ok);
