@@ -183,6 +183,21 @@ def test_topk_one_and_max():
         assert out_error(out, ref_out) <= OUT_TOL
 
 
+def test_units_with_many_pages():
+    """More than 2048 pages per unit, with exact ties in one sequence."""
+    spec = W.shrink("llama3_8b_decode", batch=2, len_lo=2100 * 16, len_hi=2100 * 16 + 15, topk=40, page_size=16)
+    w = W.generate(spec, device="cuda")
+    pt = w.page_table.copy()
+    pt[1, :] = pt[1, np.arange(pt.shape[1]) % 5]     # five distinct pages, repeated: ties everywhere
+    w.page_table = pt
+    prob = to_problem(w)
+    ref_out, ref_sel, _, _ = oracle.decode(prob)
+    assert w.num_pages.min() > 2048
+    out, sel = gpu_decode(w)
+    assert np.array_equal(sel, ref_sel)
+    assert out_error(out, ref_out) <= OUT_TOL
+
+
 def test_exact_ties_go_to_lower_page():
     """Logical pages sharing a physical slot score exactly the same."""
     spec = W.shrink("llama3_8b_decode", batch=2, len_lo=64 * 40, len_hi=64 * 40, topk=6)
