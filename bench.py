@@ -94,6 +94,16 @@ def aggregate(tokens_per_rank: int, ms_per_step: float, world: int, device=None)
     return tokens_per_rank * world / (ms_max * 1e-3), ms_max
 
 
+def workload_config(args, w, world):
+    """The workload part of the JSON line's config, the same for both arms."""
+    s = w.spec
+    return {"workload": args.workload if not args.batch else f"{args.workload}[batch={s.batch}]",
+            "batch": s.batch, "kv_heads": s.num_kv_heads, "q_heads": s.num_q_heads, "head_dim": s.head_dim,
+            "page": s.page_size, "rank_r": s.rank_r, "rank_s": s.rank_s, "topk": s.topk,
+            "context_tokens": w.context_tokens, "algorithmic_bytes": w.algorithmic_bytes()["total"],
+            "parallelism": f"replicas x{world}, no data-path collective"}
+
+
 def peaks():
     try:
         with open(PEAKS_PATH) as f:
@@ -222,6 +232,8 @@ def run_reference(args, rank, world):
     from compressed_kv_cache_routing_b200 import workloads as W
     from oracle import oracle
     spec = W.SPECS[args.workload]
+    if args.batch:
+        spec = spec.with_(batch=args.batch)
     w = W.generate(spec, device="cuda" if torch.cuda.is_available() else "cpu")
     prob = oracle_problem(w)
     cores = oracle.max_threads()
@@ -255,7 +267,10 @@ def run_reference(args, rank, world):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload}, "impl": "reference",
+            "config": {**workload_config(args, w, world),
+                       "l2": "host run; the oracle reads host memory",
+                       "timing": "host wall clock around each step, mean of K steps"},
+            "impl": "reference",
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -379,14 +394,9 @@ def run_ours(args, rank, world, local):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_step_max, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": s.dtype, "data": "synthetic",
-            "config": {"workload": args.workload if not args.batch else f"{args.workload}[batch={s.batch}]",
-                       "batch": s.batch, "kv_heads": s.num_kv_heads,
-                       "q_heads": s.num_q_heads, "head_dim": s.head_dim, "page": s.page_size,
-                       "rank_r": s.rank_r, "rank_s": s.rank_s, "topk": s.topk,
-                       "context_tokens": tokens, "algorithmic_bytes": nbytes["total"],
+            "config": {**workload_config(args, w, world),
                        "l2": "flushed between steps (2x L2 write, outside the per-step events)",
-                       "timing": "CUDA event pair around each call on the launching stream, mean of K steps",
-                       "parallelism": f"replicas x{world}, no data-path collective"},
+                       "timing": "CUDA event pair around each call on the launching stream, mean of K steps"},
             "hbm": {"achieved_gbs": nbytes["total"] / (ms_step_max * 1e-3) / 1e9, "peak_gbs": hbm_peak,
                     "frac": nbytes["total"] / (ms_step_max * 1e-3) / 1e9 / hbm_peak,
                     "frac_of_8tbs": nbytes["total"] / (ms_step_max * 1e-3) / 8e12, "peak_kind": peak_kind},

@@ -112,8 +112,6 @@ struct basiskv_handle {
   uint32_t* d_status = nullptr;
   int32_t* d_route_off = nullptr;   // [max_batch+1]
   int32_t* d_attn_off = nullptr;    // [max_batch+1]
-  uint32_t* d_qfrag = nullptr;      // [max_batch*Hkv][frag_words][32]
-  int frag_words = 0;
   // host-buffer entry point staging
   void* d_q_stage = nullptr;
   float* d_out_stage = nullptr;
@@ -127,7 +125,7 @@ struct basiskv_handle {
   AttnFn attn_fn = nullptr;
   int attn_tps = 0;
   int route_stages = 0, attn_stages = 0;
-  size_t route_smem = 0, attn_smem = 0, prep_smem = 0;
+  size_t route_smem = 0, attn_smem = 0;
   int topk_keys = 0;  // scores staged in shared memory by the selection kernel
   int route_occ = 1, attn_occ = 1;  // resident CTAs per SM of the persistent kernels
   // profiling
@@ -309,17 +307,13 @@ LaunchPlan plan(const basiskv_handle* h, int batch, int topk, bool force_route) 
   return lp;
 }
 
-int launch_prep(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk, int force, float* out,
-                int32_t* sel_out, float* fill_scores, cudaStream_t stream) {
+int launch_prep(basiskv_handle* h, const LaunchPlan& lp, int topk, int force, float* out, int32_t* sel_out,
+                float* fill_scores, cudaStream_t stream) {
   const basiskv_params& p = h->p;
   PrepArgs a;
-  a.q = q;
-  a.w_zk = p.w_zk;
-  a.b_r = p.b_r;
   a.seq_lens = h->d_seq_lens;
   a.route_off = h->d_route_off;
   a.attn_off = h->d_attn_off;
-  a.qfrag = h->d_qfrag;
   a.sel_out = sel_out;
   a.out = out;
   a.scores = fill_scores;
@@ -328,19 +322,12 @@ int launch_prep(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk
   a.gqa_group = p.gqa_group;
   a.head_dim = p.head_dim;
   a.page_size = p.page_size;
-  a.rank_r = p.rank_r;
-  a.rank_s = p.rank_s;
   a.topk = topk;
   a.force = force;
   a.attn_sub = lp.sub;
   a.ld_pt = p.max_pages_per_seq;
-  a.fr = h->frag_words;
   a.fill_scores = fill_scores != nullptr;
-  dim3 grid(p.num_kv_heads, lp.batch);
-  if (p.dtype == BASISKV_DTYPE_BF16)
-    prep_kernel<__nv_bfloat16><<<grid, kPrepThreads, h->prep_smem, stream>>>(a);
-  else
-    prep_kernel<float><<<grid, kPrepThreads, h->prep_smem, stream>>>(a);
+  prep_kernel<<<dim3(p.num_kv_heads, lp.batch), kPrepThreads, 0, stream>>>(a);
   CUDA_TRY(cudaGetLastError());
   return BASISKV_OK;
 }
@@ -377,8 +364,6 @@ RouteArgs route_args(basiskv_handle* h, const LaunchPlan& lp, const void* q, int
   a.fill_tail = force;
   a.batch = lp.batch;
   a.route_off = h->d_route_off;
-  a.qfrag = h->d_qfrag;
-  a.frag_words = h->frag_words;
   a.qf = h->d_qf;
   a.fold_flag = h->d_fold_flag;
   if (++h->route_tag == 0) h->route_tag = 1;  // 0 never matches: the flags start zeroed
@@ -559,8 +544,6 @@ int basiskv_create(const basiskv_params* p, basiskv_handle** out) {
       {(void**)&h->d_status, sizeof(uint32_t)},
       {(void**)&h->d_route_off, sizeof(int32_t) * (B + 1)},
       {(void**)&h->d_attn_off, sizeof(int32_t) * (B + 1)},
-      {(void**)&h->d_qfrag, sizeof(uint32_t) * U * 32 *
-                                (size_t)FragGeom(p->gqa_group, p->rank_r, p->rank_s).words()},
       {(void**)&h->d_q_stage, h->elem * B * Hkv * G * p->head_dim},
       {(void**)&h->d_out_stage, sizeof(float) * B * Hkv * G * p->head_dim},
       {(void**)&h->d_sel_stage, sizeof(int32_t) * U * p->max_topk},
@@ -581,15 +564,12 @@ int basiskv_create(const basiskv_params* p, basiskv_handle** out) {
   h->h_lens.assign(B, 0);
   h->h_npages.assign(B, 0);
 
-  h->frag_words = FragGeom(p->gqa_group, p->rank_r, p->rank_s).words();
   h->topk_keys = std::min(p->max_pages_per_seq, 16384);
-  h->prep_smem = sizeof(float) * (size_t)p->gqa_group * (p->head_dim + p->rank_r + p->rank_s);
   choose_kernels(h);
   int arc = h->route_fn ? set_smem_attr((const void*)h->route_fn, h->route_smem) : BASISKV_OK;
   if (!arc && h->attn_fn) arc = set_smem_attr((const void*)h->attn_fn, h->attn_smem);
   if (!arc)
-    arc = p->dtype == BASISKV_DTYPE_BF16 ? set_smem_attr((const void*)&prep_kernel<__nv_bfloat16>, h->prep_smem)
-                                         : set_smem_attr((const void*)&prep_kernel<float>, h->prep_smem);
+    arc = set_smem_attr((const void*)&prep_kernel, 0);
   if (!arc) arc = set_smem_attr((const void*)&topk_kernel, sizeof(uint32_t) * (size_t)h->topk_keys);
   if (!arc && h->route_fn &&
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&h->route_occ, h->route_fn, kRouteThreads, h->route_smem) != cudaSuccess)
@@ -616,7 +596,7 @@ int basiskv_destroy(basiskv_handle* h) {
   cudaDeviceSynchronize();
   void* ptrs[] = {h->d_page_table, h->d_seq_lens, h->d_scores, h->d_sel, h->d_part_ml, h->d_part_acc,
                   h->d_counters, h->d_status, h->d_q_stage, h->d_out_stage, h->d_sel_stage,
-                  h->d_route_off, h->d_attn_off, h->d_qfrag, h->d_qf, h->d_fold_flag};
+                  h->d_route_off, h->d_attn_off, h->d_qf, h->d_fold_flag};
   for (void* q : ptrs)
     if (q) cudaFree(q);
   for (cudaEvent_t e : h->events) cudaEventDestroy(e);
@@ -724,7 +704,7 @@ int basiskv_decode_attn(basiskv_handle* h, int batch, const void* q, int topk, f
   // batch too large for that needs the prep grid to write it
   const bool use_prep = (route_tc || h->attn_fn) && lp.route_off.empty();
   if (use_prep) {
-    rc = launch_prep(h, lp, q, topk, 0, out, sel_out, nullptr, st);
+    rc = launch_prep(h, lp, topk, 0, out, sel_out, nullptr, st);
     if (rc) return rc;
   }
   if (prof) CUDA_TRY(cudaEventRecord(ev[1], st));
@@ -787,7 +767,7 @@ int basiskv_route(basiskv_handle* h, int batch, const void* q, int topk, float* 
   float* scores = scores_out ? scores_out : h->d_scores;
   // the prep grid writes -inf past n_b, the -1 rows of empty sequences and,
   // for large batches, the plan
-  rc = launch_prep(h, lp, q, topk, 1, nullptr, sel_out, scores, st);
+  rc = launch_prep(h, lp, topk, 1, nullptr, sel_out, scores, st);
   if (rc) return rc;
   if (!lp.any_routed) return BASISKV_OK;
   RouteArgs ra = route_args(h, lp, q, topk, scores, sel_out, 1);

@@ -44,8 +44,6 @@ struct RouteArgs {
   // persistent tensor-core kernel only
   int batch;
   const int32_t* route_off; // [B+1] prefix of routed pages x Hkv (from the prep grid)
-  const uint32_t* qfrag;    // [B*Hkv][frag_words][32] query B fragments
-  int frag_words;
   float* qf;                // [B*Hkv][G][r+s] folded queries (fp32)
   uint32_t* fold_flag;      // [B*Hkv][32] per fold slice: the tag of the call that wrote it
   uint32_t tag;             // this call's tag (never 0)

@@ -198,6 +198,18 @@ def test_units_with_many_pages():
     assert out_error(out, ref_out) <= OUT_TOL
 
 
+def test_batch_past_the_parameter_plan():
+    """More than 512 sequences: the work plan is written by the prep grid
+    instead of travelling in the kernel parameters."""
+    spec = W.shrink("llama3_8b_decode", batch=600, len_lo=1, len_hi=400, topk=3)
+    w = W.generate(spec, device="cuda")
+    prob = to_problem(w)
+    ref_out, ref_sel, _, _ = oracle.decode(prob)
+    out, sel = gpu_decode(w)
+    assert np.array_equal(sel, ref_sel)
+    assert out_error(out, ref_out) <= OUT_TOL
+
+
 def test_exact_ties_go_to_lower_page():
     """Logical pages sharing a physical slot score exactly the same."""
     spec = W.shrink("llama3_8b_decode", batch=2, len_lo=64 * 40, len_hi=64 * 40, topk=6)
