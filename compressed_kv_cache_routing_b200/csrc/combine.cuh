@@ -73,76 +73,6 @@ __device__ void combine_unit(const CombineArgs& c, float* smem) {
 
 namespace basiskv {
 
-// One-warp merge of a unit's partials and expansion through B_v (same
-// arithmetic as combine_unit).  zbar: g*r floats of this warp's shared
-// memory.  np <= 64.
-template <int G, int RR, int D>
-__device__ void warp_combine(const float* part_ml, const float* part_acc, int np, const float* b_v,
-                             float* out, float* zbar) {
-  const int lane = threadIdx.x & 31;
-  // each lane owns partials j = lane and lane + 32
-  float w0[G], w1[G], M[G], l[G];
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    const float m0 = lane < np ? __ldcg(part_ml + (lane * G + h) * 2) : -INFINITY;
-    const float m1 = lane + 32 < np ? __ldcg(part_ml + ((lane + 32) * G + h) * 2) : -INFINITY;
-    M[h] = warp_max(fmaxf(m0, m1));
-    w0[h] = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M[h]);
-    w1[h] = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M[h]);
-    float ls = 0.f;
-    if (lane < np) ls += w0[h] * __ldcg(part_ml + (lane * G + h) * 2 + 1);
-    if (lane + 32 < np) ls += w1[h] * __ldcg(part_ml + ((lane + 32) * G + h) * 2 + 1);
-    l[h] = warp_sum(ls);
-  }
-  // zbar[h][i] = sum_j w_jh acc_j[h][i] / l_h, lanes over i; the loads do not
-  // depend on one another, so the unrolled loop keeps several in flight
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-#pragma unroll
-    for (int i0 = 0; i0 < RR; i0 += 32) {  // uniform trip count: shuffles stay converged
-      const int i = i0 + lane;
-      float acc = 0.f;
-#pragma unroll 8
-      for (int j = 0; j < np; ++j) {
-        const float wj = __shfl_sync(0xffffffffu, j < 32 ? w0[h] : w1[h], j & 31);
-        const float v = i < RR ? __ldcg(part_acc + ((size_t)j * G + h) * RR + i) : 0.f;
-        acc = fmaf(wj, v, acc);
-      }
-      if (i < RR) zbar[h * RR + i] = l[h] > 0.f ? acc / l[h] : 0.f;
-    }
-  }
-  __syncwarp();
-  // out[h][c] = zbar[h] . B_v[:, c], lanes over c
-  constexpr int CPL = (D + 31) / 32;
-  float o[G][CPL];
-#pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) o[h][c] = 0.f;
-#pragma unroll 8
-  for (int i = 0; i < RR; ++i) {
-    float bv[CPL];
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) bv[c] = (lane + 32 * c < D) ? __ldg(b_v + (size_t)i * D + lane + 32 * c) : 0.f;
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float z = zbar[h * RR + i];
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) o[h][c] = fmaf(z, bv[c], o[h][c]);
-    }
-  }
-#pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int c = 0; c < CPL; ++c)
-      if (lane + 32 * c < D) out[(size_t)h * D + lane + 32 * c] = o[h][c];
-  __syncwarp();
-}
-
-}  // namespace basiskv
-
-namespace basiskv {
-
 // Count one arrival at `ctr` (warp-collective, after this warp's writes);
 // true in every lane of the warp that completes `expected` arrivals, which
 // also resets the counter.  Everything the other arrivers wrote before

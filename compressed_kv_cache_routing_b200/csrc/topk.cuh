@@ -137,102 +137,6 @@ __device__ void block_topk(const float* scores, int n, int k, int32_t* sel, int3
 
 namespace basiskv {
 
-// One-warp version of block_topk for the warp that completes a unit:
-// same ordering and output.  hist: 256 ints of this warp's shared memory.
-__device__ void warp_topk(const float* scores, int n, int k, int32_t* sel, int32_t* sel_out,
-                          int out_len, int* hist) {
-  const int lane = threadIdx.x & 31;
-  const int kb = k < n ? k : n;
-  uint32_t thr = 0u;
-  int need = 0;
-  if (kb < n) {
-    uint32_t prefix = 0u, mask = 0u;
-    int remaining = kb;
-#pragma unroll 1
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = lane; i < 256; i += 32) hist[i] = 0;
-      __syncwarp();
-      for (int base = 0; base < n; base += 32) {
-        const int i = base + lane;
-        const uint32_t key = i < n ? score_key(__ldcg(scores + i)) : 0u;
-        const bool in = i < n && (key & mask) == prefix;
-        const uint32_t act = __ballot_sync(0xffffffffu, in);
-        if (in) {
-          // one shared atomic per distinct digit: lanes holding equal digits
-          // (the common case in the top byte) would otherwise serialise
-          const uint32_t digit = (key >> shift) & 255u;
-          const uint32_t grp = __match_any_sync(act, digit);
-          if ((int)(__ffs(grp) - 1) == lane) atomicAdd(&hist[digit], __popc(grp));
-        }
-      }
-      __syncwarp();
-      int local = 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) local += hist[8 * lane + q];
-      int incl = local;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_down_sync(0xffffffffu, incl, o);
-        if (lane + o < 32) incl += y;
-      }
-      const int above = incl - local;
-      const bool mine = above < remaining && remaining <= incl;
-      int digit = 0, rem = 0;
-      if (mine) {
-        int acc = above;
-        for (int q = 7; q >= 0; --q) {
-          const int c = hist[8 * lane + q];
-          if (acc + c >= remaining) {
-            digit = 8 * lane + q;
-            rem = remaining - acc;
-            break;
-          }
-          acc += c;
-        }
-      }
-      const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
-      digit = __shfl_sync(0xffffffffu, digit, src);
-      remaining = __shfl_sync(0xffffffffu, rem, src);
-      prefix |= static_cast<uint32_t>(digit) << shift;
-      mask |= 0xFFu << shift;
-      __syncwarp();
-    }
-    thr = prefix;
-    need = remaining;
-  }
-  const uint32_t lt = (1u << lane) - 1u;
-  int eq_before = 0, taken = 0;
-  for (int base = 0; base < n; base += 32) {
-    const int i = base + lane;
-    bool take = false, eq = false;
-    if (i < n) {
-      if (kb < n) {
-        const uint32_t key = score_key(__ldcg(scores + i));
-        eq = key == thr;
-        take = key > thr;
-      } else {
-        take = true;
-      }
-    }
-    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-    if (eq && eq_before + __popc(eqm & lt) < need) take = true;
-    const uint32_t tm = __ballot_sync(0xffffffffu, take);
-    if (take) {
-      const int pos = taken + __popc(tm & lt);
-      sel[pos] = i;
-      if (sel_out) sel_out[pos] = i;
-    }
-    taken += __popc(tm);
-    eq_before += __popc(eqm);
-  }
-  if (sel_out)
-    for (int i = kb + lane; i < out_len; i += 32) sel_out[i] = -1;
-}
-
-}  // namespace basiskv
-
-namespace basiskv {
-
 // ---------------------------------------------------------------------------
 // Selection kernel: one CTA per (sequence, KV head) whose pages are routed.
 // The scores are staged once in shared memory (kTopkKeysMax of them), the

@@ -97,6 +97,10 @@ SMALL = {
     "gqa8": W.shrink("llama3_8b_decode", batch=2, len_lo=3000, len_hi=4000, topk=12, gqa_group=8,
                      num_kv_heads=4),
     "gqa2": W.shrink("llama3_8b_decode", batch=2, len_lo=3000, len_hi=4000, topk=12, gqa_group=2),
+    "gqa1": W.shrink("llama3_8b_decode", batch=2, len_lo=2000, len_hi=3000, topk=10, gqa_group=1),
+    # head_dim 64 on the tensor-core kernels (two channels per lane in the fold)
+    "head_dim64": W.shrink("llama3_8b_decode", batch=3, len_lo=1500, len_hi=3000, topk=12, head_dim=64,
+                           rank_r=16, rank_s=8, page_size=32),
     "fp32_llama_shape": W.shrink("llama3_8b_decode", batch=2, len_lo=1000, len_hi=2000, topk=8,
                                  dtype="f32"),
 }
