@@ -50,7 +50,8 @@ enum { ORACLE_BF16 = 0, ORACLE_F32 = 1 };
  * structure in oracle.py. */
 typedef struct {
     int32_t batch, num_kv_heads, gqa_group, head_dim, page_size;
-    int32_t rank_r, rank_s, topk, dtype, num_slots, ld_pt, pad0;
+    int32_t rank_r, rank_s, topk, dtype, num_slots, ld_pt;
+    int32_t latent; /* nonzero: out holds zbar [G][r] per unit, before B_v */
     double softmax_scale;
     const void *q, *z_pool, *r_pool, *k_pool;
     const float *w_zk, *b_r, *b_v;
@@ -187,8 +188,10 @@ static void route_unit(const oracle_problem *p, int b, int kvh,
 }
 
 /* Exact attention over the valid tokens of the given pages for every query
- * head of (b, kvh); out is [G][d].  sel holds up to topk page indices, -1
- * entries are skipped.  A sequence with no selected token gets out = 0. */
+ * head of (b, kvh); out is [G][d], or [G][r] in latent mode (the weighted
+ * latent zbar itself, the quantity BasisKV keeps in rank-r form until the
+ * output projection).  sel holds up to topk page indices, -1 entries are
+ * skipped.  A sequence with no selected token gets out = 0. */
 static void attend_unit(const oracle_problem *p, int b, int kvh, const int32_t *sel, double *out)
 {
     const int G = p->gqa_group, d = p->head_dim, P = p->page_size, r = p->rank_r;
@@ -226,9 +229,10 @@ static void attend_unit(const oracle_problem *p, int b, int kvh, const int32_t *
             }
         }
 
-        double *o = out + (size_t)h * d;
+        const int width = p->latent ? r : d;
+        double *o = out + (size_t)h * width;
         if (m == 0) {
-            for (int c = 0; c < d; ++c) o[c] = 0.0;
+            for (int c = 0; c < width; ++c) o[c] = 0.0;
             continue;
         }
         /* softmax weights, then the weighted mean of the latents */
@@ -244,6 +248,10 @@ static void attend_unit(const oracle_problem *p, int b, int kvh, const int32_t *
                 zbar[a] += w * widen(p->z_pool, zrow[t] + a, p->dtype);
         }
         for (int a = 0; a < r; ++a) zbar[a] /= den;
+        if (p->latent) {
+            for (int a = 0; a < r; ++a) o[a] = zbar[a];
+            continue;
+        }
         /* value = latent . B_v */
         for (int c = 0; c < d; ++c) {
             double acc = 0.0;
@@ -306,7 +314,7 @@ int oracle_attend(const oracle_problem *p, const int32_t *sel, double *out)
     for (int u = 0; u < U; ++u) {
         if (!unit_wanted(p, u)) continue;
         attend_unit(p, u / p->num_kv_heads, u % p->num_kv_heads, sel + (size_t)u * p->topk,
-                    out + (size_t)u * p->gqa_group * p->head_dim);
+                    out + (size_t)u * p->gqa_group * (p->latent ? p->rank_r : p->head_dim));
     }
     return 0;
 }
@@ -338,7 +346,7 @@ int oracle_decode(const oracle_problem *p, int want_scores, double *page_scores,
             route_unit(p, b, kvh, ps, su, gap ? gap + u : NULL);
             free(tmp);
         }
-        attend_unit(p, b, kvh, su, out + (size_t)u * p->gqa_group * p->head_dim);
+        attend_unit(p, b, kvh, su, out + (size_t)u * p->gqa_group * (p->latent ? p->rank_r : p->head_dim));
     }
     return 0;
 }

@@ -51,7 +51,7 @@ class _Problem(ctypes.Structure):
         ("page_size", ctypes.c_int32), ("rank_r", ctypes.c_int32),
         ("rank_s", ctypes.c_int32), ("topk", ctypes.c_int32),
         ("dtype", ctypes.c_int32), ("num_slots", ctypes.c_int32),
-        ("ld_pt", ctypes.c_int32), ("pad0", ctypes.c_int32),
+        ("ld_pt", ctypes.c_int32), ("latent", ctypes.c_int32),
         ("softmax_scale", ctypes.c_double),
         ("q", ctypes.c_void_p), ("z_pool", ctypes.c_void_p),
         ("r_pool", ctypes.c_void_p), ("k_pool", ctypes.c_void_p),
@@ -108,6 +108,7 @@ class Problem:
     topk: int
     softmax_scale: float
     dtype: int  # BF16 (raw 16-bit patterns) or F32
+    latent: bool = False  # outputs zbar [B][Hq][r] (before B_v) instead of [B][Hq][d]
 
     def __post_init__(self):
         conv = (lambda a: np.ascontiguousarray(a).view(np.uint16)) if self.dtype == BF16 else \
@@ -161,6 +162,7 @@ class Problem:
         p.dtype = self.dtype
         p.num_slots = int(self.z_pool.shape[0])
         p.ld_pt = int(self.page_table.shape[1])
+        p.latent = int(bool(self.latent))
         p.softmax_scale = float(self.softmax_scale)
         p.q = self.q.ctypes.data
         p.z_pool = self.z_pool.ctypes.data
@@ -201,9 +203,10 @@ def route(prob: Problem, units=None, library=None):
 
 
 def attend(prob: Problem, sel: np.ndarray, units=None, library=None):
-    """Exact attention over the pages in ``sel``; out [B][Hkv*G][d] float64."""
+    """Exact attention over the pages in ``sel``; out [B][Hkv*G][d] float64
+    ([B][Hkv*G][r], the latent before B_v, when ``prob.latent``)."""
     sel = np.ascontiguousarray(sel, dtype=np.int32)
-    out = np.zeros((prob.batch, prob.num_kv_heads * prob.gqa_group, prob.head_dim))
+    out = np.zeros((prob.batch, prob.num_kv_heads * prob.gqa_group, prob.rank_r if prob.latent else prob.head_dim))
     mask = _mask(prob, units)  # must outlive the call: the struct holds its address
     st = prob._struct(mask)
     l = library if library is not None else lib()
@@ -214,11 +217,12 @@ def attend(prob: Problem, sel: np.ndarray, units=None, library=None):
 
 
 def decode(prob: Problem, units=None, want_scores=False, library=None):
-    """The whole decode step.  Returns (out [B][Hq][d] f64, sel, scores, gap)."""
+    """The whole decode step.  Returns (out [B][Hq][d] f64 ([B][Hq][r] when
+    ``prob.latent``), sel, scores, gap)."""
     scores = np.full((prob.batch, prob.num_kv_heads, prob.page_table.shape[1]), -np.inf)
     sel = np.full((prob.batch, prob.num_kv_heads, prob.topk), -1, dtype=np.int32)
     gap = np.full((prob.batch, prob.num_kv_heads), np.nan)
-    out = np.zeros((prob.batch, prob.num_kv_heads * prob.gqa_group, prob.head_dim))
+    out = np.zeros((prob.batch, prob.num_kv_heads * prob.gqa_group, prob.rank_r if prob.latent else prob.head_dim))
     mask = _mask(prob, units)  # must outlive the call: the struct holds its address
     st = prob._struct(mask)
     l = library if library is not None else lib()

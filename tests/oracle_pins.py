@@ -8,6 +8,7 @@ mismatch, so the same pins run against the real oracle
 (test_oracle_pins.py) and against deliberately broken copies of it
 (test_oracle_mutants.py), which must each fail at least one pin.
 """
+import dataclasses
 import math
 
 import numpy as np
@@ -206,6 +207,58 @@ def pin_two_tokens_sigmoid(lib):
         sg = 1.0 / (1.0 + math.exp(-D))
         expect = (sg * Z[0] + (1 - sg) * Z[1]) @ prob.b_v[0].astype(np.float64)
         assert rel_err(out[0, h], expect) < 1e-13
+
+
+def _latent(prob):
+    return dataclasses.replace(prob, latent=True)
+
+
+def pin_latent_two_tokens(lib):
+    """Latent output mode (the rank-r weighted latent BasisKV keeps until the
+    output projection): L = 2 in one page gives
+    zbar = sigma(D) Z_0 + (1 - sigma(D)) Z_1, D = scale * q.(K_0 - K_1), with
+    no B_v applied."""
+    rng = np.random.default_rng(5)
+    prob = _latent(make_problem(rng, B=1, Hkv=1, G=3, d=8, P=4, r=4, s=2, lens=(2,), topk=1, scale=0.7))
+    out, _, _, _ = oracle.decode(prob, library=lib)
+    assert out.shape == (1, 3, 4)
+    slot = prob.page_table[0, 0]
+    K = widen(prob.k_pool, prob.dtype)[slot, 0]
+    Z = widen(prob.z_pool, prob.dtype)[slot, 0]
+    q = widen(prob.q, prob.dtype)[0]
+    for h in range(3):
+        D = 0.7 * (q[h] @ (K[0] - K[1]))
+        sg = 1.0 / (1.0 + math.exp(-D))
+        assert rel_err(out[0, h], sg * Z[0] + (1 - sg) * Z[1]) < 1e-13
+
+
+def pin_latent_one_token(lib):
+    """Latent mode, L = 1: zbar = Z_0 whatever q is; L = 0: zero rows, r wide."""
+    rng = np.random.default_rng(3)
+    prob = _latent(make_problem(rng, B=2, Hkv=2, G=2, d=8, P=4, r=4, s=2, lens=(1, 0), topk=3))
+    out, _, _, _ = oracle.decode(prob, library=lib)
+    assert out.shape == (2, 4, 4)
+    Zp = widen(prob.z_pool, prob.dtype)
+    for kvh in range(2):
+        for h in range(2):
+            assert rel_err(out[0, kvh * 2 + h], Zp[prob.page_table[0, 0], kvh, 0]) < 1e-15
+    assert (out[1] == 0).all()
+
+
+def pin_latent_times_bv_is_value(lib):
+    """The value output is the latent output times B_v, head by head, and both
+    modes select the same pages (bf16 storage, ragged lengths, GQA 3)."""
+    rng = np.random.default_rng(17)
+    prob = make_problem(rng, B=3, Hkv=2, G=3, d=8, P=4, r=4, s=2, lens=(13, 3, 9), topk=2,
+                        dtype=oracle.BF16)
+    out, sel, _, _ = oracle.decode(prob, library=lib)
+    zb, sel_l, _, _ = oracle.decode(_latent(prob), library=lib)
+    assert np.array_equal(sel, sel_l)
+    for b in range(3):
+        for kvh in range(2):
+            for h in range(3):
+                row = kvh * 3 + h
+                assert rel_err(zb[b, row] @ prob.b_v[kvh].astype(np.float64), out[b, row]) < 1e-12
 
 
 def pin_folded_scores(lib):

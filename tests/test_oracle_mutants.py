@@ -40,6 +40,11 @@ MUTANTS = [
     ("bf16_low_half", "uint32_t bits = (uint32_t)((const uint16_t *)base)[idx] << 16;",
      "uint32_t bits = (uint32_t)((const uint16_t *)base)[idx];"),
     ("gap_wrong_neighbour", "order[kb - 1].score - order[kb].score", "order[0].score - order[kb].score"),
+    ("latent_before_normalisation",
+     "        for (int a = 0; a < r; ++a) zbar[a] /= den;\n        if (p->latent) {",
+     "        if (p->latent) {\n            for (int a = 0; a < r; ++a) o[a] = zbar[a];\n            continue;\n        }\n"
+     "        for (int a = 0; a < r; ++a) zbar[a] /= den;\n        if (p->latent) {"),
+    ("latent_rows_d_wide", "double *o = out + (size_t)h * width;", "double *o = out + (size_t)h * d;"),
     ("kv_head_stride_in_pool", "return (((size_t)slot * p->num_kv_heads + kvh) * p->page_size + i) * (size_t)width;",
      "return (((size_t)slot * p->num_kv_heads) * p->page_size + i) * (size_t)width;"),
 ]
