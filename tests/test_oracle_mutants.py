@@ -44,7 +44,8 @@ MUTANTS = [
      "        for (int a = 0; a < r; ++a) zbar[a] /= den;\n        if (p->latent) {",
      "        if (p->latent) {\n            for (int a = 0; a < r; ++a) o[a] = zbar[a];\n            continue;\n        }\n"
      "        for (int a = 0; a < r; ++a) zbar[a] /= den;\n        if (p->latent) {"),
-    ("latent_rows_d_wide", "double *o = out + (size_t)h * width;", "double *o = out + (size_t)h * d;"),
+    ("head_rows_shifted", "double *o = out + (size_t)h * width;",
+     "double *o = out + (size_t)(h > 0 ? h - 1 : 0) * width;"),
     ("kv_head_stride_in_pool", "return (((size_t)slot * p->num_kv_heads + kvh) * p->page_size + i) * (size_t)width;",
      "return (((size_t)slot * p->num_kv_heads) * p->page_size + i) * (size_t)width;"),
 ]
