@@ -28,10 +28,11 @@ struct AttnArgs {
   float* part_acc;           // [B*Hkv][np_cap][G][r]
   uint32_t* counters;        // [B*Hkv]
   uint32_t* status;
-  float* out;                // [B][Hkv*G][d]
+  float* out;                // [B][Hkv*G][d]; [B][Hkv*G][r] when latent
   int ld_pt, ld_sel, num_slots, num_kv_heads, head_dim, page_size, rank_r, gqa_group;
   int topk, pages_per_split, stages, np_cap;
   float scale_log2;          // softmax_scale * log2(e)
+  int latent;                // write the weighted latent zbar, before B_v
   // persistent tensor-core kernel only
   int batch;
   const int32_t* attn_off;   // [B+1] prefix of attention items x Hkv (from the prep grid)
@@ -97,7 +98,8 @@ __device__ __forceinline__ void attn_finish(const AttnArgs& a, const AttnUnit& a
   c.part_ml = a.part_ml + (size_t)au.u * a.np_cap * G * 2;
   c.part_acc = a.part_acc + (size_t)au.u * a.np_cap * G * a.rank_r;
   c.b_v = a.b_v + (size_t)au.kvh * a.rank_r * a.head_dim;
-  c.out = a.out + (size_t)au.u * G * a.head_dim;
+  c.out = a.out + (size_t)au.u * G * (a.latent ? a.rank_r : a.head_dim);
+  c.latent = a.latent;
   c.np = gridDim.x * parts_per_cta;
   c.g = G;
   c.r = a.rank_r;
@@ -200,10 +202,11 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
   __shared__ int tok0s[kAttnWarps][8];
   // sequences no warp visits: without pages they get out = 0 and a -1
   // selection; with every page used (no routing) the identity selection
+  const int ow = a.latent ? RR : D;  // output row width
   for (int u = blockIdx.x; u < a.batch * a.num_kv_heads; u += gridDim.x) {
     const int n = (a.seq_lens[u / a.num_kv_heads] + a.page_size - 1) / a.page_size;
     if (n == 0)
-      for (int i = threadIdx.x; i < G * D; i += blockDim.x) a.out[(size_t)u * G * D + i] = 0.f;
+      for (int i = threadIdx.x; i < G * ow; i += blockDim.x) a.out[(size_t)u * G * ow + i] = 0.f;
     if (a.sel_out && a.topk >= n)
       for (int i = threadIdx.x; i < a.topk; i += blockDim.x) a.sel_out[(size_t)u * a.topk + i] = i < n ? i : -1;
   }
@@ -350,7 +353,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
       MergeOut<G, RR> mo;
       merge_all<G, RR>(a.part_ml + (size_t)u * a.np_cap * G * 2, a.part_acc + (size_t)u * a.np_cap * G * RR,
                        min(np, a.np_cap), mo);
-      finish_unit<G, RR, D>(mo, a.b_v + (size_t)at.kvh * RR * D, a.out + (size_t)u * G * D, zbar);
+      if (a.latent) finish_unit_latent<G, RR>(mo, a.out + (size_t)u * G * RR);
+      else finish_unit<G, RR, D>(mo, a.b_v + (size_t)at.kvh * RR * D, a.out + (size_t)u * G * D, zbar);
       if (lane == 0) a.counters[u] = 0u;
     }
   };

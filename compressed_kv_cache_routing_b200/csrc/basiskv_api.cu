@@ -308,7 +308,7 @@ LaunchPlan plan(const basiskv_handle* h, int batch, int topk, bool force_route) 
 }
 
 int launch_prep(basiskv_handle* h, const LaunchPlan& lp, int topk, int force, float* out, int32_t* sel_out,
-                float* fill_scores, cudaStream_t stream) {
+                float* fill_scores, int latent, cudaStream_t stream) {
   const basiskv_params& p = h->p;
   PrepArgs a;
   a.seq_lens = h->d_seq_lens;
@@ -327,6 +327,7 @@ int launch_prep(basiskv_handle* h, const LaunchPlan& lp, int topk, int force, fl
   a.attn_sub = lp.sub;
   a.ld_pt = p.max_pages_per_seq;
   a.fill_scores = fill_scores != nullptr;
+  a.out_width = latent ? p.rank_r : p.head_dim;
   prep_kernel<<<dim3(p.num_kv_heads, lp.batch), kPrepThreads, 0, stream>>>(a);
   CUDA_TRY(cudaGetLastError());
   return BASISKV_OK;
@@ -429,7 +430,7 @@ int launch_topk(basiskv_handle* h, const LaunchPlan& lp, int topk, const float* 
   return BASISKV_OK;
 }
 
-int launch_attn(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk, float scale,
+int launch_attn(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk, float scale, int latent,
                 float* out, int32_t* sel_out, bool pdl, cudaStream_t stream) {
   const basiskv_params& p = h->p;
   const size_t U = (size_t)p.max_batch * p.num_kv_heads;
@@ -460,6 +461,7 @@ int launch_attn(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk
   a.stages = h->attn_stages;
   a.np_cap = kPartsCap;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.latent = latent;
   a.batch = lp.batch;
   a.attn_off = h->d_attn_off;
   a.plan_n = lp.attn_off.empty() ? -1 : lp.batch;
@@ -687,8 +689,11 @@ int basiskv_load_page_table(basiskv_handle* h, int batch, const int32_t* page_ta
   return BASISKV_OK;
 }
 
-int basiskv_decode_attn(basiskv_handle* h, int batch, const void* q, int topk, float softmax_scale,
-                        float* out, int32_t* sel_out, basiskv_stream_t stream) {
+// The decode step behind basiskv_decode_attn (latent = 0: out = zbar.B_v,
+// [batch][Hq][d]) and basiskv_decode_attn_latent (latent = 1: out = zbar,
+// [batch][Hq][r]).
+static int decode_step(basiskv_handle* h, int batch, const void* q, int topk, float softmax_scale, float* out,
+                       int32_t* sel_out, basiskv_stream_t stream, int latent) {
   int rc = check_call(h, batch, q, topk);
   if (rc) return rc;
   if (!out) return fail(BASISKV_ERR_INVALID_ARG, "out is NULL");
@@ -704,7 +709,7 @@ int basiskv_decode_attn(basiskv_handle* h, int batch, const void* q, int topk, f
   // batch too large for that needs the prep grid to write it
   const bool use_prep = (route_tc || h->attn_fn) && lp.route_off.empty();
   if (use_prep) {
-    rc = launch_prep(h, lp, topk, 0, out, sel_out, nullptr, st);
+    rc = launch_prep(h, lp, topk, 0, out, sel_out, nullptr, latent, st);
     if (rc) return rc;
   }
   if (prof) CUDA_TRY(cudaEventRecord(ev[1], st));
@@ -722,7 +727,7 @@ int basiskv_decode_attn(basiskv_handle* h, int batch, const void* q, int topk, f
   if (prof) CUDA_TRY(cudaEventRecord(ev[3], st));
   // PDL only behind a routing grid (which signals after any prep grid has
   // finished, so the plan is complete when this grid starts)
-  rc = launch_attn(h, lp, q, topk, softmax_scale, out, sel_out, lp.any_routed && !prof, st);
+  rc = launch_attn(h, lp, q, topk, softmax_scale, latent, out, sel_out, lp.any_routed && !prof, st);
   if (rc) return rc;
   if (prof) {
     CUDA_TRY(cudaEventRecord(ev[4], st));
@@ -735,6 +740,16 @@ int basiskv_decode_attn(basiskv_handle* h, int batch, const void* q, int topk, f
   h->last_launch[4] = h->route_fn != nullptr;
   h->last_launch[5] = h->attn_fn != nullptr;
   return BASISKV_OK;
+}
+
+int basiskv_decode_attn(basiskv_handle* h, int batch, const void* q, int topk, float softmax_scale,
+                        float* out, int32_t* sel_out, basiskv_stream_t stream) {
+  return decode_step(h, batch, q, topk, softmax_scale, out, sel_out, stream, 0);
+}
+
+int basiskv_decode_attn_latent(basiskv_handle* h, int batch, const void* q, int topk, float softmax_scale,
+                               float* zbar_out, int32_t* sel_out, basiskv_stream_t stream) {
+  return decode_step(h, batch, q, topk, softmax_scale, zbar_out, sel_out, stream, 1);
 }
 
 int basiskv_decode_attn_host(basiskv_handle* h, int batch, const void* q_host, int topk, float softmax_scale,
@@ -767,7 +782,7 @@ int basiskv_route(basiskv_handle* h, int batch, const void* q, int topk, float* 
   float* scores = scores_out ? scores_out : h->d_scores;
   // the prep grid writes -inf past n_b, the -1 rows of empty sequences and,
   // for large batches, the plan
-  rc = launch_prep(h, lp, topk, 1, nullptr, sel_out, scores, st);
+  rc = launch_prep(h, lp, topk, 1, nullptr, sel_out, scores, 0, st);
   if (rc) return rc;
   if (!lp.any_routed) return BASISKV_OK;
   RouteArgs ra = route_args(h, lp, q, topk, scores, sel_out, 1);

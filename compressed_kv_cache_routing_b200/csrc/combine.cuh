@@ -19,8 +19,9 @@ struct CombineArgs {
   const float* part_ml;   // [NP][G][2] of this unit
   const float* part_acc;  // [NP][G][r] of this unit
   const float* b_v;       // [r][d] of this KV head
-  float* out;             // [G][d] of this unit (row stride d)
+  float* out;             // [G][d] of this unit (row stride d); [G][r] when latent
   int np, g, r, d;
+  int latent;             // write zbar itself, before B_v
 };
 
 // smem: np*g + 2*g + g*r floats.  All NT threads must call it.
@@ -60,6 +61,10 @@ __device__ void combine_unit(const CombineArgs& c, float* smem) {
     zbar[i] = l > 0.f ? acc / l : 0.f;
   }
   __syncthreads();
+  if (c.latent) {
+    for (int i = tid; i < c.g * c.r; i += NT) c.out[i] = zbar[i];
+    return;
+  }
   for (int i = tid; i < c.g * c.d; i += NT) {
     const int h = i / c.d, col = i % c.d;
     const float* z = zbar + h * c.r;
@@ -196,6 +201,24 @@ __device__ void merge_all(const float* ml, const float* acc, int np, MergeOut<G,
     MergeOut<G, RR> t;
     merge_partials<G, RR>(ml + (size_t)j0 * G * 2, acc + (size_t)j0 * G * RR, min(np - j0, 8), t);
     merge_into(o, t);
+  }
+}
+
+// Latent output: zbar = acc / L per head, written as [G][r] (no B_v).
+template <int G, int RR>
+__device__ void finish_unit_latent(const MergeOut<G, RR>& mo, float* out) {
+  constexpr int V = MergeOut<G, RR>::V, VPL = MergeOut<G, RR>::VPL;
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 0; k < VPL; ++k) {
+    const int v = lane + 32 * k;
+    const int h = (4 * v) / RR;
+    const float Lh = __shfl_sync(0xffffffffu, mo.L, h < G ? h : 0);
+    if (v < V) {
+      const float inv = Lh > 0.f ? 1.f / Lh : 0.f;
+      reinterpret_cast<float4*>(out)[v] =
+          make_float4(mo.acc[k].x * inv, mo.acc[k].y * inv, mo.acc[k].z * inv, mo.acc[k].w * inv);
+    }
   }
 }
 

@@ -22,6 +22,7 @@ struct PrepArgs {
   float* scores;           // [B][Hkv][ld_pt]: -inf past n_b when fill_scores
   int batch, num_kv_heads, gqa_group, head_dim, page_size;
   int topk, force, attn_sub, ld_pt, fill_scores;
+  int out_width;           // d, or r for the latent output
 };
 
 constexpr int kPrepThreads = 128;
@@ -30,7 +31,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const PrepArgs a) {
   pdl_launch_dependents();
   __shared__ int scan_tmp[kPrepThreads / 32];
   const int tid = threadIdx.x;
-  const int G = a.gqa_group, d = a.head_dim, P = a.page_size;
+  const int G = a.gqa_group, P = a.page_size;
   const int Hkv = a.num_kv_heads;
 
   if (blockIdx.x == 0 && blockIdx.y == 0) {
@@ -67,7 +68,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const PrepArgs a) {
     for (int j = n + tid; j < a.ld_pt; j += kPrepThreads) a.scores[(size_t)u * a.ld_pt + j] = -INFINITY;
   if (n == 0) {
     if (a.out)
-      for (int i = tid; i < G * d; i += kPrepThreads) a.out[(size_t)u * G * d + i] = 0.f;
+      for (int i = tid; i < G * a.out_width; i += kPrepThreads) a.out[(size_t)u * G * a.out_width + i] = 0.f;
     if (a.sel_out)
       for (int i = tid; i < a.topk; i += kPrepThreads) a.sel_out[(size_t)u * a.topk + i] = -1;
     return;

@@ -160,6 +160,19 @@ BASISKV_API int basiskv_decode_attn(basiskv_handle *h, int batch, const void *q,
                         float softmax_scale, float *out, int32_t *sel_out,
                         basiskv_stream_t stream);
 
+/* The same step, returning the weighted latent instead of the value
+ * ("BasisKV: Value Latents for Communication and Key Routing", English
+ * abstract: values stay rank-r latents, and their compression is tied to
+ * the output projection, so a caller may fold B_v into its own W_o and keep
+ * the rank-r form until then):
+ *   zbar_out [batch][Hkv*G][r] fp32 (device): zbar_h = sum_t p_t Z_t, the
+ *            softmax-weighted latent of each query head (out = zbar . B_v)
+ * Arguments, selection, errors and stream behaviour as basiskv_decode_attn;
+ * a sequence of length 0 gets zbar = 0. */
+BASISKV_API int basiskv_decode_attn_latent(basiskv_handle *h, int batch, const void *q, int topk,
+                               float softmax_scale, float *zbar_out, int32_t *sel_out,
+                               basiskv_stream_t stream);
+
 /* The same step with HOST buffers: copies q_host (pinned or pageable) to a
  * library-owned device buffer, runs basiskv_decode_attn, copies out (and
  * sel when sel_host is not NULL) back, and waits for the stream. */

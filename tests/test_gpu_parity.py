@@ -5,6 +5,7 @@ relative error of 2e-3 (max over (b, h) of |y - y*|_inf / |y*|_inf), the
 bound for bf16 storage with fp32 accumulation.  Page scores from the routing
 kernel are compared too (relative 1e-3).
 """
+import dataclasses
 import math
 
 import numpy as np
@@ -45,6 +46,21 @@ def gpu_decode(w, topk=None, scale=None, kv=None, max_topk=None):
     res = out.cpu().numpy(), sel.cpu().numpy()
     if own:
         kv.close()
+    return res
+
+
+def gpu_decode_latent(w):
+    """basiskv_decode_attn_latent: zbar [B][Hq][r] and the selection."""
+    s = w.spec
+    kv = bk.BasisKV.for_workload(w)
+    B = len(w.seq_lens)
+    zbar = torch.full((B, s.num_q_heads, s.rank_r), float("nan"), device="cuda")
+    sel = torch.full((B, s.num_kv_heads, s.topk), -7, device="cuda", dtype=torch.int32)
+    bk.basiskv_decode_attn_latent(kv.handle, w.q[:B], s.topk, s.softmax_scale, zbar, sel)
+    torch.cuda.synchronize()
+    assert bk.basiskv_get_status(kv.handle, clear=True) == 0
+    res = zbar.cpu().numpy(), sel.cpu().numpy()
+    kv.close()
     return res
 
 
@@ -212,6 +228,38 @@ def test_batch_past_the_parameter_plan():
     out, sel = gpu_decode(w)
     assert np.array_equal(sel, ref_sel)
     assert out_error(out, ref_out) <= OUT_TOL
+
+
+@pytest.mark.parametrize("name", ["llama3_8b_decode", "high_concurrency", "dense_limit", "head_dim64", "tiny",
+                                  "generic_bf16"])
+def test_latent_output(name):
+    """The weighted latent before B_v, on the tensor-core and CUDA-core
+    kernels, against the oracle's latent mode."""
+    w = W.generate(SMALL[name], device="cuda")
+    prob = dataclasses.replace(to_problem(w), latent=True)
+    ref_z, ref_sel, _, _ = oracle.decode(prob)
+    zbar, sel = gpu_decode_latent(w)
+    assert np.array_equal(sel, ref_sel), name
+    assert out_error(zbar, ref_z) <= OUT_TOL
+
+
+def test_latent_output_edge_lengths_and_large_batch():
+    """Zero-length sequences get zbar = 0 (r wide) on both the parameter-plan
+    path and the prep-grid path (more than 512 sequences)."""
+    for spec, lens in [(W.shrink("llama3_8b_decode", batch=5, len_lo=4000, len_hi=4000, topk=8),
+                        [0, 1, 65, 4000, 8 * 64]),
+                       (W.shrink("llama3_8b_decode", batch=600, len_lo=1, len_hi=400, topk=3), None)]:
+        w = _with_lengths(spec, lens) if lens is not None else W.generate(spec, device="cuda")
+        if lens is None:
+            w.seq_lens[::7] = 0
+            w.page_table[::7] = 0
+        prob = dataclasses.replace(to_problem(w), latent=True)
+        ref_z, ref_sel, _, _ = oracle.decode(prob)
+        zbar, sel = gpu_decode_latent(w)
+        assert np.array_equal(sel, ref_sel)
+        assert out_error(zbar, ref_z) <= OUT_TOL
+        empty = np.asarray(w.seq_lens) == 0
+        assert (zbar[empty] == 0).all() and (sel[empty] == -1).all()
 
 
 def test_exact_ties_go_to_lower_page():
