@@ -233,6 +233,40 @@ def decode(prob: Problem, units=None, want_scores=False, library=None):
     return out, sel, scores, gap
 
 
+def _round_to_storage(x: np.ndarray, dtype: int) -> np.ndarray:
+    """float64 -> the stored value as float64: fp32, or bf16 by rounding the
+    fp32 value to nearest, ties to even (on its bit pattern)."""
+    f = np.asarray(x, dtype=np.float32)
+    if dtype == F32:
+        return f.astype(np.float64)
+    bits = f.view(np.uint32).astype(np.uint64)
+    bits = (bits + 0x7FFF + ((bits >> 16) & 1)) >> 16 << 16
+    return bits.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def encode(k: np.ndarray, v: np.ndarray, w_zk: np.ndarray, b_r: np.ndarray, b_v: np.ndarray, dtype: int):
+    """The stored rows for incoming keys and values ("BasisKV: Value Latents
+    for Communication and Key Routing", English abstract: values are kept as
+    rank-r latents, and a Key-specific residual holds what the Value latent
+    cannot predict).  Least-squares reading, per KV head:
+        Z = V . pinv(B_v)                          (the latent nearest to V)
+        R = (K - Z_stored . W_zk) . pinv(B_r)      (the residual of the stored latent)
+    k, v: [Hkv][n][d]; returns (Z [Hkv][n][r], R [Hkv][n][s]) as the stored
+    values (rounded to ``dtype``), in float64."""
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    hkv, n, _ = k.shape
+    r, s = b_v.shape[1], b_r.shape[1] if b_r.size else 0
+    Z = np.zeros((hkv, n, r))
+    R = np.zeros((hkv, n, s))
+    for h in range(hkv):
+        Z[h] = _round_to_storage(v[h] @ np.linalg.pinv(b_v[h].astype(np.float64)), dtype)
+        if s:
+            res = k[h] - Z[h] @ w_zk[h].astype(np.float64)
+            R[h] = _round_to_storage(res @ np.linalg.pinv(b_r[h].astype(np.float64)), dtype)
+    return Z, R
+
+
 def set_threads(n: int) -> None:
     lib().oracle_set_threads(int(n))
 

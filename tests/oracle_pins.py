@@ -261,6 +261,51 @@ def pin_latent_times_bv_is_value(lib):
                 assert rel_err(zb[b, row] @ prob.b_v[kvh].astype(np.float64), out[b, row]) < 1e-12
 
 
+def _bases(rng, hkv=2, d=16, r=6, s=4):
+    W = rng.standard_normal((hkv, r, d)).astype(np.float32)
+    Br = rng.standard_normal((hkv, s, d)).astype(np.float32)
+    Bv = rng.standard_normal((hkv, r, d)).astype(np.float32)
+    return W, Br, Bv
+
+
+def pin_encode_recovers_latents(lib):
+    """Encode: values in the row space of B_v and keys in the span of the
+    prediction plus the residual basis come back as their exact latents
+    (up to fp32 storage)."""
+    rng = np.random.default_rng(23)
+    W, Br, Bv = _bases(rng)
+    Z0 = rng.standard_normal((2, 5, 6)).astype(np.float32).astype(np.float64)
+    R0 = rng.standard_normal((2, 5, 4)).astype(np.float32).astype(np.float64)
+    V = np.einsum("hna,had->hnd", Z0, Bv.astype(np.float64))
+    K = np.einsum("hna,had->hnd", Z0, W.astype(np.float64)) + np.einsum("hnb,hbd->hnd", R0, Br.astype(np.float64))
+    Z, R = oracle.encode(K, V, W, Br, Bv, oracle.F32)
+    assert rel_err(Z, Z0) < 1e-6 and rel_err(R, R0) < 1e-5
+
+
+def pin_encode_least_squares(lib):
+    """Encode of arbitrary keys and values: what is left is orthogonal to
+    the basis rows (the normal equations of the least-squares fit), for both
+    the latent and the residual; bf16 storage leaves the latent on its grid."""
+    rng = np.random.default_rng(29)
+    W, Br, Bv = _bases(rng)
+    V = rng.standard_normal((2, 7, 16))
+    K = rng.standard_normal((2, 7, 16))
+    Z, R = oracle.encode(K, V, W, Br, Bv, oracle.F32)
+    for h in range(2):
+        bv, w, br = (m[h].astype(np.float64) for m in (Bv, W, Br))
+        lv = (V[h] - Z[h] @ bv) @ bv.T
+        assert np.abs(lv).max() < 1e-4 * np.abs(V[h]).max() * np.abs(bv).max()
+        lk = (K[h] - Z[h] @ w - R[h] @ br) @ br.T
+        assert np.abs(lk).max() < 1e-4 * np.abs(K[h]).max() * np.abs(br).max()
+    Zb, _ = oracle.encode(K, V, W, Br, Bv, oracle.BF16)
+    assert np.array_equal(widen(bf16_bits(Zb), oracle.BF16), Zb)
+    assert rel_err(Zb, Z) < 2 ** -8
+    # the bf16 rounding itself against torch's conversion (nearest, ties even)
+    x = np.concatenate([rng.standard_normal(4096) * 10.0 ** rng.integers(-3, 4, 4096),
+                        [1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -(1.0 + 2 ** -8), 0.0]])
+    assert np.array_equal(oracle._round_to_storage(x, oracle.BF16), widen(bf16_bits(x), oracle.BF16))
+
+
 def pin_folded_scores(lib):
     """Page scores against the folded form  u = Z.(W_zk q) + R.(B_r q)
     (associativity), evaluated with numpy matmuls on the gathered sequence,
