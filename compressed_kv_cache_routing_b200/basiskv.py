@@ -36,7 +36,7 @@ EXPORTED = (
     "basiskv_reset_seq", "basiskv_load_page_table", "basiskv_decode_attn",
     "basiskv_decode_attn_host", "basiskv_route", "basiskv_get_status", "basiskv_profile_begin",
     "basiskv_profile_end", "basiskv_last_launch", "basiskv_last_error", "basiskv_version",
-    "basiskv_decode_attn_noalloc", "basiskv_decode_attn_latent",
+    "basiskv_decode_attn_noalloc", "basiskv_decode_attn_latent", "basiskv_encode_rows",
 )
 
 
@@ -83,6 +83,7 @@ def load(path: str = LIB_PATH):
         "basiskv_decode_attn": [H, i32, vp, i32, f32, vp, vp, vp],
         "basiskv_decode_attn_host": [H, i32, vp, i32, f32, vp, vp, vp],
         "basiskv_decode_attn_latent": [H, i32, vp, i32, f32, vp, vp, vp],
+        "basiskv_encode_rows": [H, i32, i32, i32, vp, vp, vp],
         "basiskv_route": [H, i32, vp, i32, vp, vp, vp],
         "basiskv_get_status": [H, ctypes.POINTER(ctypes.c_uint32), i32],
         "basiskv_profile_begin": [H, i32],
@@ -162,6 +163,12 @@ def basiskv_decode_attn_latent(h, q, topk, softmax_scale, zbar_out, sel_out=None
     b = int(q.shape[0]) if batch is None else batch
     _check(load().basiskv_decode_attn_latent(h, b, _ptr(q), topk, float(softmax_scale), _ptr(zbar_out),
                                              _ptr(sel_out), _stream(stream)))
+
+
+def basiskv_encode_rows(h, slot, row0, k, v, stream=None):
+    """Encode k, v [Hkv][n][d] (pool dtype, device) into rows [row0, row0+n)
+    of pool slot ``slot``: K as given, Z and R by least squares."""
+    _check(load().basiskv_encode_rows(h, slot, row0, int(k.shape[1]), _ptr(k), _ptr(v), _stream(stream)))
 
 
 def basiskv_decode_attn_host(h, q_host, topk, softmax_scale, out_host, sel_host=None, stream=None):

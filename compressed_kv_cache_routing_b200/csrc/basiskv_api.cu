@@ -15,6 +15,7 @@
 
 #include "../../include/basiskv.h"
 #include "attn.cuh"
+#include "encode.cuh"
 #include "plan.cuh"
 #include "route.cuh"
 
@@ -91,6 +92,53 @@ const std::map<AttnKey, AttnFn>& attn_table() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// A = B^T (B B^T)^-1, the pseudo-inverse of a full-row-rank B [m][d], as
+// A [d][m]; double precision, Gauss-Jordan with partial pivoting on the
+// Gram matrix.  False when the rows of B are numerically dependent.
+bool right_pinv(const float* B, int m, int d, float* A) {
+  std::vector<double> G((size_t)m * m), Gi((size_t)m * m, 0.0);
+  double gmax = 0.0;
+  for (int i = 0; i < m; ++i)
+    for (int j = 0; j < m; ++j) {
+      double acc = 0.0;
+      for (int c = 0; c < d; ++c) acc += (double)B[(size_t)i * d + c] * B[(size_t)j * d + c];
+      G[(size_t)i * m + j] = acc;
+      gmax = std::max(gmax, std::fabs(acc));
+    }
+  for (int i = 0; i < m; ++i) Gi[(size_t)i * m + i] = 1.0;
+  for (int col = 0; col < m; ++col) {
+    int piv = col;
+    for (int row = col + 1; row < m; ++row)
+      if (std::fabs(G[(size_t)row * m + col]) > std::fabs(G[(size_t)piv * m + col])) piv = row;
+    const double pv = G[(size_t)piv * m + col];
+    if (!(std::fabs(pv) > 1e-10 * gmax)) return false;
+    for (int c = 0; c < m; ++c) {
+      std::swap(G[(size_t)col * m + c], G[(size_t)piv * m + c]);
+      std::swap(Gi[(size_t)col * m + c], Gi[(size_t)piv * m + c]);
+    }
+    for (int c = 0; c < m; ++c) {
+      G[(size_t)col * m + c] /= pv;
+      Gi[(size_t)col * m + c] /= pv;
+    }
+    for (int row = 0; row < m; ++row) {
+      if (row == col) continue;
+      const double f = G[(size_t)row * m + col];
+      if (f == 0.0) continue;
+      for (int c = 0; c < m; ++c) {
+        G[(size_t)row * m + c] -= f * G[(size_t)col * m + c];
+        Gi[(size_t)row * m + c] -= f * Gi[(size_t)col * m + c];
+      }
+    }
+  }
+  for (int c = 0; c < d; ++c)
+    for (int j = 0; j < m; ++j) {
+      double acc = 0.0;
+      for (int i = 0; i < m; ++i) acc += (double)B[(size_t)i * d + c] * Gi[(size_t)i * m + j];
+      A[(size_t)c * m + j] = (float)acc;
+    }
+  return true;
+}
+
 }  // namespace
 
 struct basiskv_handle {
@@ -109,6 +157,8 @@ struct basiskv_handle {
   float* d_qf = nullptr;            // [max_batch*Hkv][G][r+s] folded routing queries
   uint32_t* d_fold_flag = nullptr;  // [max_batch*Hkv][32] tag of the call that wrote each fold slice
   uint32_t route_tag = 0;           // tag of the last routing launch
+  float* d_enc = nullptr;           // pinv(B_v) [Hkv][d][r], then pinv(B_r) [Hkv][d][s] (basiskv_encode_rows)
+  bool enc_ready = false;
   uint32_t* d_status = nullptr;
   int32_t* d_route_off = nullptr;   // [max_batch+1]
   int32_t* d_attn_off = nullptr;    // [max_batch+1]
@@ -542,6 +592,7 @@ int basiskv_create(const basiskv_params* p, basiskv_handle** out) {
       {(void**)&h->d_part_acc, sizeof(float) * U * kPartsCap * G * p->rank_r},
       {(void**)&h->d_counters, sizeof(uint32_t) * 3 * U},
       {(void**)&h->d_qf, sizeof(float) * U * G * (p->rank_r + p->rank_s)},
+      {(void**)&h->d_enc, sizeof(float) * Hkv * p->head_dim * (p->rank_r + p->rank_s)},
       {(void**)&h->d_fold_flag, sizeof(uint32_t) * U * 32},
       {(void**)&h->d_status, sizeof(uint32_t)},
       {(void**)&h->d_route_off, sizeof(int32_t) * (B + 1)},
@@ -598,7 +649,7 @@ int basiskv_destroy(basiskv_handle* h) {
   cudaDeviceSynchronize();
   void* ptrs[] = {h->d_page_table, h->d_seq_lens, h->d_scores, h->d_sel, h->d_part_ml, h->d_part_acc,
                   h->d_counters, h->d_status, h->d_q_stage, h->d_out_stage, h->d_sel_stage,
-                  h->d_route_off, h->d_attn_off, h->d_qf, h->d_fold_flag};
+                  h->d_route_off, h->d_attn_off, h->d_qf, h->d_fold_flag, h->d_enc};
   for (void* q : ptrs)
     if (q) cudaFree(q);
   for (cudaEvent_t e : h->events) cudaEventDestroy(e);
@@ -750,6 +801,57 @@ int basiskv_decode_attn(basiskv_handle* h, int batch, const void* q, int topk, f
 int basiskv_decode_attn_latent(basiskv_handle* h, int batch, const void* q, int topk, float softmax_scale,
                                float* zbar_out, int32_t* sel_out, basiskv_stream_t stream) {
   return decode_step(h, batch, q, topk, softmax_scale, zbar_out, sel_out, stream, 1);
+}
+
+int basiskv_encode_rows(basiskv_handle* h, int slot, int row0, int n_rows, const void* k, const void* v,
+                        basiskv_stream_t stream) {
+  int rc = check_handle(h);
+  if (rc) return rc;
+  const basiskv_params& p = h->p;
+  if (slot < 0 || slot >= p.num_slots) return fail(BASISKV_ERR_INVALID_ARG, "slot %d outside [0, %d)", slot, p.num_slots);
+  if (n_rows < 1 || row0 < 0 || row0 + n_rows > p.page_size)
+    return fail(BASISKV_ERR_INVALID_ARG, "rows [%d, %d) outside a page of %d", row0, row0 + n_rows, p.page_size);
+  if (!k || !v) return fail(BASISKV_ERR_INVALID_ARG, "k or v is NULL");
+  const int Hkv = p.num_kv_heads, d = p.head_dim, r = p.rank_r, s = p.rank_s;
+  if (!h->enc_ready) {
+    // the pseudo-inverses of the bases, once, on the host (a set-up step)
+    std::vector<float> bv((size_t)Hkv * r * d), br((size_t)Hkv * s * d), enc((size_t)Hkv * d * (r + s));
+    CUDA_TRY(cudaMemcpy(bv.data(), p.b_v, sizeof(float) * bv.size(), cudaMemcpyDeviceToHost));
+    if (s > 0) CUDA_TRY(cudaMemcpy(br.data(), p.b_r, sizeof(float) * br.size(), cudaMemcpyDeviceToHost));
+    for (int kvh = 0; kvh < Hkv; ++kvh) {
+      if (!right_pinv(bv.data() + (size_t)kvh * r * d, r, d, enc.data() + (size_t)kvh * d * r))
+        return fail(BASISKV_ERR_INVALID_ARG, "the rows of B_v of KV head %d are linearly dependent", kvh);
+      if (s > 0 && !right_pinv(br.data() + (size_t)kvh * s * d, s, d,
+                               enc.data() + (size_t)Hkv * d * r + (size_t)kvh * d * s))
+        return fail(BASISKV_ERR_INVALID_ARG, "the rows of B_r of KV head %d are linearly dependent", kvh);
+    }
+    CUDA_TRY(cudaMemcpy(h->d_enc, enc.data(), sizeof(float) * enc.size(), cudaMemcpyHostToDevice));
+    h->enc_ready = true;
+  }
+  EncodeArgs a;
+  a.k = k;
+  a.v = v;
+  a.k_pool = const_cast<void*>(p.k_pool);
+  a.z_pool = const_cast<void*>(p.z_pool);
+  a.r_pool = const_cast<void*>(p.r_pool);
+  a.a_v = h->d_enc;
+  a.a_r = h->d_enc + (size_t)Hkv * d * r;
+  a.w_zk = p.w_zk;
+  a.num_kv_heads = Hkv;
+  a.page_size = p.page_size;
+  a.head_dim = d;
+  a.rank_r = r;
+  a.rank_s = s;
+  a.slot = slot;
+  a.row0 = row0;
+  a.n = n_rows;
+  const dim3 grid(n_rows, Hkv);
+  const size_t smem = sizeof(float) * (3 * (size_t)d + r);
+  cudaStream_t st = (cudaStream_t)stream;
+  if (p.dtype == BASISKV_DTYPE_BF16) encode_rows_kernel<__nv_bfloat16><<<grid, kEncodeThreads, smem, st>>>(a);
+  else encode_rows_kernel<float><<<grid, kEncodeThreads, smem, st>>>(a);
+  CUDA_TRY(cudaGetLastError());
+  return BASISKV_OK;
 }
 
 int basiskv_decode_attn_host(basiskv_handle* h, int batch, const void* q_host, int topk, float softmax_scale,

@@ -97,7 +97,7 @@ typedef struct basiskv_params {
     int32_t num_slots;          /* pages the pools hold                      */
     int32_t dtype;              /* BASISKV_DTYPE_*                           */
     int32_t reserved;           /* must be 0                                 */
-    const void *z_pool;         /* caller-owned, read-only during calls      */
+    const void *z_pool;         /* caller-owned; written only by encode_rows */
     const void *r_pool;
     const void *k_pool;
     const float *w_zk;
@@ -179,6 +179,23 @@ BASISKV_API int basiskv_decode_attn_latent(basiskv_handle *h, int batch, const v
 BASISKV_API int basiskv_decode_attn_host(basiskv_handle *h, int batch, const void *q_host, int topk,
                              float softmax_scale, float *out_host, int32_t *sel_host,
                              basiskv_stream_t stream);
+
+/* Encode rows [row0, row0 + n_rows) of pool slot `slot`, every KV head,
+ * from incoming keys and values k, v [Hkv][n_rows][d] (pool dtype, device)
+ * ("BasisKV: Value Latents for Communication and Key Routing", English
+ * abstract: values kept as rank-r latents, and a Key-specific residual
+ * storing what the Value latent cannot predict; least-squares reading):
+ *   K rows stored as given;
+ *   Z = V . pinv(B_v), rounded to the pool dtype;
+ *   R = (K - Z . W_zk) . pinv(B_r), from the rounded Z, rounded.
+ * The only call that writes the caller's pools.  The first call computes
+ * the pseudo-inverses of the bases on the host (synchronous); later calls
+ * only enqueue on `stream`.  The page table is not touched: follow with
+ * basiskv_append_page or basiskv_append_tokens.  Errors: INVALID_ARG (slot
+ * or rows out of range, NULL k or v, bases with linearly dependent rows),
+ * CUDA. */
+BASISKV_API int basiskv_encode_rows(basiskv_handle *h, int slot, int row0, int n_rows, const void *k,
+                        const void *v, basiskv_stream_t stream);
 
 /* Routing alone (steps route-prep, route-score, top-k) for every sequence
  * with at least one page, whether or not topk >= n_b.  scores_out

@@ -253,18 +253,23 @@ def encode(k: np.ndarray, v: np.ndarray, w_zk: np.ndarray, b_r: np.ndarray, b_v:
         R = (K - Z_stored . W_zk) . pinv(B_r)      (the residual of the stored latent)
     k, v: [Hkv][n][d]; returns (Z [Hkv][n][r], R [Hkv][n][s]) as the stored
     values (rounded to ``dtype``), in float64."""
-    k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
-    hkv, n, _ = k.shape
-    r, s = b_v.shape[1], b_r.shape[1] if b_r.size else 0
-    Z = np.zeros((hkv, n, r))
-    R = np.zeros((hkv, n, s))
-    for h in range(hkv):
-        Z[h] = _round_to_storage(v[h] @ np.linalg.pinv(b_v[h].astype(np.float64)), dtype)
+    Z = np.stack([_round_to_storage(v[h] @ np.linalg.pinv(b_v[h].astype(np.float64)), dtype)
+                  for h in range(v.shape[0])])
+    return Z, encode_residual(k, Z, w_zk, b_r, dtype)
+
+
+def encode_residual(k: np.ndarray, z: np.ndarray, w_zk: np.ndarray, b_r: np.ndarray, dtype: int):
+    """The residual rows R = (K - Z . W_zk) . pinv(B_r), rounded to ``dtype``,
+    for the stored latents ``z`` [Hkv][n][r]; [Hkv][n][s] float64."""
+    k = np.asarray(k, dtype=np.float64)
+    s = b_r.shape[1] if b_r.size else 0
+    R = np.zeros(k.shape[:2] + (s,))
+    for h in range(k.shape[0]):
         if s:
-            res = k[h] - Z[h] @ w_zk[h].astype(np.float64)
+            res = k[h] - np.asarray(z[h], dtype=np.float64) @ w_zk[h].astype(np.float64)
             R[h] = _round_to_storage(res @ np.linalg.pinv(b_r[h].astype(np.float64)), dtype)
-    return Z, R
+    return R
 
 
 def set_threads(n: int) -> None:
