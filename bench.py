@@ -412,7 +412,7 @@ def run_ours(args, rank, world, local):
             "gpu_launches": K * launches_per_step,
             "e2e": {"value": tokens * world / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_s * 1e3,
-                    "how": "basiskv_decode_attn_host: pinned q H2D, decode, out+sel D2H, stream sync; host wall clock"},
+                    "how": "basiskv_decode_attn_host: pinned q H2D, decode writing out+sel into pinned host memory, stream sync; host wall clock"},
             "wall_ms_per_step_incl_flush": wall * 1e3 / K,
             "clocks": clocks,
             "device_status": status,

@@ -863,11 +863,26 @@ int basiskv_decode_attn_host(basiskv_handle* h, int batch, const void* q_host, i
   cudaStream_t st = (cudaStream_t)stream;
   const size_t rows = (size_t)batch * h->p.num_kv_heads * h->p.gqa_group;
   CUDA_TRY(cudaMemcpyAsync(h->d_q_stage, q_host, h->elem * rows * h->p.head_dim, cudaMemcpyHostToDevice, st));
-  rc = basiskv_decode_attn(h, batch, h->d_q_stage, topk, softmax_scale, h->d_out_stage,
-                           sel_host ? h->d_sel_stage : nullptr, stream);
+  // Pinned (page-locked) result buffers are written by the kernels through
+  // their device mapping, so no copy follows the step; pageable ones go
+  // through the library's staging buffers.
+  auto mapped = [](void* host) -> void* {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, host) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    return at.type == cudaMemoryTypeHost ? at.devicePointer : nullptr;
+  };
+  float* dout = static_cast<float*>(mapped(out_host));
+  int32_t* dsel = sel_host ? static_cast<int32_t*>(mapped(sel_host)) : nullptr;
+  rc = basiskv_decode_attn(h, batch, h->d_q_stage, topk, softmax_scale, dout ? dout : h->d_out_stage,
+                           sel_host ? (dsel ? dsel : h->d_sel_stage) : nullptr, stream);
   if (rc) return rc;
-  CUDA_TRY(cudaMemcpyAsync(out_host, h->d_out_stage, sizeof(float) * rows * h->p.head_dim, cudaMemcpyDeviceToHost, st));
-  if (sel_host)
+  if (!dout)
+    CUDA_TRY(cudaMemcpyAsync(out_host, h->d_out_stage, sizeof(float) * rows * h->p.head_dim, cudaMemcpyDeviceToHost,
+                             st));
+  if (sel_host && !dsel)
     CUDA_TRY(cudaMemcpyAsync(sel_host, h->d_sel_stage, sizeof(int32_t) * batch * h->p.num_kv_heads * topk,
                              cudaMemcpyDeviceToHost, st));
   CUDA_TRY(cudaStreamSynchronize(st));

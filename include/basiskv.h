@@ -174,8 +174,10 @@ BASISKV_API int basiskv_decode_attn_latent(basiskv_handle *h, int batch, const v
                                basiskv_stream_t stream);
 
 /* The same step with HOST buffers: copies q_host (pinned or pageable) to a
- * library-owned device buffer, runs basiskv_decode_attn, copies out (and
- * sel when sel_host is not NULL) back, and waits for the stream. */
+ * library-owned device buffer, runs basiskv_decode_attn and waits for the
+ * stream.  out_host (and sel_host when not NULL) are written by the kernels
+ * through their device mapping when they are pinned, else copied back from
+ * library-owned buffers. */
 BASISKV_API int basiskv_decode_attn_host(basiskv_handle *h, int batch, const void *q_host, int topk,
                              float softmax_scale, float *out_host, int32_t *sel_host,
                              basiskv_stream_t stream);

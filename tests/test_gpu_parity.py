@@ -262,6 +262,25 @@ def test_latent_output_edge_lengths_and_large_batch():
         assert (zbar[empty] == 0).all() and (sel[empty] == -1).all()
 
 
+def test_shared_prefix_pages():
+    """Sequences whose page tables point at the same slots for a common prefix
+    (pages shared between sequences, as a prompt cache would): each sequence
+    routes and attends over its own table; the shared slots are read where
+    they are referenced."""
+    spec = W.shrink("llama3_8b_decode", batch=4, len_lo=3000, len_hi=4000, topk=12)
+    w = W.generate(spec, device="cuda")
+    pt = w.page_table.copy()
+    prefix = 20
+    for b in range(1, 4):
+        pt[b, :prefix] = pt[0, :prefix]
+    w.page_table = pt
+    prob = to_problem(w)
+    ref_out, ref_sel, _, _ = oracle.decode(prob)
+    out, sel = gpu_decode(w)
+    assert np.array_equal(sel, ref_sel)
+    assert out_error(out, ref_out) <= OUT_TOL
+
+
 def test_exact_ties_go_to_lower_page():
     """Logical pages sharing a physical slot score exactly the same."""
     spec = W.shrink("llama3_8b_decode", batch=2, len_lo=64 * 40, len_hi=64 * 40, topk=6)
@@ -285,11 +304,14 @@ def test_deterministic_and_host_entry_point():
     o1, s1 = gpu_decode(w, kv=kv)
     o2, s2 = gpu_decode(w, kv=kv)
     assert np.array_equal(o1, o2) and np.array_equal(s1, s2)
-    qh = w.q.cpu().pin_memory()
-    oh = torch.empty((s.batch, s.num_q_heads, s.head_dim), dtype=torch.float32).pin_memory()
-    sh = torch.empty((s.batch, s.num_kv_heads, s.topk), dtype=torch.int32).pin_memory()
-    bk.basiskv_decode_attn_host(kv.handle, qh, s.topk, s.softmax_scale, oh, sh)
-    assert np.array_equal(oh.numpy(), o1) and np.array_equal(sh.numpy(), s1)
+    for pinned in (True, False):  # kernels write pinned results in place; pageable ones are copied back
+        qh = w.q.cpu()
+        oh = torch.full((s.batch, s.num_q_heads, s.head_dim), float("nan"), dtype=torch.float32)
+        sh = torch.full((s.batch, s.num_kv_heads, s.topk), -7, dtype=torch.int32)
+        if pinned:
+            qh, oh, sh = qh.pin_memory(), oh.pin_memory(), sh.pin_memory()
+        bk.basiskv_decode_attn_host(kv.handle, qh, s.topk, s.softmax_scale, oh, sh)
+        assert np.array_equal(oh.numpy(), o1) and np.array_equal(sh.numpy(), s1)
     kv.close()
 
 
