@@ -31,6 +31,13 @@
  * Pool layouts (row-major):  z_pool [slots][Hkv][P][r]
  *                            r_pool [slots][Hkv][P][s]
  *                            k_pool [slots][Hkv][P][d]
+ *   Keys may instead be stored as int8 codes with one fp32 scale per token
+ *   (k_format = ORACLE_KEYS_INT8): k_pool [slots][Hkv][P][d] int8 and
+ *   k_scale [slots][Hkv][P]; the key is then K_t = k_scale_t * code_t.  This
+ *   follows the lossy key compression with fused decompression of "PackKV:
+ *   Reducing KV Cache Memory Footprint through LLM-Aware Lossy Compression"
+ *   (abstract), read as symmetric per-token int8; the oracle widens code and
+ *   scale exactly and forms their product in double.
  *   query q [B][Hkv*G][d] in the pool dtype; query head h of KV head kvh is
  *   q[b][kvh*G + h].  Bases are fp32: w_zk [Hkv][r][d], b_r [Hkv][s][d],
  *   b_v [Hkv][r][d].  page_table [B][ld_pt] holds the slot of logical page j
@@ -45,6 +52,7 @@
 #endif
 
 enum { ORACLE_BF16 = 0, ORACLE_F32 = 1 };
+enum { ORACLE_KEYS_NATIVE = 0, ORACLE_KEYS_INT8 = 1 };
 
 /* Shape and pointers of one problem.  Mirrored field by field by the ctypes
  * structure in oracle.py. */
@@ -52,8 +60,10 @@ typedef struct {
     int32_t batch, num_kv_heads, gqa_group, head_dim, page_size;
     int32_t rank_r, rank_s, topk, dtype, num_slots, ld_pt;
     int32_t latent; /* nonzero: out holds zbar [G][r] per unit, before B_v */
+    int32_t k_format; /* ORACLE_KEYS_*: keys in the pool dtype, or int8 codes */
     double softmax_scale;
     const void *q, *z_pool, *r_pool, *k_pool;
+    const float *k_scale; /* [slots][Hkv][P] when k_format = ORACLE_KEYS_INT8 */
     const float *w_zk, *b_r, *b_v;
     const int32_t *page_table, *seq_lens;
     const uint8_t *unit_mask; /* [B][Hkv], nonzero = compute; NULL = all */
@@ -67,6 +77,16 @@ static double widen(const void *base, size_t idx, int dtype)
     float f;
     memcpy(&f, &bits, sizeof f);
     return (double)f;
+}
+
+/* Element c of the key stored in pool row `row` (row = offset of the row's
+ * element 0 divided by d): the pool value, or code times the row's scale. */
+static double key_value(const oracle_problem *p, size_t row, int c)
+{
+    const size_t idx = row * (size_t)p->head_dim + c;
+    if (p->k_format == ORACLE_KEYS_INT8)
+        return (double)((const int8_t *)p->k_pool)[idx] * (double)p->k_scale[row];
+    return widen(p->k_pool, idx, p->dtype);
 }
 
 /* Offset of element 0 of token i of page `slot`, KV head kvh, in a pool whose
@@ -83,6 +103,8 @@ static int check_problem(const oracle_problem *p)
         p->num_slots < 0 || p->ld_pt < 0)
         return -1;
     if (p->dtype != ORACLE_BF16 && p->dtype != ORACLE_F32)
+        return -1;
+    if (p->k_format != ORACLE_KEYS_NATIVE && (p->k_format != ORACLE_KEYS_INT8 || !p->k_scale))
         return -1;
     for (int b = 0; b < p->batch; ++b) {
         int L = p->seq_lens[b];
@@ -219,10 +241,10 @@ static void attend_unit(const oracle_problem *p, int b, int kvh, const int32_t *
             const int slot = p->page_table[(size_t)b * p->ld_pt + j];
             for (int a = 0; a < P; ++a) {
                 if (j * P + a >= L) break;
-                const size_t krow = pool_row(p, slot, kvh, a, d);
+                const size_t krow = pool_row(p, slot, kvh, a, 1);
                 double dot = 0.0;
                 for (int c = 0; c < d; ++c)
-                    dot += qh[c] * widen(p->k_pool, krow + c, p->dtype);
+                    dot += qh[c] * key_value(p, krow, c);
                 score[m] = p->softmax_scale * dot;
                 zrow[m] = pool_row(p, slot, kvh, a, r);
                 ++m;

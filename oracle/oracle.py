@@ -31,6 +31,8 @@ _LIB = os.path.join(_HERE, "libbasiskv_oracle.so")
 
 BF16 = 0
 F32 = 1
+KEYS_NATIVE = 0
+KEYS_INT8 = 1
 
 
 def build(force: bool = False) -> str:
@@ -52,9 +54,11 @@ class _Problem(ctypes.Structure):
         ("rank_s", ctypes.c_int32), ("topk", ctypes.c_int32),
         ("dtype", ctypes.c_int32), ("num_slots", ctypes.c_int32),
         ("ld_pt", ctypes.c_int32), ("latent", ctypes.c_int32),
+        ("k_format", ctypes.c_int32),
         ("softmax_scale", ctypes.c_double),
         ("q", ctypes.c_void_p), ("z_pool", ctypes.c_void_p),
         ("r_pool", ctypes.c_void_p), ("k_pool", ctypes.c_void_p),
+        ("k_scale", ctypes.c_void_p),
         ("w_zk", ctypes.c_void_p), ("b_r", ctypes.c_void_p), ("b_v", ctypes.c_void_p),
         ("page_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
         ("unit_mask", ctypes.c_void_p),
@@ -94,6 +98,8 @@ class Problem:
     Layouts: q [B][Hkv*G][d]; z_pool [slots][Hkv][P][r]; r_pool [slots][Hkv][P][s];
     k_pool [slots][Hkv][P][d]; w_zk [Hkv][r][d], b_r [Hkv][s][d], b_v [Hkv][r][d]
     (fp32); page_table [B][ld_pt] int32; seq_lens [B] int32.
+    With ``k_scale`` [slots][Hkv][P] float32 given, k_pool holds int8 key
+    codes and the key of a row is its scale times its codes.
     """
     q: np.ndarray
     z_pool: np.ndarray
@@ -109,6 +115,7 @@ class Problem:
     softmax_scale: float
     dtype: int  # BF16 (raw 16-bit patterns) or F32
     latent: bool = False  # outputs zbar [B][Hq][r] (before B_v) instead of [B][Hq][d]
+    k_scale: np.ndarray | None = None  # per-token key scales: k_pool holds int8 codes
 
     def __post_init__(self):
         conv = (lambda a: np.ascontiguousarray(a).view(np.uint16)) if self.dtype == BF16 else \
@@ -116,7 +123,15 @@ class Problem:
         self.q = conv(self.q)
         self.z_pool = conv(self.z_pool)
         self.r_pool = conv(self.r_pool)
-        self.k_pool = conv(self.k_pool)
+        if self.k_scale is None:
+            self.k_pool = conv(self.k_pool)
+        else:
+            if np.asarray(self.k_pool).dtype != np.int8:
+                raise ValueError("with k_scale, k_pool must hold int8 codes")
+            self.k_pool = np.ascontiguousarray(self.k_pool)
+            self.k_scale = np.ascontiguousarray(self.k_scale, dtype=np.float32)
+            if self.k_scale.shape != self.k_pool.shape[:3]:
+                raise ValueError("k_scale must be [slots][Hkv][P]")
         self.w_zk = np.ascontiguousarray(self.w_zk, dtype=np.float32)
         self.b_r = np.ascontiguousarray(self.b_r, dtype=np.float32)
         self.b_v = np.ascontiguousarray(self.b_v, dtype=np.float32)
@@ -163,11 +178,13 @@ class Problem:
         p.num_slots = int(self.z_pool.shape[0])
         p.ld_pt = int(self.page_table.shape[1])
         p.latent = int(bool(self.latent))
+        p.k_format = KEYS_NATIVE if self.k_scale is None else KEYS_INT8
         p.softmax_scale = float(self.softmax_scale)
         p.q = self.q.ctypes.data
         p.z_pool = self.z_pool.ctypes.data
         p.r_pool = self.r_pool.ctypes.data if self.r_pool.size else None
         p.k_pool = self.k_pool.ctypes.data
+        p.k_scale = self.k_scale.ctypes.data if self.k_scale is not None else None
         p.w_zk = self.w_zk.ctypes.data
         p.b_r = self.b_r.ctypes.data if self.b_r.size else None
         p.b_v = self.b_v.ctypes.data
@@ -270,6 +287,31 @@ def encode_residual(k: np.ndarray, z: np.ndarray, w_zk: np.ndarray, b_r: np.ndar
             res = k[h] - np.asarray(z[h], dtype=np.float64) @ w_zk[h].astype(np.float64)
             R[h] = _round_to_storage(res @ np.linalg.pinv(b_r[h].astype(np.float64)), dtype)
     return R
+
+
+def quantize_keys(k: np.ndarray):
+    """int8 codes and per-row scales of keys k [..., d] (the stored values,
+    as float32 or float64 that float32 holds exactly).
+
+    Lossy key compression in the manner of "PackKV: Reducing KV Cache Memory
+    Footprint through LLM-Aware Lossy Compression" (abstract: keys are stored
+    compressed, and decompression is folded into the attention product),
+    read as symmetric int8 with one scale per token:
+        scale = max_c |k_c| / 127        (IEEE float32 division)
+        code  = rint(k_c / scale)        (float32 division, ties to even)
+    so the largest entry maps to +-127 and a row of zeros has scale 0 and
+    codes 0.  Every step is done in float32, the precision the decision is
+    taken in.  Returns (codes int8 [..., d], scales float32 [...])."""
+    k = np.asarray(k)
+    kf = k.astype(np.float32)
+    if not np.array_equal(kf.astype(np.float64), np.asarray(k, dtype=np.float64)):
+        raise ValueError("keys must be exactly representable in float32")
+    amax = np.abs(kf).max(axis=-1)
+    scale = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    q = np.rint((kf / safe[..., None]).astype(np.float32))
+    q = np.where(scale[..., None] > 0, q, 0)
+    return np.clip(q, -127, 127).astype(np.int8), scale
 
 
 def set_threads(n: int) -> None:

@@ -504,4 +504,138 @@ def pin_masked_tail(lib):
         assert np.array_equal(x, y)
 
 
+# ---- keys stored as int8 codes with one scale per token ---------------------
+def _int8_keys(prob, codes, scales):
+    return dataclasses.replace(prob, k_pool=codes, k_scale=scales)
+
+
+def _grid_keys(rng, shape):
+    """Keys that int8 with a per-row scale holds exactly: integer codes in
+    [-127, 127] with one entry of each row at +-127, times a power of two."""
+    codes = rng.integers(-127, 128, size=shape).astype(np.int8)
+    flat = codes.reshape(-1, shape[-1])
+    flat[np.arange(flat.shape[0]), rng.integers(0, shape[-1], size=flat.shape[0])] = \
+        rng.choice(np.array([-127, 127], dtype=np.int8), size=flat.shape[0])
+    scales = np.ldexp(1.0, rng.integers(-12, 3, size=shape[:-1])).astype(np.float32)
+    return codes, scales, (codes.astype(np.float64) * scales[..., None]).astype(np.float32)
+
+
+def pin_int8_keys_exact_grid(lib):
+    """Keys on an int8 grid: the quantizer returns that grid (codes and
+    scales), and decoding with the codes gives the very same selection, page
+    scores and output as decoding with the float keys (the product code x
+    scale is the key itself)."""
+    rng = np.random.default_rng(31)
+    prob = make_problem(rng, B=3, Hkv=2, G=2, d=8, P=4, r=4, s=2, lens=(14, 5, 0), topk=2)
+    codes, scales, keys = _grid_keys(rng, prob.k_pool.shape)
+    c2, s2 = oracle.quantize_keys(keys)
+    assert np.array_equal(c2, codes) and np.array_equal(s2, scales)
+    ref = oracle.decode(dataclasses.replace(prob, k_pool=keys), library=lib, want_scores=True)
+    got = oracle.decode(_int8_keys(prob, codes, scales), library=lib, want_scores=True)
+    assert np.array_equal(ref[0], got[0]) and np.array_equal(ref[1], got[1])
+    assert np.array_equal(ref[2], got[2])
+
+
+def pin_int8_two_tokens(lib):
+    """L = 2 in one page with int8 keys: out = sigma(D) Z_0 + (1 - sigma(D)) Z_1
+    (then B_v) with D = scale * q.(s_0 c_0 - s_1 c_1), written out by hand."""
+    rng = np.random.default_rng(37)
+    prob = make_problem(rng, B=1, Hkv=1, G=2, d=8, P=4, r=4, s=2, lens=(2,), topk=1, scale=0.3)
+    codes = rng.integers(-127, 128, size=prob.k_pool.shape).astype(np.int8)
+    scales = rng.uniform(0.001, 0.05, size=prob.k_pool.shape[:3]).astype(np.float32)
+    out, _, _, _ = oracle.decode(_int8_keys(prob, codes, scales), library=lib)
+    slot = prob.page_table[0, 0]
+    c0, c1 = codes[slot, 0, 0].astype(np.float64), codes[slot, 0, 1].astype(np.float64)
+    s0, s1 = float(scales[slot, 0, 0]), float(scales[slot, 0, 1])
+    Z = widen(prob.z_pool, prob.dtype)[slot, 0]
+    q = widen(prob.q, prob.dtype)[0]
+    for h in range(2):
+        D = 0.3 * (s0 * (q[h] @ c0) - s1 * (q[h] @ c1))
+        sg = 1.0 / (1.0 + math.exp(-D))
+        expect = (sg * Z[0] + (1 - sg) * Z[1]) @ prob.b_v[0].astype(np.float64)
+        assert rel_err(out[0, h], expect) < 1e-13
+
+
+def pin_int8_keys_dense_limit(lib):
+    """Every page selected, int8 keys: exact softmax attention over the
+    dequantised keys K_t = s_t c_t (brute force, every valid token)."""
+    rng = np.random.default_rng(41)
+    prob = make_problem(rng, B=2, Hkv=2, G=3, d=8, P=4, r=8, s=0, lens=(11, 6), topk=4, bv_identity=True)
+    codes = rng.integers(-127, 128, size=prob.k_pool.shape).astype(np.int8)
+    scales = rng.uniform(0.001, 0.05, size=prob.k_pool.shape[:3]).astype(np.float32)
+    out, _, _, _ = oracle.decode(_int8_keys(prob, codes, scales), library=lib)
+    deq = codes.astype(np.float64) * scales[..., None].astype(np.float64)  # [slots][Hkv][P][d]
+    Z = widen(prob.z_pool, prob.dtype)
+    q = widen(prob.q, prob.dtype)
+    for b in range(2):
+        L = int(prob.seq_lens[b])
+        toks = [(int(prob.page_table[b, t // 4]), t % 4) for t in range(L)]
+        for kvh in range(2):
+            K = np.stack([deq[sl, kvh, i] for sl, i in toks])
+            V = np.stack([Z[sl, kvh, i] for sl, i in toks])  # B_v = I
+            for h in range(3):
+                logits = prob.softmax_scale * (K @ q[b, kvh * 3 + h])
+                w = np.exp(logits - logits.max())
+                assert rel_err(out[b, kvh * 3 + h], (w / w.sum()) @ V) < 1e-12
+
+
+def pin_int8_routing_reads_no_keys(lib):
+    """Routing uses only Z and R: int8 keys of any content leave the page
+    scores and the selection of the float-key problem unchanged."""
+    rng = np.random.default_rng(43)
+    prob = make_problem(rng, B=2, Hkv=2, G=2, d=8, P=4, r=4, s=2, lens=(15, 9), topk=2)
+    codes = rng.integers(-127, 128, size=prob.k_pool.shape).astype(np.int8)
+    scales = rng.uniform(0.0, 3.0, size=prob.k_pool.shape[:3]).astype(np.float32)
+    a = oracle.route(prob, library=lib)
+    b = oracle.route(_int8_keys(prob, codes, scales), library=lib)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
+
+
+# ---- the key quantizer (host side of the oracle, numpy) ---------------------
+def qpin_hand_rows(quantize):
+    """Hand rows with exact scales (max 15.875 = 127 / 8, so scale = 1/8):
+    entries 2.5 and 3.5 scales away tie and go to the even code, the largest
+    entry maps to +-127, a row of zeros has scale 0 and codes 0, and a lone
+    negative maximum maps to -127."""
+    rows = np.array([[15.875, 0.3125, 0.4375, -0.3125, -0.4375, 0.0, 1.0, -15.875],
+                     [0.0] * 8,
+                     [0.0, -3.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0],
+                     [111.125, 5.6875, -5.6875, 10.9375, 0.0, 0.0, 0.0, 0.0]], dtype=np.float32)
+    c, s = quantize(rows)
+    assert c.dtype == np.int8 and s.dtype == np.float32
+    assert c[0].tolist() == [127, 2, 4, -2, -4, 0, 8, -127], c[0]
+    assert s[0] == np.float32(0.125)
+    # scale 111.125 / 127 = 0.875 exactly; 5.6875 and 10.9375 are 6.5 and 12.5
+    # scales, exact ties that a quotient formed through the float32 reciprocal
+    # of the scale misses
+    assert s[3] == np.float32(0.875) and c[3].tolist() == [127, 6, -6, 12, 0, 0, 0, 0], c[3]
+    assert s[1] == 0 and (c[1] == 0).all()
+    assert c[2].tolist() == [0, -127, 0, 0, 0, 0, 0, 0] and s[2] == np.float32(np.float32(3.0) / np.float32(127.0))
+
+
+def qpin_error_bound(quantize):
+    """Random rows (bf16-like magnitudes with outlier channels): every code is
+    within half a step of k / scale (float32 rounding aside), the largest
+    |code| of every row is 127, and the scale is max|k| / 127 in float32."""
+    rng = np.random.default_rng(47)
+    k = (rng.standard_normal((64, 128)) * np.exp(rng.normal(0, 0.5, 128))).astype(np.float32)
+    c, s = quantize(k)
+    assert np.array_equal(s, (np.abs(k).max(axis=1) / np.float32(127.0)).astype(np.float32))
+    dev = np.abs(c.astype(np.float64) - k.astype(np.float64) / s[:, None].astype(np.float64))
+    assert dev.max() <= 0.5 + 1e-5, dev.max()
+    assert (np.abs(c.astype(np.int32)).max(axis=1) == 127).all()
+
+
+def qpin_shape_and_grid(quantize):
+    """Leading dimensions are kept and exact grids come back unchanged."""
+    rng = np.random.default_rng(53)
+    codes, scales, keys = _grid_keys(rng, (3, 2, 4, 16))
+    c, s = quantize(keys)
+    assert c.shape == codes.shape and s.shape == scales.shape
+    assert np.array_equal(c, codes) and np.array_equal(s, scales)
+
+
+QPINS = [v for k, v in sorted(globals().items()) if k.startswith("qpin_")]

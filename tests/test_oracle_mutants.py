@@ -34,8 +34,8 @@ MUTANTS = [
      "const size_t qoff = ((size_t)b * p->num_kv_heads * G + (size_t)h * p->num_kv_heads + kvh) * d;"),
     ("route_ignores_page_table", "const size_t zrow = pool_row(p, slot, kvh, i, r);",
      "const size_t zrow = pool_row(p, j, kvh, i, r);"),
-    ("attend_ignores_page_table", "const size_t krow = pool_row(p, slot, kvh, a, d);",
-     "const size_t krow = pool_row(p, j, kvh, a, d);"),
+    ("attend_ignores_page_table", "const size_t krow = pool_row(p, slot, kvh, a, 1);",
+     "const size_t krow = pool_row(p, j, kvh, a, 1);"),
     ("selection_unsorted", "qsort(chosen, (size_t)kb, sizeof(int), int_cmp);", ""),
     ("bf16_low_half", "uint32_t bits = (uint32_t)((const uint16_t *)base)[idx] << 16;",
      "uint32_t bits = (uint32_t)((const uint16_t *)base)[idx];"),
@@ -46,6 +46,10 @@ MUTANTS = [
      "        for (int a = 0; a < r; ++a) zbar[a] /= den;\n        if (p->latent) {"),
     ("head_rows_shifted", "double *o = out + (size_t)h * width;",
      "double *o = out + (size_t)(h > 0 ? h - 1 : 0) * width;"),
+    ("int8_scale_ignored", "(double)((const int8_t *)p->k_pool)[idx] * (double)p->k_scale[row];",
+     "(double)((const int8_t *)p->k_pool)[idx];"),
+    ("int8_scale_per_page", "(double)p->k_scale[row];", "(double)p->k_scale[row / p->page_size];"),
+    ("int8_codes_unsigned", "(double)((const int8_t *)p->k_pool)[idx]", "(double)((const uint8_t *)p->k_pool)[idx]"),
     ("kv_head_stride_in_pool", "return (((size_t)slot * p->num_kv_heads + kvh) * p->page_size + i) * (size_t)width;",
      "return (((size_t)slot * p->num_kv_heads) * p->page_size + i) * (size_t)width;"),
 ]
@@ -73,3 +77,36 @@ def test_mutant_is_caught(tmp_path, source, name, old, new):
         except (AssertionError, ValueError):
             failed.append(pin.__name__)
     assert failed, f"mutant {name} passed every pin"
+
+
+# Mistakes planted in a copy of the numpy key quantizer; each must fail one
+# of the quantizer pins.
+PY_MUTANTS = [
+    ("round_half_away", "q = np.rint((kf / safe[..., None]).astype(np.float32))",
+     "q = np.trunc((kf / safe[..., None]).astype(np.float32) + np.copysign(0.5, kf))"),
+    ("scale_over_128", "scale = (amax / np.float32(127.0)).astype(np.float32)",
+     "scale = (amax / np.float32(128.0)).astype(np.float32)"),
+    ("truncate_codes", "q = np.rint((kf / safe[..., None]).astype(np.float32))",
+     "q = np.trunc((kf / safe[..., None]).astype(np.float32))"),
+    ("max_not_abs", "amax = np.abs(kf).max(axis=-1)", "amax = kf.max(axis=-1)"),
+    ("reciprocal_multiply", "q = np.rint((kf / safe[..., None]).astype(np.float32))",
+     "q = np.rint((kf * (np.float32(1.0) / safe[..., None])).astype(np.float32))"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", PY_MUTANTS, ids=[m[0] for m in PY_MUTANTS])
+def test_quantizer_mutant_is_caught(name, old, new):
+    import inspect
+    import textwrap
+    import numpy as np
+    src = textwrap.dedent(inspect.getsource(oracle.quantize_keys))
+    assert src.count(old) == 1, f"mutation anchor for {name} not found"
+    ns = {"np": np}
+    exec(compile(src.replace(old, new), f"<{name}>", "exec"), ns)
+    failed = []
+    for pin in oracle_pins.QPINS:
+        try:
+            pin(ns["quantize_keys"])
+        except (AssertionError, ValueError):
+            failed.append(pin.__name__)
+    assert failed, f"mutant {name} passed every quantizer pin"
