@@ -4,8 +4,11 @@ One step = one ``basiskv_decode_attn`` call (routing scores + top-k, exact QK
 on the selected pages, softmax, latent sum, combine and B_v) for every
 (sequence, KV head) of the workload, inputs resident in HBM.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--keys int8]
     python bench.py --impl reference ...     # the float64 CPU oracle arm
+
+``--keys int8`` stores the original keys as int8 codes with a per-token scale
+(quantised on the device before timing) instead of bf16.
 
 Prints one JSON line (rank 0).  Multi-GPU: one process per GPU under
 torchrun; every rank runs its own replica of the workload (no collective on
@@ -41,6 +44,8 @@ def parse():
     ap.add_argument("--workload", default="llama3_8b_decode")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller profiling cases)")
+    ap.add_argument("--keys", choices=["native", "int8"], default="native",
+                    help="int8: keys as int8 codes with a per-token scale")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     return ap.parse_args()
@@ -97,10 +102,13 @@ def aggregate(tokens_per_rank: int, ms_per_step: float, world: int, device=None)
 def workload_config(args, w, world):
     """The workload part of the JSON line's config, the same for both arms."""
     s = w.spec
-    return {"workload": args.workload if not args.batch else f"{args.workload}[batch={s.batch}]",
+    int8 = getattr(args, "keys", "native") == "int8"
+    name = args.workload if not args.batch else f"{args.workload}[batch={s.batch}]"
+    return {"workload": name + ("+int8_keys" if int8 else ""),
+            "keys": "int8 codes + fp32 scale per token" if int8 else s.dtype,
             "batch": s.batch, "kv_heads": s.num_kv_heads, "q_heads": s.num_q_heads, "head_dim": s.head_dim,
             "page": s.page_size, "rank_r": s.rank_r, "rank_s": s.rank_s, "topk": s.topk,
-            "context_tokens": w.context_tokens, "algorithmic_bytes": w.algorithmic_bytes()["total"],
+            "context_tokens": w.context_tokens, "algorithmic_bytes": w.algorithmic_bytes(int8)["total"],
             "parallelism": f"replicas x{world}, no data-path collective"}
 
 
@@ -181,8 +189,9 @@ def ncu_traffic(kernel: str, workload: str):
         return None
 
 
-def oracle_problem(w):
-    """Host copies of a workload's stored tensors for the oracle."""
+def oracle_problem(w, int8_keys=False):
+    """Host copies of a workload's stored tensors for the oracle; with
+    int8_keys, the keys quantised by the oracle's own quantiser."""
     import torch
     from oracle import oracle
     s = w.spec
@@ -192,12 +201,22 @@ def oracle_problem(w):
         t = t.detach().cpu().contiguous()
         return t.view(torch.int16).numpy() if bf16 else t.numpy()
 
+    k = host(w.k_pool)
+    k_scale = None
+    if int8_keys:
+        codes = np.empty(k.shape, np.int8)
+        k_scale = np.empty(k.shape[:3], np.float32)
+        for i in range(0, k.shape[0], 256):  # slot chunks bound the float temporaries
+            kf = (k[i:i + 256].view(np.uint16).astype(np.uint32) << 16).view(np.float32) if bf16 \
+                else k[i:i + 256]
+            codes[i:i + 256], k_scale[i:i + 256] = oracle.quantize_keys(kf)
+        k = codes
     return oracle.Problem(
-        q=host(w.q), z_pool=host(w.z_pool), r_pool=host(w.r_pool), k_pool=host(w.k_pool),
+        q=host(w.q), z_pool=host(w.z_pool), r_pool=host(w.r_pool), k_pool=k,
         w_zk=w.w_zk.cpu().numpy(), b_r=w.b_r.cpu().numpy(), b_v=w.b_v.cpu().numpy(),
         page_table=np.where(w.page_table >= 0, w.page_table, 0).astype(np.int32),
         seq_lens=w.seq_lens, gqa_group=s.gqa_group, topk=s.topk, softmax_scale=s.softmax_scale,
-        dtype=oracle.BF16 if bf16 else oracle.F32)
+        dtype=oracle.BF16 if bf16 else oracle.F32, k_scale=k_scale)
 
 
 def cpu_oracle_timing(prob, w, budget_s: float):
@@ -235,7 +254,7 @@ def run_reference(args, rank, world):
     if args.batch:
         spec = spec.with_(batch=args.batch)
     w = W.generate(spec, device="cuda" if torch.cuda.is_available() else "cpu")
-    prob = oracle_problem(w)
+    prob = oracle_problem(w, args.keys == "int8")
     cores = oracle.max_threads()
     # per-step sample: unit 0 on every thread, sequence cut so the whole run
     # stays near two minutes
@@ -295,7 +314,19 @@ def run_ours(args, rank, world, local):
         spec = spec.with_(batch=args.batch)
     spec = replica_spec(spec, rank)
     w = W.generate(spec, device=dev)
-    kv = bk.BasisKV.for_workload(w)
+    int8 = args.keys == "int8"
+    if int8:
+        # the keys as int8 codes and per-token scales, quantised on the device
+        codes = torch.empty(tuple(w.k_pool.shape), dtype=torch.int8, device=dev)
+        k_scale = torch.empty(tuple(w.k_pool.shape[:3]), dtype=torch.float32, device=dev)
+        kv = bk.BasisKV(z_pool=w.z_pool, r_pool=w.r_pool, k_pool=codes, w_zk=w.w_zk, b_r=w.b_r, b_v=w.b_v,
+                        gqa_group=w.spec.gqa_group, max_batch=w.spec.batch,
+                        max_pages_per_seq=max(1, w.page_table.shape[1]), max_topk=w.spec.topk, k_scale=k_scale)
+        bk.basiskv_quantize_keys(kv.handle, w.k_pool)
+        bk.basiskv_load_page_table(kv.handle, np.where(w.page_table >= 0, w.page_table, 0), w.seq_lens)
+        torch.cuda.synchronize(dev)
+    else:
+        kv = bk.BasisKV.for_workload(w)
     s = w.spec
     out = torch.empty((s.batch, s.num_q_heads, s.head_dim), device=dev, dtype=torch.float32)
     sel = torch.empty((s.batch, s.num_kv_heads, s.topk), device=dev, dtype=torch.int32)
@@ -347,7 +378,7 @@ def run_ours(args, rank, world, local):
     ms_step = float(np.mean(step_ms))
     tokens = w.context_tokens
     value, ms_step_max = aggregate(tokens, ms_step, world, dev)
-    nbytes = w.algorithmic_bytes()
+    nbytes = w.algorithmic_bytes(int8)
     hbm_peak, peak_kind = peaks()
     route_mean = float(np.mean(prof["route"])) if launch["route_ctas"] else 0.0
     attn_mean = float(np.mean(prof["attn"]))
@@ -361,7 +392,7 @@ def run_ours(args, rank, world, local):
     launches_per_step = (1 + launch["route_tensor_core"] if launch["route_ctas"] else 0) + 1 + \
         (1 if s.batch > 512 else 0)
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
-    traffic = ncu_traffic(kname, args.workload)
+    traffic = ncu_traffic(kname, args.workload + ("+int8_keys" if int8 and kname.startswith("attn") else ""))
 
     # end to end through the host-buffer entry point: q in, out (+ selection) back
     q_host = w.q.cpu().pin_memory()
@@ -385,7 +416,7 @@ def run_ours(args, rank, world, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        prob = oracle_problem(w)
+        prob = oracle_problem(w, int8)
         v, cores, sample = cpu_oracle_timing(prob, w, args.cpu_budget_s)
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
 

@@ -30,6 +30,9 @@ BASISKV_STATUS_BAD_PAGE = 4
 BASISKV_DTYPE_BF16 = 0
 BASISKV_DTYPE_F32 = 1
 
+BASISKV_KEYS_NATIVE = 0
+BASISKV_KEYS_INT8 = 1
+
 # every entry point declared in include/basiskv.h
 EXPORTED = (
     "basiskv_create", "basiskv_destroy", "basiskv_append_page", "basiskv_append_tokens",
@@ -37,6 +40,7 @@ EXPORTED = (
     "basiskv_decode_attn_host", "basiskv_route", "basiskv_get_status", "basiskv_profile_begin",
     "basiskv_profile_end", "basiskv_last_launch", "basiskv_last_error", "basiskv_version",
     "basiskv_decode_attn_noalloc", "basiskv_decode_attn_latent", "basiskv_encode_rows",
+    "basiskv_quantize_keys",
 )
 
 
@@ -47,9 +51,10 @@ class basiskv_params(ctypes.Structure):
         ("page_size", ctypes.c_int32), ("rank_r", ctypes.c_int32),
         ("rank_s", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
         ("max_topk", ctypes.c_int32), ("num_slots", ctypes.c_int32),
-        ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("dtype", ctypes.c_int32), ("k_format", ctypes.c_int32),
         ("z_pool", ctypes.c_void_p), ("r_pool", ctypes.c_void_p), ("k_pool", ctypes.c_void_p),
         ("w_zk", ctypes.c_void_p), ("b_r", ctypes.c_void_p), ("b_v", ctypes.c_void_p),
+        ("k_scale", ctypes.c_void_p),
     ]
 
 
@@ -84,6 +89,7 @@ def load(path: str = LIB_PATH):
         "basiskv_decode_attn_host": [H, i32, vp, i32, f32, vp, vp, vp],
         "basiskv_decode_attn_latent": [H, i32, vp, i32, f32, vp, vp, vp],
         "basiskv_encode_rows": [H, i32, i32, i32, vp, vp, vp],
+        "basiskv_quantize_keys": [H, vp, ctypes.c_int64, ctypes.c_int64, vp],
         "basiskv_route": [H, i32, vp, i32, vp, vp, vp],
         "basiskv_get_status": [H, ctypes.POINTER(ctypes.c_uint32), i32],
         "basiskv_profile_begin": [H, i32],
@@ -171,6 +177,14 @@ def basiskv_encode_rows(h, slot, row0, k, v, stream=None):
     _check(load().basiskv_encode_rows(h, slot, row0, int(k.shape[1]), _ptr(k), _ptr(v), _stream(stream)))
 
 
+def basiskv_quantize_keys(h, k, row0=0, stream=None):
+    """Quantise keys k [n][d] (pool dtype, device; any leading shape whose
+    rows follow the pool's flat row order) into the handle's int8 key pool
+    and scales, rows [row0, row0 + n)."""
+    n = int(k.numel() // k.shape[-1]) if k.numel() else 0
+    _check(load().basiskv_quantize_keys(h, _ptr(k), int(row0), n, _stream(stream)))
+
+
 def basiskv_decode_attn_host(h, q_host, topk, softmax_scale, out_host, sel_host=None, stream=None):
     """q_host, out_host, sel_host: host torch tensors (pinned for async copies)."""
     _check(load().basiskv_decode_attn_host(h, int(q_host.shape[0]), _ptr(q_host), topk,
@@ -236,12 +250,17 @@ class BasisKV:
     """
 
     def __init__(self, *, z_pool, r_pool, k_pool, w_zk, b_r, b_v, gqa_group, max_batch,
-                 max_pages_per_seq, max_topk):
+                 max_pages_per_seq, max_topk, k_scale=None):
+        """An int8 ``k_pool`` holds key codes and needs ``k_scale``
+        [slots][Hkv][P] fp32 (BASISKV_KEYS_INT8)."""
         import torch
         if not torch.cuda.is_available():
             raise RuntimeError("no CUDA device: the BasisKV library has no CPU path")
         bf16 = z_pool.dtype == torch.bfloat16
-        self._keep = (z_pool, r_pool, k_pool, w_zk, b_r, b_v)
+        int8_keys = k_pool.dtype == torch.int8
+        if int8_keys != (k_scale is not None):
+            raise ValueError("int8 keys and k_scale go together")
+        self._keep = (z_pool, r_pool, k_pool, w_zk, b_r, b_v, k_scale)
         p = basiskv_params()
         p.max_batch = max_batch
         p.num_kv_heads = int(z_pool.shape[1])
@@ -254,7 +273,8 @@ class BasisKV:
         p.max_topk = max_topk
         p.num_slots = int(z_pool.shape[0])
         p.dtype = BASISKV_DTYPE_BF16 if bf16 else BASISKV_DTYPE_F32
-        p.reserved = 0
+        p.k_format = BASISKV_KEYS_INT8 if int8_keys else BASISKV_KEYS_NATIVE
+        p.k_scale = _ptr(k_scale)
         p.z_pool = _ptr(z_pool)
         p.r_pool = _ptr(r_pool)
         p.k_pool = _ptr(k_pool)

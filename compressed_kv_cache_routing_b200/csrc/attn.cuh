@@ -10,14 +10,48 @@
 // the last CTA of the unit merges all partials and applies B_v.
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include "combine.cuh"
 #include "common.cuh"
 
 namespace basiskv {
 
+// ---- f16 tensor-core helpers for int8 keys -----------------------------------
+// The same product with f16 operands (A and B both f16).
+__device__ __forceinline__ void mma_k16_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                            uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Pack two floats into an f16x2 register (first argument in the low half).
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// The four int8 codes of w (two's complement, byte i = code i) as f16 pairs
+// (c0, c1) and (c2, c3), exactly.  Flipping a byte's top bit gives
+// u = c + 128 in [0, 255]; the f16 whose bits are 0x64 in the high byte and
+// u in the low byte is 1024 + u, because f16 values in [1024, 2048) are the
+// integers; subtracting 1152 = 1024 + 128 (0x6480) then leaves c, exactly.
+__device__ __forceinline__ void codes_to_f16x2(uint32_t w, uint32_t& c01, uint32_t& c23) {
+  const uint32_t u = w ^ 0x80808080u;
+  const uint32_t p01 = __byte_perm(u, 0x64646464u, 0x4140);
+  const uint32_t p23 = __byte_perm(u, 0x64646464u, 0x4342);
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(c01) : "r"(p01), "r"(0x64806480u));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(c23) : "r"(p23), "r"(0x64806480u));
+}
+
+
 struct AttnArgs {
   const void* q;             // [B][Hkv*G][d]
-  const void* k_pool;        // [slots][Hkv][P][d]
+  const void* k_pool;        // [slots][Hkv][P][d]: pool dtype, or int8 codes when k_int8
+  const float* k_scale;      // [slots][Hkv][P] per-token key scale (k_int8 only)
   const void* z_pool;        // [slots][Hkv][P][r]
   const float* b_v;          // [Hkv][r][d]
   const int32_t* page_table; // [B][ld_pt]
@@ -33,6 +67,7 @@ struct AttnArgs {
   int topk, pages_per_split, stages, np_cap;
   float scale_log2;          // softmax_scale * log2(e)
   int latent;                // write the weighted latent zbar, before B_v
+  int k_int8;                // keys are int8 codes: K_t = k_scale[t] * code_t
   // persistent tensor-core kernel only
   int batch;
   const int32_t* attn_off;   // [B+1] prefix of attention items x Hkv (from the prep grid)
@@ -123,7 +158,13 @@ __device__ __forceinline__ void attn_finish(const AttnArgs& a, const AttnUnit& a
 // acc[g] + acc[g+8] is the latent sum with ~16-bit weights; Z fragments come
 // from ldmatrix.trans.
 // Each stage carries TPS tokens of one selected page (K then Z), staged by
-// bulk copies into a per-warp ring.  At the end of its segment of a unit a
+// bulk copies into a per-warp ring.
+// Int8 keys (K8): a stage carries the codes, Z, then the TPS token scales.
+// Codes become f16 exactly in registers (codes_to_f16x2) and meet the query
+// rounded to f16 in an f16 MMA; the 16-byte load of a token row covers 64
+// channels, so the k index runs over channel 64*sp + 16*t + 4*j + e for MMA
+// j of span sp (the query fragments follow the same order), and the token's
+// scale multiplies its dot product before the softmax.  At the end of its segment of a unit a
 // warp writes one partial (m, l, acc); the warp that completes the unit
 // merges the partials and applies B_v.
 struct AttnCursor {
@@ -181,16 +222,18 @@ struct AttnCursor {
   }
 };
 
-template <int G, int D, int RR, int TPS>
+template <int G, int D, int RR, int TPS, bool K8 = false>
 __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_constant__ AttnArgs a) {
   static_assert(G >= 1 && G <= 8, "GQA group must be 1..8");
   static_assert(D % 32 == 0 && RR % 8 == 0 && TPS % 16 == 0, "shape");
+  static_assert(!K8 || D % 64 == 0, "int8 keys need d % 64 == 0");
   constexpr int DS = D / 32;     // 32-wide spans of the head dim
   constexpr int RT = RR / 8;     // n8 tiles of the latent
   constexpr int NTS = TPS / 8;   // n8 token tiles per stage
   constexpr int KBS = TPS / 16;  // k16 token blocks per stage
-  constexpr uint32_t kbytes = TPS * D * 2, zbytes = TPS * RR * 2;
-  constexpr uint32_t stage_bytes = kbytes + zbytes;
+  constexpr int KB = K8 ? 1 : 2; // bytes per key element
+  constexpr uint32_t kbytes = TPS * D * KB, zbytes = TPS * RR * 2, sbytes = K8 ? TPS * 4 : 0;
+  constexpr uint32_t stage_bytes = kbytes + zbytes + sbytes;
 
   const int P = a.page_size, S = a.stages;
   const int sub = P / TPS;
@@ -234,14 +277,36 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
   uint32_t qa[DS][2][2];
   auto load_q = [&](int u) {
     const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)u * G + (g < G ? g : 0)) * D;
+    if constexpr (K8) {
+      // f16 pairs of channels 64*sp + 16*t + [0, 16): MMA j of span sp
+      // takes (c, c+1) and (c+2, c+3) with c = 64*sp + 16*t + 4*j
+      auto h2 = [](uint32_t w) { return pack_f16(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
 #pragma unroll
-    for (int s = 0; s < DS; ++s) {
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (g < G) v = __ldg(reinterpret_cast<const uint4*>(qrow + 32 * s + 8 * t));
-      qa[s][0][0] = v.x;
-      qa[s][0][1] = v.y;
-      qa[s][1][0] = v.z;
-      qa[s][1][1] = v.w;
+      for (int sp = 0; sp < D / 64; ++sp) {
+        uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
+        if (g < G) {
+          v0 = __ldg(reinterpret_cast<const uint4*>(qrow + 64 * sp + 16 * t));
+          v1 = __ldg(reinterpret_cast<const uint4*>(qrow + 64 * sp + 16 * t + 8));
+        }
+        qa[2 * sp][0][0] = h2(v0.x);
+        qa[2 * sp][0][1] = h2(v0.y);
+        qa[2 * sp][1][0] = h2(v0.z);
+        qa[2 * sp][1][1] = h2(v0.w);
+        qa[2 * sp + 1][0][0] = h2(v1.x);
+        qa[2 * sp + 1][0][1] = h2(v1.y);
+        qa[2 * sp + 1][1][0] = h2(v1.z);
+        qa[2 * sp + 1][1][1] = h2(v1.w);
+      }
+    } else {
+#pragma unroll
+      for (int s = 0; s < DS; ++s) {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (g < G) v = __ldg(reinterpret_cast<const uint4*>(qrow + 32 * s + 8 * t));
+        qa[s][0][0] = v.x;
+        qa[s][0][1] = v.y;
+        qa[s][1][0] = v.z;
+        qa[s][1][1] = v.w;
+      }
     }
   };
   int cur_u = -1;
@@ -252,7 +317,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
   pdl_wait_primary();  // the selection is written by the previous grid
   if (count <= 0) return;
 
-  const __nv_bfloat16* kpool = static_cast<const __nv_bfloat16*>(a.k_pool);
+  const uint8_t* kpool = static_cast<const uint8_t*>(a.k_pool);
   const __nv_bfloat16* zpool = static_cast<const __nv_bfloat16*>(a.z_pool);
   const uint64_t pol = policy_evict_first();
   // lane 0 issues item i of this warp into stage i % S; the selection and
@@ -269,8 +334,9 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
     uint64_t* bar = &bars[warp][i % S];
     uint8_t* dst = ring + (size_t)(i % S) * stage_bytes;
     mbar_arrive_expect_tx(bar, stage_bytes);
-    bulk_load(dst, kpool + row0 * D, kbytes, bar, pol);
+    bulk_load(dst, kpool + row0 * D * KB, kbytes, bar, pol);
     bulk_load(dst + kbytes, zpool + row0 * RR, zbytes, bar, pol);
+    if constexpr (K8) bulk_load(dst + kbytes + zbytes, a.k_scale + row0, sbytes, bar, pol);
     ic.advance(a, sub);
   };
   AttnCursor ia;       // lane 0: the item after the next one to issue
@@ -383,22 +449,41 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;
     const int valid = cc.L - tok0s[warp][i % S];  // tokens of this stage inside the sequence
-    const __nv_bfloat16* ks = reinterpret_cast<const __nv_bfloat16*>(ring + (size_t)(i % S) * stage_bytes);
-    const __nv_bfloat16* zs = ks + TPS * D;
+    const uint8_t* stage = ring + (size_t)(i % S) * stage_bytes;
+    const __nv_bfloat16* zs = reinterpret_cast<const __nv_bfloat16*>(stage + kbytes);
 
     // exact QK for the group
     float s[NTS][2];
 #pragma unroll
     for (int nt = 0; nt < NTS; ++nt) {
       float d[4] = {0.f, 0.f, 0.f, 0.f};
-      const __nv_bfloat16* krow = ks + (nt * 8 + g) * D;
-#pragma unroll
-      for (int sp = 0; sp < DS; ++sp) {
-        const uint4 v = lds128(krow + 32 * sp + 8 * t);
-        mma_k16(d, qa[sp][0][0], 0u, qa[sp][0][1], 0u, v.x, v.y);
-        mma_k16(d, qa[sp][1][0], 0u, qa[sp][1][1], 0u, v.z, v.w);
-      }
+      const uint8_t* krow = stage + (nt * 8 + g) * D * KB;
       const int tok = nt * 8 + 2 * t;
+      if constexpr (K8) {
+#pragma unroll
+        for (int sp = 0; sp < D / 64; ++sp) {
+          const uint4 v = lds128(krow + 64 * sp + 16 * t);
+          uint32_t b0, b1;
+          codes_to_f16x2(v.x, b0, b1);
+          mma_k16_f16(d, qa[2 * sp][0][0], 0u, qa[2 * sp][0][1], 0u, b0, b1);
+          codes_to_f16x2(v.y, b0, b1);
+          mma_k16_f16(d, qa[2 * sp][1][0], 0u, qa[2 * sp][1][1], 0u, b0, b1);
+          codes_to_f16x2(v.z, b0, b1);
+          mma_k16_f16(d, qa[2 * sp + 1][0][0], 0u, qa[2 * sp + 1][0][1], 0u, b0, b1);
+          codes_to_f16x2(v.w, b0, b1);
+          mma_k16_f16(d, qa[2 * sp + 1][1][0], 0u, qa[2 * sp + 1][1][1], 0u, b0, b1);
+        }
+        const uint2 sc = lds64(stage + kbytes + zbytes + 4 * tok);
+        d[0] *= __uint_as_float(sc.x);
+        d[1] *= __uint_as_float(sc.y);
+      } else {
+#pragma unroll
+        for (int sp = 0; sp < DS; ++sp) {
+          const uint4 v = lds128(krow + 2 * (32 * sp + 8 * t));
+          mma_k16(d, qa[sp][0][0], 0u, qa[sp][0][1], 0u, v.x, v.y);
+          mma_k16(d, qa[sp][1][0], 0u, qa[sp][1][1], 0u, v.z, v.w);
+        }
+      }
       s[nt][0] = tok < valid ? d[0] * a.scale_log2 : -INFINITY;
       s[nt][1] = tok + 1 < valid ? d[1] * a.scale_log2 : -INFINITY;
     }
@@ -503,9 +588,15 @@ __global__ void __launch_bounds__(kAttnThreads) attn_generic_kernel(const __grid
     const int valid = min(P, au.L - page * P);
     for (int idx = threadIdx.x; idx < valid * G; idx += blockDim.x) {
       const int tok = idx / G, h = idx % G;
-      const T* kr = kpool + (row0 + tok) * D;
       float dot = 0.f;
-      for (int c = 0; c < D; ++c) dot = fmaf(qs[h * D + c], to_f32(kr[c]), dot);
+      if (a.k_int8) {
+        const int8_t* kc = static_cast<const int8_t*>(a.k_pool) + (row0 + tok) * D;
+        for (int c = 0; c < D; ++c) dot = fmaf(qs[h * D + c], (float)kc[c], dot);
+        dot *= a.k_scale[row0 + tok];
+      } else {
+        const T* kr = kpool + (row0 + tok) * D;
+        for (int c = 0; c < D; ++c) dot = fmaf(qs[h * D + c], to_f32(kr[c]), dot);
+      }
       sc[h * P + tok] = dot * a.scale_log2;
     }
     __syncthreads();

@@ -59,8 +59,9 @@ struct RouteKey {
 };
 struct AttnKey {
   int g, d, r, tps;
+  bool k8;  // int8 keys
   bool operator<(const AttnKey& o) const {
-    return std::tie(g, d, r, tps) < std::tie(o.g, o.d, o.r, o.tps);
+    return std::tie(g, d, r, tps, k8) < std::tie(o.g, o.d, o.r, o.tps, o.k8);
   }
 };
 
@@ -80,11 +81,16 @@ const std::map<RouteKey, KernelFn>& route_table() {
 
 const std::map<AttnKey, AttnFn>& attn_table() {
   static const std::map<AttnKey, AttnFn> t = {
-#define AK(G, D, R, T) {AttnKey{G, D, R, T}, &attn_mma_kernel<G, D, R, T>}
+#define AK(G, D, R, T) {AttnKey{G, D, R, T, false}, &attn_mma_kernel<G, D, R, T, false>}
+#define AK8(G, D, R, T) {AttnKey{G, D, R, T, true}, &attn_mma_kernel<G, D, R, T, true>}
       AK(4, 128, 32, 64), AK(4, 128, 32, 32), AK(4, 128, 24, 32), AK(4, 128, 24, 16),
       AK(4, 128, 16, 64), AK(4, 128, 64, 32), AK(4, 128, 128, 32), AK(4, 128, 128, 16),
       AK(4, 64, 16, 16),  AK(4, 64, 32, 32),  AK(8, 128, 32, 64), AK(8, 128, 32, 32),
       AK(8, 128, 24, 32), AK(8, 128, 64, 32), AK(2, 128, 32, 64), AK(1, 128, 32, 64),
+      AK8(4, 128, 32, 64), AK8(4, 128, 32, 32), AK8(4, 128, 24, 32), AK8(4, 128, 24, 16),
+      AK8(4, 128, 128, 32), AK8(4, 128, 128, 16), AK8(4, 64, 16, 16), AK8(4, 64, 32, 32),
+      AK8(8, 128, 32, 32), AK8(1, 128, 32, 64),
+#undef AK8
 #undef AK
   };
   return t;
@@ -205,7 +211,10 @@ int validate_params(const basiskv_params* p) {
     return fail(BASISKV_ERR_INVALID_ARG, "max_batch and num_kv_heads must be <= 65535");
   if (p->dtype != BASISKV_DTYPE_BF16 && p->dtype != BASISKV_DTYPE_F32)
     return fail(BASISKV_ERR_INVALID_ARG, "dtype must be BASISKV_DTYPE_BF16 or BASISKV_DTYPE_F32");
-  if (p->reserved != 0) return fail(BASISKV_ERR_INVALID_ARG, "reserved must be 0");
+  if (p->k_format != BASISKV_KEYS_NATIVE && p->k_format != BASISKV_KEYS_INT8)
+    return fail(BASISKV_ERR_INVALID_ARG, "k_format must be BASISKV_KEYS_NATIVE or BASISKV_KEYS_INT8");
+  if (p->k_format == BASISKV_KEYS_INT8 && (!p->k_scale || !aligned16(p->k_scale)))
+    return fail(BASISKV_ERR_INVALID_ARG, "int8 keys need a 16-byte aligned k_scale");
   if (!p->z_pool || !p->k_pool || !p->w_zk || !p->b_v || (p->rank_s > 0 && (!p->r_pool || !p->b_r)))
     return fail(BASISKV_ERR_INVALID_ARG, "pool or basis pointer is NULL");
   const void* ptrs[] = {p->z_pool, p->k_pool, p->w_zk, p->b_v};
@@ -234,11 +243,12 @@ void choose_kernels(basiskv_handle* h) {
       h->route_smem = kRouteWarps * st * stage;
     }
   }
+  const bool k8 = p.k_format == BASISKV_KEYS_INT8;
   for (int tps : {64, 32, 16}) {
     if (p.page_size % tps) continue;
-    auto ait = attn_table().find(AttnKey{p.gqa_group, p.head_dim, p.rank_r, tps});
+    auto ait = attn_table().find(AttnKey{p.gqa_group, p.head_dim, p.rank_r, tps, k8});
     if (ait == attn_table().end()) continue;
-    const size_t stage = (size_t)tps * (p.head_dim + p.rank_r) * es;
+    const size_t stage = (size_t)tps * (p.head_dim * (k8 ? 1 : es) + p.rank_r * es + (k8 ? 4 : 0));
     int st = (int)std::min<size_t>(4, kAttnSmemBudget / (kAttnWarps * stage));
     if (st < 1) continue;
     if (st < 2 && tps > 16) continue;  // prefer a smaller stage with double buffering
@@ -487,6 +497,8 @@ int launch_attn(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk
   AttnArgs a;
   a.q = q;
   a.k_pool = p.k_pool;
+  a.k_scale = p.k_scale;
+  a.k_int8 = p.k_format == BASISKV_KEYS_INT8;
   a.z_pool = p.z_pool;
   a.b_v = p.b_v;
   a.page_table = h->d_page_table;
@@ -832,6 +844,8 @@ int basiskv_encode_rows(basiskv_handle* h, int slot, int row0, int n_rows, const
   a.k = k;
   a.v = v;
   a.k_pool = const_cast<void*>(p.k_pool);
+  a.k_scale = const_cast<float*>(p.k_scale);
+  a.k_int8 = p.k_format == BASISKV_KEYS_INT8;
   a.z_pool = const_cast<void*>(p.z_pool);
   a.r_pool = const_cast<void*>(p.r_pool);
   a.a_v = h->d_enc;
@@ -850,6 +864,37 @@ int basiskv_encode_rows(basiskv_handle* h, int slot, int row0, int n_rows, const
   cudaStream_t st = (cudaStream_t)stream;
   if (p.dtype == BASISKV_DTYPE_BF16) encode_rows_kernel<__nv_bfloat16><<<grid, kEncodeThreads, smem, st>>>(a);
   else encode_rows_kernel<float><<<grid, kEncodeThreads, smem, st>>>(a);
+  CUDA_TRY(cudaGetLastError());
+  return BASISKV_OK;
+}
+
+int basiskv_quantize_keys(basiskv_handle* h, const void* k, int64_t row0, int64_t n_rows,
+                          basiskv_stream_t stream) {
+  int rc = check_handle(h);
+  if (rc) return rc;
+  const basiskv_params& p = h->p;
+  if (p.k_format != BASISKV_KEYS_INT8) return fail(BASISKV_ERR_INVALID_ARG, "the handle's keys are not int8");
+  const long long rows = (long long)p.num_slots * p.num_kv_heads * p.page_size;
+  if (!k) return fail(BASISKV_ERR_INVALID_ARG, "k is NULL");
+  if (n_rows < 0 || row0 < 0 || row0 + n_rows > rows)
+    return fail(BASISKV_ERR_INVALID_ARG, "rows [%lld, %lld) outside the pool's %lld", (long long)row0,
+                (long long)(row0 + n_rows), rows);
+  if (n_rows == 0) return BASISKV_OK;
+  QuantizeArgs a;
+  a.k = k;
+  a.codes = static_cast<int8_t*>(const_cast<void*>(p.k_pool));
+  a.scales = const_cast<float*>(p.k_scale);
+  a.row0 = row0;
+  a.n = n_rows;
+  a.head_dim = p.head_dim;
+  constexpr int rows_per_cta = kEncodeThreads / 32;
+  const long long ctas = (n_rows + rows_per_cta - 1) / rows_per_cta;
+  if (ctas > 0x7fffffffLL) return fail(BASISKV_ERR_INVALID_ARG, "too many rows for one call");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (p.dtype == BASISKV_DTYPE_BF16)
+    quantize_rows_kernel<__nv_bfloat16><<<(unsigned)ctas, kEncodeThreads, 0, st>>>(a);
+  else
+    quantize_rows_kernel<float><<<(unsigned)ctas, kEncodeThreads, 0, st>>>(a);
   CUDA_TRY(cudaGetLastError());
   return BASISKV_OK;
 }
@@ -1077,6 +1122,8 @@ extern "C" int basiskv_decode_attn_noalloc(const basiskv_params* p, int batch, c
   AttnArgs aa{};
   aa.q = q;
   aa.k_pool = p->k_pool;
+  aa.k_scale = p->k_scale;
+  aa.k_int8 = p->k_format == BASISKV_KEYS_INT8;
   aa.z_pool = p->z_pool;
   aa.b_v = p->b_v;
   aa.page_table = page_table;

@@ -6,7 +6,11 @@
 //     R = (K - Z_stored . W_zk) . A_r  A_r = pinv(B_r)  [d][s]
 // The residual is taken against the stored (rounded) latent, so that
 // Z.W_zk + R.B_r predicts K from exactly what routing will read.  K rows
-// are stored as given.
+// are stored as given, or as int8 codes with a per-token scale (the lossy
+// key compression of "PackKV: Reducing KV Cache Memory Footprint through
+// LLM-Aware Lossy Compression", abstract, read as symmetric int8):
+//     scale = max_c |k_c| / 127,   code_c = rint(k_c / scale)
+// in float32 with IEEE division, ties to even; a zero row gets scale 0.
 #pragma once
 
 #include "common.cuh"
@@ -16,7 +20,9 @@ namespace basiskv {
 struct EncodeArgs {
   const void* k;      // [Hkv][n][d] pool dtype
   const void* v;      // [Hkv][n][d] pool dtype
-  void* k_pool;       // [slots][Hkv][P][d]
+  void* k_pool;       // [slots][Hkv][P][d]: pool dtype, or int8 codes when k_int8
+  float* k_scale;     // [slots][Hkv][P] (k_int8 only)
+  int k_int8;
   void* z_pool;       // [slots][Hkv][P][r]
   void* r_pool;       // [slots][Hkv][P][s]
   const float* a_v;   // [Hkv][d][r]
@@ -27,6 +33,41 @@ struct EncodeArgs {
 };
 
 constexpr int kEncodeThreads = 128;
+
+// One key row of d values to int8 codes and its scale, by one warp.
+template <typename T>
+__device__ __forceinline__ void warp_quantize_row(const T* k, int d, int8_t* codes, float* scale, int lane) {
+  float amax = 0.f;
+  for (int c = lane; c < d; c += 32) amax = fmaxf(amax, fabsf(to_f32(k[c])));
+  amax = warp_max(amax);
+  const float sc = __fdiv_rn(amax, 127.f);
+  for (int c = lane; c < d; c += 32) {
+    int q = 0;
+    if (sc > 0.f) q = __float2int_rn(__fdiv_rn(to_f32(k[c]), sc));
+    codes[c] = (int8_t)max(-127, min(127, q));
+  }
+  if (lane == 0) *scale = sc;
+}
+
+// Rows [row0, row0 + n) of a key pool in its flat row order
+// ((slot * Hkv + kvh) * P + token), from keys k [n][d] in the pool dtype.
+struct QuantizeArgs {
+  const void* k;
+  int8_t* codes;   // the int8 key pool
+  float* scales;   // [rows]
+  long long row0, n;
+  int head_dim;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kEncodeThreads) quantize_rows_kernel(const QuantizeArgs a) {
+  const int lane = threadIdx.x & 31;
+  const long long i = (long long)blockIdx.x * (kEncodeThreads / 32) + (threadIdx.x >> 5);
+  if (i >= a.n) return;
+  const long long row = a.row0 + i;
+  warp_quantize_row(static_cast<const T*>(a.k) + i * a.head_dim, a.head_dim, a.codes + row * a.head_dim,
+                    a.scales + row, lane);
+}
 
 template <typename T>
 __device__ __forceinline__ T from_f32(float x);
@@ -54,12 +95,13 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_rows_kernel(const Encod
   const size_t row = ((size_t)a.slot * a.num_kv_heads + kvh) * a.page_size + a.row0 + i;
   const T* k = static_cast<const T*>(a.k) + in;
   const T* v = static_cast<const T*>(a.v) + in;
-  T* kp = static_cast<T*>(a.k_pool) + row * d;
   for (int c = tid; c < d; c += kEncodeThreads) {
     kr[c] = to_f32(k[c]);
     vr[c] = to_f32(v[c]);
-    kp[c] = k[c];
+    if (!a.k_int8) static_cast<T*>(a.k_pool)[row * d + c] = k[c];
   }
+  if (a.k_int8 && tid < 32)
+    warp_quantize_row(k, d, static_cast<int8_t*>(a.k_pool) + row * d, a.k_scale + row, tid);
   __syncthreads();
   const float* Av = a.a_v + (size_t)kvh * d * r;
   T* zp = static_cast<T*>(a.z_pool) + row * r;

@@ -128,18 +128,20 @@ class Workload:
     def num_pages(self) -> np.ndarray:
         return -(-self.seq_lens.astype(np.int64) // self.spec.page_size)
 
-    def algorithmic_bytes(self) -> dict:
+    def algorithmic_bytes(self, int8_keys: bool = False) -> dict:
         """Bytes the routed path must move per call: the routing read of every
         valid token's Z and R rows (units with k < n_b), and the selected pages'
-        K and Z (whole pages).  Dense units (k >= n_b) read K and Z of every page."""
+        K and Z (whole pages).  Dense units (k >= n_b) read K and Z of every page.
+        With int8 keys a key row is d one-byte codes plus a 4-byte scale."""
         s = self.spec
         es = 2 if s.dtype == "bf16" else 4
+        kbytes = s.head_dim + 4 if int8_keys else s.head_dim * es
         route = attn = 0
         for L, n in zip(self.seq_lens.tolist(), self.num_pages.tolist()):
             kb = min(s.topk, n)
             if kb < n:
                 route += s.num_kv_heads * L * (s.rank_r + s.rank_s) * es
-            attn += s.num_kv_heads * kb * s.page_size * (s.head_dim + s.rank_r) * es
+            attn += s.num_kv_heads * kb * s.page_size * (kbytes + s.rank_r * es)
         return {"route": route, "attn": attn, "total": route + attn}
 
 

@@ -19,7 +19,11 @@
  * Layouts (row-major, element type = the pool dtype unless stated):
  *   z_pool [num_slots][Hkv][P][r]     value latents Z
  *   r_pool [num_slots][Hkv][P][s]     key residuals R (NULL when s = 0)
- *   k_pool [num_slots][Hkv][P][d]     original keys K
+ *   k_pool [num_slots][Hkv][P][d]     original keys K, in the pool dtype or,
+ *                                     with k_format = BASISKV_KEYS_INT8, as
+ *                                     int8 codes with
+ *   k_scale [num_slots][Hkv][P] fp32  one scale per token: K_t = k_scale_t *
+ *                                     code_t (see basiskv_quantize_keys)
  *   w_zk   [Hkv][r][d]  fp32          latent-to-key basis
  *   b_r    [Hkv][s][d]  fp32          residual-to-key basis (NULL when s = 0)
  *   b_v    [Hkv][r][d]  fp32          latent-to-value basis
@@ -78,12 +82,23 @@ enum {
 
 enum { BASISKV_DTYPE_BF16 = 0, BASISKV_DTYPE_F32 = 1 };
 
+/* How the original keys are stored.  NATIVE: in the pool dtype.  INT8: int8
+ * codes with an fp32 scale per token, the lossy key compression of "PackKV:
+ * Reducing KV Cache Memory Footprint through LLM-Aware Lossy Compression"
+ * (abstract) read as symmetric per-token int8; the attention kernels read
+ * the codes and apply the scale to each token's dot product, so no
+ * dequantised copy exists.  Halves the key bytes the exact-attention step
+ * reads.  On the tensor-core path the query meets the codes in f16 (the
+ * query is rounded to f16: exact for |q| in [2^-14, 65504]). */
+enum { BASISKV_KEYS_NATIVE = 0, BASISKV_KEYS_INT8 = 1 };
+
 /* Creation parameters.  Shapes: Hkv = num_kv_heads, G = gqa_group (1..8),
  * d = head_dim, P = page_size, r = rank_r (1..d), s = rank_s (0 allowed).
  * The fast bf16 path needs d % 32 == 0, P % 16 == 0, r % 8 == 0,
  * s % 8 == 0 and (G, d, r, s) among the compiled shapes; every other shape
- * runs the generic CUDA-core kernels (also the fp32 path).  All pools and
- * bases must be 16-byte aligned; pool row strides follow from the shapes. */
+ * runs the generic CUDA-core kernels (also the fp32 path); int8 keys on the
+ * fast path also need d % 64 == 0.  All pools, bases and k_scale must be
+ * 16-byte aligned; pool row strides follow from the shapes. */
 typedef struct basiskv_params {
     int32_t max_batch;          /* sequences addressable by the page table   */
     int32_t num_kv_heads;
@@ -96,13 +111,16 @@ typedef struct basiskv_params {
     int32_t max_topk;           /* largest topk a decode call may ask for    */
     int32_t num_slots;          /* pages the pools hold                      */
     int32_t dtype;              /* BASISKV_DTYPE_*                           */
-    int32_t reserved;           /* must be 0                                 */
-    const void *z_pool;         /* caller-owned; written only by encode_rows */
+    int32_t k_format;           /* BASISKV_KEYS_* (0: keys in the pool dtype) */
+    const void *z_pool;         /* caller-owned; written only by encode_rows
+                                   (k_pool also by quantize_keys)            */
     const void *r_pool;
     const void *k_pool;
     const float *w_zk;
     const float *b_r;
     const float *b_v;
+    const float *k_scale;       /* [num_slots][Hkv][P] with BASISKV_KEYS_INT8,
+                                   else NULL; caller-owned                   */
 } basiskv_params;
 
 typedef struct basiskv_handle basiskv_handle;
@@ -187,10 +205,12 @@ BASISKV_API int basiskv_decode_attn_host(basiskv_handle *h, int batch, const voi
  * ("BasisKV: Value Latents for Communication and Key Routing", English
  * abstract: values kept as rank-r latents, and a Key-specific residual
  * storing what the Value latent cannot predict; least-squares reading):
- *   K rows stored as given;
+ *   K rows stored as given (int8 keys: quantised as basiskv_quantize_keys
+ *   does, codes and scale);
  *   Z = V . pinv(B_v), rounded to the pool dtype;
  *   R = (K - Z . W_zk) . pinv(B_r), from the rounded Z, rounded.
- * The only call that writes the caller's pools.  The first call computes
+ * With basiskv_quantize_keys, the only calls that write the caller's pools
+ * (and k_scale).  The first call computes
  * the pseudo-inverses of the bases on the host (synchronous); later calls
  * only enqueue on `stream`.  The page table is not touched: follow with
  * basiskv_append_page or basiskv_append_tokens.  Errors: INVALID_ARG (slot
@@ -198,6 +218,20 @@ BASISKV_API int basiskv_decode_attn_host(basiskv_handle *h, int batch, const voi
  * CUDA. */
 BASISKV_API int basiskv_encode_rows(basiskv_handle *h, int slot, int row0, int n_rows, const void *k,
                         const void *v, basiskv_stream_t stream);
+
+/* Store keys into an int8 key pool (k_format = BASISKV_KEYS_INT8): rows
+ * [row0, row0 + n_rows) of the pool in its flat row order, row =
+ * (slot * Hkv + kvh) * P + token, from k [n_rows][d] (pool dtype, device).
+ * Per row, in float32 with IEEE division ("PackKV: Reducing KV Cache Memory
+ * Footprint through LLM-Aware Lossy Compression", abstract; symmetric
+ * per-token int8 reading):
+ *   k_scale[row] = max_c |k_c| / 127,  code_c = rint(k_c / k_scale[row])
+ * (ties to even); a row of zeros gets scale 0 and codes 0.  Quantising a
+ * whole native pool into an int8 one is one call with row0 = 0 and n_rows =
+ * num_slots * Hkv * P.  Enqueued on `stream`.  Errors: INVALID_ARG (the
+ * handle's keys are not int8, NULL k, rows outside the pool), CUDA. */
+BASISKV_API int basiskv_quantize_keys(basiskv_handle *h, const void *k, int64_t row0, int64_t n_rows,
+                          basiskv_stream_t stream);
 
 /* Routing alone (steps route-prep, route-score, top-k) for every sequence
  * with at least one page, whether or not topk >= n_b.  scores_out

@@ -38,7 +38,7 @@ def test_version(lib):
 def _params(**kw):
     p = bk.basiskv_params()
     base = dict(max_batch=2, num_kv_heads=2, gqa_group=4, head_dim=128, page_size=64, rank_r=32,
-                rank_s=16, max_pages_per_seq=8, max_topk=4, num_slots=16, dtype=0, reserved=0,
+                rank_s=16, max_pages_per_seq=8, max_topk=4, num_slots=16, dtype=0, k_format=0,
                 z_pool=0x1000, r_pool=0x2000, k_pool=0x3000, w_zk=0x4000, b_r=0x5000, b_v=0x6000)
     base.update(kw)
     for k, v in base.items():
@@ -50,7 +50,7 @@ def _params(**kw):
     dict(max_batch=0), dict(num_kv_heads=0), dict(gqa_group=0), dict(gqa_group=9),
     dict(head_dim=0), dict(page_size=0), dict(rank_r=0), dict(rank_r=129), dict(rank_s=-1),
     dict(max_pages_per_seq=0), dict(max_topk=0), dict(num_slots=0), dict(dtype=7),
-    dict(reserved=1), dict(z_pool=None), dict(k_pool=None), dict(r_pool=None),
+    dict(k_format=2), dict(k_format=1), dict(k_format=1, k_scale=0x7008), dict(z_pool=None), dict(k_pool=None), dict(r_pool=None),
     dict(b_v=None), dict(w_zk=0x1001), dict(k_pool=0x3008),
 ])
 def test_create_rejects_bad_params(lib, bad):
