@@ -297,6 +297,49 @@ def run_reference(args, rank, world):
     return 0
 
 
+def aux_measurements(kv, w, stream, dev, int8_codes=None):
+    """Device time of the write-side entry points, after the timed region:
+    basiskv_encode_rows for one page of P tokens of every KV head (a prefill
+    chunk) and for one token (a decode-time append), into the last pool slot;
+    with int8 keys, basiskv_quantize_keys over the whole key pool.  CUDA
+    events around 20 calls each, after one untimed call (the first encode
+    call computes the bases' pseudo-inverses on the host)."""
+    import torch
+    from compressed_kv_cache_routing_b200 import basiskv as bk
+    s = w.spec
+    g = torch.Generator(device=dev).manual_seed(99)
+    dt = w.k_pool.dtype
+    slot = int(w.k_pool.shape[0]) - 1
+
+    def timed(fn, n=20):
+        fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / n * 1e3  # us per call
+
+    out = {}
+    for name, rows in (("encode_rows_page", s.page_size), ("encode_rows_token", 1)):
+        k = torch.randn((s.num_kv_heads, rows, s.head_dim), generator=g, device=dev).to(dt)
+        v = torch.randn((s.num_kv_heads, rows, s.head_dim), generator=g, device=dev).to(dt)
+        us = timed(lambda: bk.basiskv_encode_rows(kv.handle, slot, 0, k, v, stream=stream))
+        out[name] = {"us_per_call": us, "rows_per_call": rows * s.num_kv_heads,
+                     "rows_per_s": rows * s.num_kv_heads / (us * 1e-6)}
+    if int8_codes is not None:
+        nbytes = w.k_pool.numel() * w.k_pool.element_size() + int8_codes.numel() + 4 * int8_codes.numel() // s.head_dim
+        us = timed(lambda: bk.basiskv_quantize_keys(kv.handle, w.k_pool, stream=stream), n=5)
+        out["quantize_keys_pool"] = {"us_per_call": us, "rows": int8_codes.numel() // s.head_dim,
+                                     "gb_per_s": nbytes / (us * 1e-6) / 1e9,
+                                     "bytes": int(nbytes)}
+    if bk.basiskv_get_status(kv.handle, clear=True):
+        raise SystemExit("device status error in the write-side measurements")
+    return out
+
+
 def run_ours(args, rank, world, local):
     import torch
     from compressed_kv_cache_routing_b200 import basiskv as bk
@@ -315,6 +358,7 @@ def run_ours(args, rank, world, local):
     spec = replica_spec(spec, rank)
     w = W.generate(spec, device=dev)
     int8 = args.keys == "int8"
+    codes = None
     if int8:
         # the keys as int8 codes and per-token scales, quantised on the device
         codes = torch.empty(tuple(w.k_pool.shape), dtype=torch.int8, device=dev)
@@ -413,6 +457,7 @@ def run_ours(args, rank, world, local):
     e2e_s = max_over_ranks(float(np.mean(e2e_times)), world, dev)
     h2d = q_host.numel() * q_host.element_size()
     d2h = out_host.numel() * 4 + sel_host.numel() * 4
+    aux = aux_measurements(kv, w, stream, dev, codes if int8 else None)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -448,6 +493,7 @@ def run_ours(args, rank, world, local):
             "clocks": clocks,
             "device_status": status,
             "cpu_baseline": cpu,
+            "aux": aux,
         }
         print(json.dumps(line), flush=True)
     kv.close()

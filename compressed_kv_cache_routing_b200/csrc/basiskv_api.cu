@@ -875,7 +875,7 @@ int basiskv_quantize_keys(basiskv_handle* h, const void* k, int64_t row0, int64_
   const basiskv_params& p = h->p;
   if (p.k_format != BASISKV_KEYS_INT8) return fail(BASISKV_ERR_INVALID_ARG, "the handle's keys are not int8");
   const long long rows = (long long)p.num_slots * p.num_kv_heads * p.page_size;
-  if (!k) return fail(BASISKV_ERR_INVALID_ARG, "k is NULL");
+  if (!k || !aligned16(k)) return fail(BASISKV_ERR_INVALID_ARG, "k must be a 16-byte aligned device pointer");
   if (n_rows < 0 || row0 < 0 || row0 + n_rows > rows)
     return fail(BASISKV_ERR_INVALID_ARG, "rows [%lld, %lld) outside the pool's %lld", (long long)row0,
                 (long long)(row0 + n_rows), rows);
@@ -887,7 +887,7 @@ int basiskv_quantize_keys(basiskv_handle* h, const void* k, int64_t row0, int64_
   a.row0 = row0;
   a.n = n_rows;
   a.head_dim = p.head_dim;
-  constexpr int rows_per_cta = kEncodeThreads / 32;
+  constexpr int rows_per_cta = kEncodeThreads / 32 * kQuantRowsPerWarp;
   const long long ctas = (n_rows + rows_per_cta - 1) / rows_per_cta;
   if (ctas > 0x7fffffffLL) return fail(BASISKV_ERR_INVALID_ARG, "too many rows for one call");
   cudaStream_t st = (cudaStream_t)stream;

@@ -59,14 +59,49 @@ struct QuantizeArgs {
   int head_dim;
 };
 
+// Rows per warp of quantize_rows_kernel: their loads are issued together so
+// that each warp keeps several rows in flight.
+constexpr int kQuantRowsPerWarp = 4;
+
+// code of x for scale sc (as warp_quantize_row)
+__device__ __forceinline__ uint32_t quant_code(float x, float sc) {
+  const int q = sc > 0.f ? __float2int_rn(__fdiv_rn(x, sc)) : 0;
+  return (uint32_t)(uint8_t)(int8_t)max(-127, min(127, q));
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kEncodeThreads) quantize_rows_kernel(const QuantizeArgs a) {
   const int lane = threadIdx.x & 31;
-  const long long i = (long long)blockIdx.x * (kEncodeThreads / 32) + (threadIdx.x >> 5);
-  if (i >= a.n) return;
-  const long long row = a.row0 + i;
-  warp_quantize_row(static_cast<const T*>(a.k) + i * a.head_dim, a.head_dim, a.codes + row * a.head_dim,
-                    a.scales + row, lane);
+  const long long i0 = ((long long)blockIdx.x * (kEncodeThreads / 32) + (threadIdx.x >> 5)) * kQuantRowsPerWarp;
+  if (i0 >= a.n) return;
+  if constexpr (sizeof(T) == 2) {
+    if (a.head_dim == 128) {
+      // bf16 rows of 128: four values per lane, one 8-byte load per row
+      uint2 v[kQuantRowsPerWarp];
+#pragma unroll
+      for (int r = 0; r < kQuantRowsPerWarp; ++r)
+        v[r] = i0 + r < a.n ? __ldg(reinterpret_cast<const uint2*>(static_cast<const T*>(a.k) + (i0 + r) * 128) + lane)
+                            : make_uint2(0u, 0u);
+#pragma unroll
+      for (int r = 0; r < kQuantRowsPerWarp; ++r) {
+        if (i0 + r >= a.n) break;
+        const float x0 = __uint_as_float(v[r].x << 16), x1 = __uint_as_float(v[r].x & 0xffff0000u);
+        const float x2 = __uint_as_float(v[r].y << 16), x3 = __uint_as_float(v[r].y & 0xffff0000u);
+        const float amax = warp_max(fmaxf(fmaxf(fabsf(x0), fabsf(x1)), fmaxf(fabsf(x2), fabsf(x3))));
+        const float sc = __fdiv_rn(amax, 127.f);
+        const long long row = a.row0 + i0 + r;
+        reinterpret_cast<uint32_t*>(a.codes + row * 128)[lane] =
+            quant_code(x0, sc) | quant_code(x1, sc) << 8 | quant_code(x2, sc) << 16 | quant_code(x3, sc) << 24;
+        if (lane == 0) a.scales[row] = sc;
+      }
+      return;
+    }
+  }
+  for (int r = 0; r < kQuantRowsPerWarp && i0 + r < a.n; ++r) {
+    const long long i = i0 + r, row = a.row0 + i;
+    warp_quantize_row(static_cast<const T*>(a.k) + i * a.head_dim, a.head_dim, a.codes + row * a.head_dim,
+                      a.scales + row, lane);
+  }
 }
 
 template <typename T>

@@ -221,7 +221,8 @@ BASISKV_API int basiskv_encode_rows(basiskv_handle *h, int slot, int row0, int n
 
 /* Store keys into an int8 key pool (k_format = BASISKV_KEYS_INT8): rows
  * [row0, row0 + n_rows) of the pool in its flat row order, row =
- * (slot * Hkv + kvh) * P + token, from k [n_rows][d] (pool dtype, device).
+ * (slot * Hkv + kvh) * P + token, from k [n_rows][d] (pool dtype, device,
+ * 16-byte aligned).
  * Per row, in float32 with IEEE division ("PackKV: Reducing KV Cache Memory
  * Footprint through LLM-Aware Lossy Compression", abstract; symmetric
  * per-token int8 reading):
@@ -229,7 +230,8 @@ BASISKV_API int basiskv_encode_rows(basiskv_handle *h, int slot, int row0, int n
  * (ties to even); a row of zeros gets scale 0 and codes 0.  Quantising a
  * whole native pool into an int8 one is one call with row0 = 0 and n_rows =
  * num_slots * Hkv * P.  Enqueued on `stream`.  Errors: INVALID_ARG (the
- * handle's keys are not int8, NULL k, rows outside the pool), CUDA. */
+ * handle's keys are not int8, NULL or misaligned k, rows outside the
+ * pool), CUDA. */
 BASISKV_API int basiskv_quantize_keys(basiskv_handle *h, const void *k, int64_t row0, int64_t n_rows,
                           basiskv_stream_t stream);
 
