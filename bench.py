@@ -300,7 +300,9 @@ def run_reference(args, rank, world):
 def aux_measurements(kv, w, stream, dev, int8_codes=None):
     """Device time of the write-side entry points, after the timed region:
     basiskv_encode_rows for one page of P tokens of every KV head (a prefill
-    chunk) and for one token (a decode-time append), into the last pool slot;
+    chunk) and for one token, into the last pool slot; basiskv_encode_tokens
+    for one token of every sequence (the decode-time append) into the last
+    slots;
     with int8 keys, basiskv_quantize_keys over the whole key pool.  CUDA
     events around 20 calls each, after one untimed call (the first encode
     call computes the bases' pseudo-inverses on the host)."""
@@ -329,6 +331,15 @@ def aux_measurements(kv, w, stream, dev, int8_codes=None):
         us = timed(lambda: bk.basiskv_encode_rows(kv.handle, slot, 0, k, v, stream=stream))
         out[name] = {"us_per_call": us, "rows_per_call": rows * s.num_kv_heads,
                      "rows_per_s": rows * s.num_kv_heads / (us * 1e-6)}
+    # the decode-time append: one new token per sequence, one launch
+    nb = s.batch
+    slots = torch.arange(slot, slot - nb, -1, device=dev, dtype=torch.int32).clamp_(min=0)
+    rows = torch.zeros(nb, device=dev, dtype=torch.int32)
+    k = torch.randn((nb, s.num_kv_heads, s.head_dim), generator=g, device=dev).to(dt)
+    v = torch.randn((nb, s.num_kv_heads, s.head_dim), generator=g, device=dev).to(dt)
+    us = timed(lambda: bk.basiskv_encode_tokens(kv.handle, slots, rows, k, v, stream=stream))
+    out["encode_tokens_batch"] = {"us_per_call": us, "rows_per_call": nb * s.num_kv_heads,
+                                  "rows_per_s": nb * s.num_kv_heads / (us * 1e-6)}
     if int8_codes is not None:
         nbytes = w.k_pool.numel() * w.k_pool.element_size() + int8_codes.numel() + 4 * int8_codes.numel() // s.head_dim
         us = timed(lambda: bk.basiskv_quantize_keys(kv.handle, w.k_pool, stream=stream), n=5)

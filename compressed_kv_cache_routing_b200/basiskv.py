@@ -40,7 +40,7 @@ EXPORTED = (
     "basiskv_decode_attn_host", "basiskv_route", "basiskv_get_status", "basiskv_profile_begin",
     "basiskv_profile_end", "basiskv_last_launch", "basiskv_last_error", "basiskv_version",
     "basiskv_decode_attn_noalloc", "basiskv_decode_attn_latent", "basiskv_encode_rows",
-    "basiskv_quantize_keys",
+    "basiskv_quantize_keys", "basiskv_encode_tokens",
 )
 
 
@@ -90,6 +90,7 @@ def load(path: str = LIB_PATH):
         "basiskv_decode_attn_latent": [H, i32, vp, i32, f32, vp, vp, vp],
         "basiskv_encode_rows": [H, i32, i32, i32, vp, vp, vp],
         "basiskv_quantize_keys": [H, vp, ctypes.c_int64, ctypes.c_int64, vp],
+        "basiskv_encode_tokens": [H, i32, vp, vp, vp, vp, vp],
         "basiskv_route": [H, i32, vp, i32, vp, vp, vp],
         "basiskv_get_status": [H, ctypes.POINTER(ctypes.c_uint32), i32],
         "basiskv_profile_begin": [H, i32],
@@ -175,6 +176,13 @@ def basiskv_encode_rows(h, slot, row0, k, v, stream=None):
     """Encode k, v [Hkv][n][d] (pool dtype, device) into rows [row0, row0+n)
     of pool slot ``slot``: K as given, Z and R by least squares."""
     _check(load().basiskv_encode_rows(h, slot, row0, int(k.shape[1]), _ptr(k), _ptr(v), _stream(stream)))
+
+
+def basiskv_encode_tokens(h, slots, rows, k, v, stream=None):
+    """Encode k, v [n][Hkv][d] (pool dtype, device) into row rows[i] of pool
+    slot slots[i] (device int32 tensors [n]) for every token i, one launch."""
+    _check(load().basiskv_encode_tokens(h, int(k.shape[0]), _ptr(slots), _ptr(rows), _ptr(k), _ptr(v),
+                                        _stream(stream)))
 
 
 def basiskv_quantize_keys(h, k, row0=0, stream=None):

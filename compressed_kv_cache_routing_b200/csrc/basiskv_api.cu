@@ -260,6 +260,16 @@ void choose_kernels(basiskv_handle* h) {
   }
 }
 
+// Dynamic shared memory of encode_kernel: the row buffers, plus the KV
+// head's A_v, W_zk and A_r when they fit (*stage).
+constexpr size_t kEncodeStageMax = 200 * 1024;
+size_t encode_smem(const basiskv_params& p, bool* stage) {
+  const size_t d = p.head_dim, r = p.rank_r, s = p.rank_s;
+  const size_t rows = sizeof(float) * (3 * d + r), bases = sizeof(float) * (2 * d * r + d * s);
+  *stage = rows + bases <= kEncodeStageMax;
+  return rows + (*stage ? bases : 0);
+}
+
 size_t generic_route_smem(const basiskv_params& p) {
   return sizeof(float) * (size_t)p.gqa_group * (p.head_dim + p.rank_r + p.rank_s);
 }
@@ -273,8 +283,13 @@ size_t generic_attn_smem(const basiskv_params& p) {
 // then keep one L1/shared split for all of this library's grids, so a grid
 // launched early (programmatic dependent launch) can share SMs with the one
 // still finishing.
+// The limit belongs to the function, not to a handle, so it is only ever
+// raised: a handle with smaller shapes must not lower it under another's.
 int set_smem_attr(const void* fn, size_t bytes) {
-  CUDA_TRY(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
+  cudaFuncAttributes fa;
+  CUDA_TRY(cudaFuncGetAttributes(&fa, fn));
+  if ((size_t)fa.maxDynamicSharedSizeBytes < bytes)
+    CUDA_TRY(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
   CUDA_TRY(cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared));
   return BASISKV_OK;
 }
@@ -646,6 +661,12 @@ int basiskv_create(const basiskv_params* p, basiskv_handle** out) {
   h->attn_occ = std::max(1, h->attn_occ);
   if (!arc)
     arc = p->dtype == BASISKV_DTYPE_BF16 ? set_generic_attrs<__nv_bfloat16>(*p) : set_generic_attrs<float>(*p);
+  if (!arc) {
+    bool stage = false;
+    const size_t esmem = encode_smem(*p, &stage);
+    arc = p->dtype == BASISKV_DTYPE_BF16 ? set_smem_attr((const void*)&encode_kernel<__nv_bfloat16>, esmem)
+                                        : set_smem_attr((const void*)&encode_kernel<float>, esmem);
+  }
   if (arc) {
     std::string msg = g_last_error;
     basiskv_destroy(h);
@@ -815,34 +836,39 @@ int basiskv_decode_attn_latent(basiskv_handle* h, int batch, const void* q, int 
   return decode_step(h, batch, q, topk, softmax_scale, zbar_out, sel_out, stream, 1);
 }
 
-int basiskv_encode_rows(basiskv_handle* h, int slot, int row0, int n_rows, const void* k, const void* v,
-                        basiskv_stream_t stream) {
-  int rc = check_handle(h);
+}  // extern "C"
+
+namespace {
+
+// The pseudo-inverses of the bases, once per handle, on the host (a set-up
+// step, synchronous).
+int ensure_encode_bases(basiskv_handle* h) {
+  if (h->enc_ready) return BASISKV_OK;
+  const basiskv_params& p = h->p;
+  const int Hkv = p.num_kv_heads, d = p.head_dim, r = p.rank_r, s = p.rank_s;
+  std::vector<float> bv((size_t)Hkv * r * d), br((size_t)Hkv * s * d), enc((size_t)Hkv * d * (r + s));
+  CUDA_TRY(cudaMemcpy(bv.data(), p.b_v, sizeof(float) * bv.size(), cudaMemcpyDeviceToHost));
+  if (s > 0) CUDA_TRY(cudaMemcpy(br.data(), p.b_r, sizeof(float) * br.size(), cudaMemcpyDeviceToHost));
+  for (int kvh = 0; kvh < Hkv; ++kvh) {
+    if (!right_pinv(bv.data() + (size_t)kvh * r * d, r, d, enc.data() + (size_t)kvh * d * r))
+      return fail(BASISKV_ERR_INVALID_ARG, "the rows of B_v of KV head %d are linearly dependent", kvh);
+    if (s > 0 && !right_pinv(br.data() + (size_t)kvh * s * d, s, d,
+                             enc.data() + (size_t)Hkv * d * r + (size_t)kvh * d * s))
+      return fail(BASISKV_ERR_INVALID_ARG, "the rows of B_r of KV head %d are linearly dependent", kvh);
+  }
+  CUDA_TRY(cudaMemcpy(h->d_enc, enc.data(), sizeof(float) * enc.size(), cudaMemcpyHostToDevice));
+  h->enc_ready = true;
+  return BASISKV_OK;
+}
+
+
+// Fill the pool fields of `a`, size the grid (a few tokens per CTA once
+// there are more token-heads than two waves of CTAs) and launch.
+int launch_encode(basiskv_handle* h, EncodeArgs& a, cudaStream_t st) {
+  int rc = ensure_encode_bases(h);
   if (rc) return rc;
   const basiskv_params& p = h->p;
-  if (slot < 0 || slot >= p.num_slots) return fail(BASISKV_ERR_INVALID_ARG, "slot %d outside [0, %d)", slot, p.num_slots);
-  if (n_rows < 1 || row0 < 0 || row0 + n_rows > p.page_size)
-    return fail(BASISKV_ERR_INVALID_ARG, "rows [%d, %d) outside a page of %d", row0, row0 + n_rows, p.page_size);
-  if (!k || !v) return fail(BASISKV_ERR_INVALID_ARG, "k or v is NULL");
   const int Hkv = p.num_kv_heads, d = p.head_dim, r = p.rank_r, s = p.rank_s;
-  if (!h->enc_ready) {
-    // the pseudo-inverses of the bases, once, on the host (a set-up step)
-    std::vector<float> bv((size_t)Hkv * r * d), br((size_t)Hkv * s * d), enc((size_t)Hkv * d * (r + s));
-    CUDA_TRY(cudaMemcpy(bv.data(), p.b_v, sizeof(float) * bv.size(), cudaMemcpyDeviceToHost));
-    if (s > 0) CUDA_TRY(cudaMemcpy(br.data(), p.b_r, sizeof(float) * br.size(), cudaMemcpyDeviceToHost));
-    for (int kvh = 0; kvh < Hkv; ++kvh) {
-      if (!right_pinv(bv.data() + (size_t)kvh * r * d, r, d, enc.data() + (size_t)kvh * d * r))
-        return fail(BASISKV_ERR_INVALID_ARG, "the rows of B_v of KV head %d are linearly dependent", kvh);
-      if (s > 0 && !right_pinv(br.data() + (size_t)kvh * s * d, s, d,
-                               enc.data() + (size_t)Hkv * d * r + (size_t)kvh * d * s))
-        return fail(BASISKV_ERR_INVALID_ARG, "the rows of B_r of KV head %d are linearly dependent", kvh);
-    }
-    CUDA_TRY(cudaMemcpy(h->d_enc, enc.data(), sizeof(float) * enc.size(), cudaMemcpyHostToDevice));
-    h->enc_ready = true;
-  }
-  EncodeArgs a;
-  a.k = k;
-  a.v = v;
   a.k_pool = const_cast<void*>(p.k_pool);
   a.k_scale = const_cast<float*>(p.k_scale);
   a.k_int8 = p.k_format == BASISKV_KEYS_INT8;
@@ -856,16 +882,61 @@ int basiskv_encode_rows(basiskv_handle* h, int slot, int row0, int n_rows, const
   a.head_dim = d;
   a.rank_r = r;
   a.rank_s = s;
+  a.num_slots = p.num_slots;
+  a.status = h->d_status;
+  const long long heads = (long long)a.n * Hkv, wave = 2LL * h->num_sms;
+  a.tokens_per_cta = (int)std::max<long long>(1, (heads + wave - 1) / wave);
+  bool stage = false;
+  const size_t smem = encode_smem(p, &stage);
+  a.stage = stage;
+  const dim3 grid((a.n + a.tokens_per_cta - 1) / a.tokens_per_cta, Hkv);
+  if (p.dtype == BASISKV_DTYPE_BF16) encode_kernel<__nv_bfloat16><<<grid, kEncodeThreads, smem, st>>>(a);
+  else encode_kernel<float><<<grid, kEncodeThreads, smem, st>>>(a);
+  CUDA_TRY(cudaGetLastError());
+  return BASISKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int basiskv_encode_rows(basiskv_handle* h, int slot, int row0, int n_rows, const void* k, const void* v,
+                        basiskv_stream_t stream) {
+  int rc = check_handle(h);
+  if (rc) return rc;
+  const basiskv_params& p = h->p;
+  if (slot < 0 || slot >= p.num_slots) return fail(BASISKV_ERR_INVALID_ARG, "slot %d outside [0, %d)", slot, p.num_slots);
+  if (n_rows < 1 || row0 < 0 || row0 + n_rows > p.page_size)
+    return fail(BASISKV_ERR_INVALID_ARG, "rows [%d, %d) outside a page of %d", row0, row0 + n_rows, p.page_size);
+  if (!k || !v) return fail(BASISKV_ERR_INVALID_ARG, "k or v is NULL");
+  EncodeArgs a{};
+  a.k = k;
+  a.v = v;
+  a.tok_stride = p.head_dim;
+  a.head_stride = (long long)n_rows * p.head_dim;
   a.slot = slot;
   a.row0 = row0;
   a.n = n_rows;
-  const dim3 grid(n_rows, Hkv);
-  const size_t smem = sizeof(float) * (3 * (size_t)d + r);
-  cudaStream_t st = (cudaStream_t)stream;
-  if (p.dtype == BASISKV_DTYPE_BF16) encode_rows_kernel<__nv_bfloat16><<<grid, kEncodeThreads, smem, st>>>(a);
-  else encode_rows_kernel<float><<<grid, kEncodeThreads, smem, st>>>(a);
-  CUDA_TRY(cudaGetLastError());
-  return BASISKV_OK;
+  return launch_encode(h, a, (cudaStream_t)stream);
+}
+
+int basiskv_encode_tokens(basiskv_handle* h, int n, const int32_t* slots, const int32_t* rows, const void* k,
+                          const void* v, basiskv_stream_t stream) {
+  int rc = check_handle(h);
+  if (rc) return rc;
+  if (n < 0) return fail(BASISKV_ERR_INVALID_ARG, "n %d < 0", n);
+  if (n == 0) return BASISKV_OK;
+  if (!slots || !rows || !k || !v) return fail(BASISKV_ERR_INVALID_ARG, "slots, rows, k or v is NULL");
+  const basiskv_params& p = h->p;
+  EncodeArgs a{};
+  a.k = k;
+  a.v = v;
+  a.tok_stride = (long long)p.num_kv_heads * p.head_dim;
+  a.head_stride = p.head_dim;
+  a.slots = slots;
+  a.rows = rows;
+  a.n = n;
+  return launch_encode(h, a, (cudaStream_t)stream);
 }
 
 int basiskv_quantize_keys(basiskv_handle* h, const void* k, int64_t row0, int64_t n_rows,
@@ -1110,10 +1181,12 @@ extern "C" int basiskv_decode_attn_noalloc(const basiskv_params* p, int batch, c
   const dim3 rgrid((p->max_pages_per_seq + ppc - 1) / ppc, p->num_kv_heads, batch);
   const size_t rsmem = generic_route_smem(*p);
   if (p->dtype == BASISKV_DTYPE_BF16) {
-    CUDA_TRY(cudaFuncSetAttribute(&route_generic_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
+    rc = set_smem_attr((const void*)&route_generic_kernel<__nv_bfloat16>, rsmem);
+    if (rc) return rc;
     route_generic_kernel<__nv_bfloat16><<<rgrid, kRouteThreads, rsmem, st>>>(ra);
   } else {
-    CUDA_TRY(cudaFuncSetAttribute(&route_generic_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
+    rc = set_smem_attr((const void*)&route_generic_kernel<float>, rsmem);
+    if (rc) return rc;
     route_generic_kernel<float><<<rgrid, kRouteThreads, rsmem, st>>>(ra);
   }
   CUDA_TRY(cudaGetLastError());
@@ -1154,10 +1227,12 @@ extern "C" int basiskv_decode_attn_noalloc(const basiskv_params* p, int batch, c
   const size_t asmem = sizeof(float) * std::max(g * (p->head_dim + p->page_size + p->rank_r) + 3 * g,
                                                 combine_smem_floats(splits, p->gqa_group, p->rank_r));
   if (p->dtype == BASISKV_DTYPE_BF16) {
-    CUDA_TRY(cudaFuncSetAttribute(&attn_generic_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asmem));
+    rc = set_smem_attr((const void*)&attn_generic_kernel<__nv_bfloat16>, asmem);
+    if (rc) return rc;
     attn_generic_kernel<__nv_bfloat16><<<agrid, kAttnThreads, asmem, st>>>(aa);
   } else {
-    CUDA_TRY(cudaFuncSetAttribute(&attn_generic_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asmem));
+    rc = set_smem_attr((const void*)&attn_generic_kernel<float>, asmem);
+    if (rc) return rc;
     attn_generic_kernel<float><<<agrid, kAttnThreads, asmem, st>>>(aa);
   }
   CUDA_TRY(cudaGetLastError());

@@ -18,8 +18,11 @@
 namespace basiskv {
 
 struct EncodeArgs {
-  const void* k;      // [Hkv][n][d] pool dtype
-  const void* v;      // [Hkv][n][d] pool dtype
+  // incoming keys and values, pool dtype: element (token i, KV head h, channel c)
+  // at i * tok_stride + h * head_stride + c
+  const void* k;
+  const void* v;
+  long long tok_stride, head_stride;
   void* k_pool;       // [slots][Hkv][P][d]: pool dtype, or int8 codes when k_int8
   float* k_scale;     // [slots][Hkv][P] (k_int8 only)
   int k_int8;
@@ -28,8 +31,15 @@ struct EncodeArgs {
   const float* a_v;   // [Hkv][d][r]
   const float* a_r;   // [Hkv][d][s]
   const float* w_zk;  // [Hkv][r][d]
-  int num_kv_heads, page_size, head_dim, rank_r, rank_s;
-  int slot, row0, n;  // rows [row0, row0 + n) of pool slot `slot`
+  int num_kv_heads, page_size, head_dim, rank_r, rank_s, num_slots;
+  // destinations: token i goes to row (row0 + i) of pool slot `slot`, or,
+  // when `slots` is not null, to row rows[i] of slot slots[i]
+  int slot, row0, n;
+  const int32_t* slots;
+  const int32_t* rows;
+  int tokens_per_cta;
+  int stage;          // copy the KV head's A_v, W_zk, A_r to shared memory first
+  uint32_t* status;
 };
 
 constexpr int kEncodeThreads = 128;
@@ -115,53 +125,96 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
 }
 
-// One CTA per (row, KV head); fp32 arithmetic, outputs rounded to the pool
-// dtype.  Dynamic shared memory: (3d + r) floats.
+// Grid (ceil(n / tokens_per_cta), Hkv): a CTA encodes tokens_per_cta
+// consecutive tokens of one KV head, in fp32, outputs rounded to the pool
+// dtype.  With `stage`, the head's A_v [d][r], W_zk [r][d] and A_r [d][s]
+// are first copied to shared memory (coalesced) and every product reads
+// them there; otherwise they are read from global memory.  Dynamic shared
+// memory: (3d + r) floats, plus (2dr + ds) floats with `stage`.
+// Destinations outside the pool set BAD_SLOT and are skipped.
 template <typename T>
-__global__ void __launch_bounds__(kEncodeThreads) encode_rows_kernel(const EncodeArgs a) {
+__global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs a) {
   extern __shared__ float esm[];
-  const int i = blockIdx.x, kvh = blockIdx.y, tid = threadIdx.x;
+  const int kvh = blockIdx.y, tid = threadIdx.x;
   const int d = a.head_dim, r = a.rank_r, s = a.rank_s;
   float* kr = esm;      // [d] incoming key
   float* vr = kr + d;   // [d] incoming value
   float* z = vr + d;    // [r] stored latent, widened back
   float* res = z + r;   // [d] key minus its prediction from the stored latent
-  const size_t in = ((size_t)kvh * a.n + i) * d;
-  const size_t row = ((size_t)a.slot * a.num_kv_heads + kvh) * a.page_size + a.row0 + i;
-  const T* k = static_cast<const T*>(a.k) + in;
-  const T* v = static_cast<const T*>(a.v) + in;
-  for (int c = tid; c < d; c += kEncodeThreads) {
-    kr[c] = to_f32(k[c]);
-    vr[c] = to_f32(v[c]);
-    if (!a.k_int8) static_cast<T*>(a.k_pool)[row * d + c] = k[c];
-  }
-  if (a.k_int8 && tid < 32)
-    warp_quantize_row(k, d, static_cast<int8_t*>(a.k_pool) + row * d, a.k_scale + row, tid);
-  __syncthreads();
   const float* Av = a.a_v + (size_t)kvh * d * r;
-  T* zp = static_cast<T*>(a.z_pool) + row * r;
-  for (int j = tid; j < r; j += kEncodeThreads) {
-    float acc = 0.f;
-    for (int c = 0; c < d; ++c) acc = fmaf(vr[c], Av[(size_t)c * r + j], acc);
-    const T zt = from_f32<T>(acc);
-    zp[j] = zt;
-    z[j] = to_f32(zt);
-  }
-  if (s == 0) return;
-  __syncthreads();
   const float* W = a.w_zk + (size_t)kvh * r * d;
-  for (int c = tid; c < d; c += kEncodeThreads) {
-    float acc = kr[c];
-    for (int t = 0; t < r; ++t) acc = fmaf(-z[t], W[(size_t)t * d + c], acc);
-    res[c] = acc;
-  }
-  __syncthreads();
   const float* Ar = a.a_r + (size_t)kvh * d * s;
-  T* rp = static_cast<T*>(a.r_pool) + row * s;
-  for (int j = tid; j < s; j += kEncodeThreads) {
-    float acc = 0.f;
-    for (int c = 0; c < d; ++c) acc = fmaf(res[c], Ar[(size_t)c * s + j], acc);
-    rp[j] = from_f32<T>(acc);
+  if (a.stage) {
+    float* sav = res + d;
+    float* sw = sav + d * r;
+    float* sar = sw + r * d;
+    const bool vec = ((d * r) % 4 == 0) && ((d * s) % 4 == 0) &&
+                     ((reinterpret_cast<uintptr_t>(Av) | reinterpret_cast<uintptr_t>(W) |
+                       reinterpret_cast<uintptr_t>(Ar) | reinterpret_cast<uintptr_t>(sav)) & 15u) == 0;
+    if (vec) {  // 16-byte loads: a quarter of the load instructions
+      for (int e = tid; e < d * r / 4; e += kEncodeThreads) {
+        reinterpret_cast<float4*>(sav)[e] = __ldg(reinterpret_cast<const float4*>(Av) + e);
+        reinterpret_cast<float4*>(sw)[e] = __ldg(reinterpret_cast<const float4*>(W) + e);
+      }
+      for (int e = tid; e < d * s / 4; e += kEncodeThreads)
+        reinterpret_cast<float4*>(sar)[e] = __ldg(reinterpret_cast<const float4*>(Ar) + e);
+    } else {
+      for (int e = tid; e < d * r; e += kEncodeThreads) {
+        sav[e] = Av[e];
+        sw[e] = W[e];
+      }
+      for (int e = tid; e < d * s; e += kEncodeThreads) sar[e] = Ar[e];
+    }
+    Av = sav;
+    W = sw;
+    Ar = sar;
+  }
+  const int i_end = min(a.n, (int)(blockIdx.x + 1) * a.tokens_per_cta);
+  for (int i = blockIdx.x * a.tokens_per_cta; i < i_end; ++i) {
+    int slot = a.slot, prow = a.row0 + i;
+    if (a.slots) {
+      slot = a.slots[i];
+      prow = a.rows[i];
+    }
+    if (slot < 0 || slot >= a.num_slots || prow < 0 || prow >= a.page_size) {
+      if (tid == 0) atomicOr(a.status, kStatusBadSlot);
+      continue;  // uniform over the CTA: the same token for every thread
+    }
+    const size_t in = (size_t)i * a.tok_stride + (size_t)kvh * a.head_stride;
+    const size_t row = ((size_t)slot * a.num_kv_heads + kvh) * a.page_size + prow;
+    const T* k = static_cast<const T*>(a.k) + in;
+    const T* v = static_cast<const T*>(a.v) + in;
+    __syncthreads();  // the previous token's buffers (and the staged bases) are settled
+    for (int c = tid; c < d; c += kEncodeThreads) {
+      kr[c] = to_f32(k[c]);
+      vr[c] = to_f32(v[c]);
+      if (!a.k_int8) static_cast<T*>(a.k_pool)[row * d + c] = k[c];
+    }
+    if (a.k_int8 && tid < 32)
+      warp_quantize_row(k, d, static_cast<int8_t*>(a.k_pool) + row * d, a.k_scale + row, tid);
+    __syncthreads();
+    T* zp = static_cast<T*>(a.z_pool) + row * r;
+    for (int j = tid; j < r; j += kEncodeThreads) {
+      float acc = 0.f;
+      for (int c = 0; c < d; ++c) acc = fmaf(vr[c], Av[(size_t)c * r + j], acc);
+      const T zt = from_f32<T>(acc);
+      zp[j] = zt;
+      z[j] = to_f32(zt);
+    }
+    if (s == 0) continue;
+    __syncthreads();
+    for (int c = tid; c < d; c += kEncodeThreads) {
+      float acc = kr[c];
+      for (int t = 0; t < r; ++t) acc = fmaf(-z[t], W[(size_t)t * d + c], acc);
+      res[c] = acc;
+    }
+    __syncthreads();
+    T* rp = static_cast<T*>(a.r_pool) + row * s;
+    for (int j = tid; j < s; j += kEncodeThreads) {
+      float acc = 0.f;
+      for (int c = 0; c < d; ++c) acc = fmaf(res[c], Ar[(size_t)c * s + j], acc);
+      rp[j] = from_f32<T>(acc);
+    }
   }
 }
 

@@ -209,7 +209,8 @@ BASISKV_API int basiskv_decode_attn_host(basiskv_handle *h, int batch, const voi
  *   does, codes and scale);
  *   Z = V . pinv(B_v), rounded to the pool dtype;
  *   R = (K - Z . W_zk) . pinv(B_r), from the rounded Z, rounded.
- * With basiskv_quantize_keys, the only calls that write the caller's pools
+ * With basiskv_encode_tokens and basiskv_quantize_keys, the only calls that
+ * write the caller's pools
  * (and k_scale).  The first call computes
  * the pseudo-inverses of the bases on the host (synchronous); later calls
  * only enqueue on `stream`.  The page table is not touched: follow with
@@ -218,6 +219,18 @@ BASISKV_API int basiskv_decode_attn_host(basiskv_handle *h, int batch, const voi
  * CUDA. */
 BASISKV_API int basiskv_encode_rows(basiskv_handle *h, int slot, int row0, int n_rows, const void *k,
                         const void *v, basiskv_stream_t stream);
+
+/* The same encode for a list of n tokens at arbitrary pool positions, in
+ * one launch: the decode-time append of one new token per sequence.  Token
+ * i, every KV head, goes to row rows[i] of pool slot slots[i] (slots, rows:
+ * device int32 [n]); k, v [n][Hkv][d] (pool dtype, device: the layout of a
+ * layer's new keys and values).  Entries outside the pool (slot not in
+ * [0, num_slots) or row not in [0, P)) set BASISKV_STATUS_BAD_SLOT and are
+ * skipped.  Arithmetic, rounding and the page table as basiskv_encode_rows.
+ * Errors: INVALID_ARG (n < 0, NULL pointer; bases with linearly dependent
+ * rows), CUDA. */
+BASISKV_API int basiskv_encode_tokens(basiskv_handle *h, int n, const int32_t *slots, const int32_t *rows,
+                          const void *k, const void *v, basiskv_stream_t stream);
 
 /* Store keys into an int8 key pool (k_format = BASISKV_KEYS_INT8): rows
  * [row0, row0 + n_rows) of the pool in its flat row order, row =
