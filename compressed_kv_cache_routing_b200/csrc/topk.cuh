@@ -26,6 +26,7 @@ struct TopkSmem {
   int scan_tmp[32];
   int digit;
   int remaining;
+  int whole;  // the digit's whole bucket is selected: later passes cannot change the set
 };
 
 // Select min(k, n) of the n scores at `scores` (global, written by other
@@ -171,7 +172,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkArgs a) {
   for (int i = tid; i < n; i += kTopkThreads) keys[i] = score_key(__ldcg(sc + i));
   __syncthreads();
   const int kb = a.topk < n ? a.topk : n;
-  uint32_t thr = 0u;
+  uint32_t thr = 0u, tmask = 0xFFFFFFFFu;  // keys compare on their bits under tmask
   int need = 0;
   if (kb < n) {
     uint32_t prefix = 0u, mask = 0u;
@@ -210,6 +211,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkArgs a) {
             if (acc + c >= remaining) {
               sm.digit = 8 * lane + q;
               sm.remaining = remaining - acc;
+              sm.whole = remaining - acc == c;
               break;
             }
             acc += c;
@@ -220,9 +222,12 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkArgs a) {
       prefix |= static_cast<uint32_t>(sm.digit) << shift;
       mask |= 0xFFu << shift;
       remaining = sm.remaining;
+      const bool whole = sm.whole;
       __syncthreads();
+      if (whole) break;  // every key of the bucket is taken: the set is decided
     }
     thr = prefix;
+    tmask = mask;
     need = remaining;
   }
   // page-ordered compaction: each thread owns a contiguous run
@@ -230,12 +235,12 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkArgs a) {
   const int i0 = min(n, tid * per), i1 = min(n, i0 + per);
   int total;
   int eq = 0, take = 0;
-  for (int i = i0; i < i1; ++i) eq += keys[i] == thr;
+  for (int i = i0; i < i1; ++i) eq += (keys[i] & tmask) == thr;
   const int eq_before = kb < n ? block_exclusive_scan<kTopkThreads>(eq, sm.scan_tmp, &total) : 0;
   {
     int e = eq_before;
     for (int i = i0; i < i1; ++i) {
-      const uint32_t key = keys[i];
+      const uint32_t key = keys[i] & tmask;
       take += kb >= n || key > thr || (key == thr && e < need);
       e += key == thr;
     }
@@ -244,7 +249,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkArgs a) {
   {
     int e = eq_before;
     for (int i = i0; i < i1; ++i) {
-      const uint32_t key = keys[i];
+      const uint32_t key = keys[i] & tmask;
       if (kb >= n || key > thr || (key == thr && e < need)) {
         sel[pos] = i;
         if (so) so[pos] = i;
