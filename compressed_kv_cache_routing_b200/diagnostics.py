@@ -44,6 +44,8 @@ def routing_recall(*, q, z_pool, r_pool, k_pool, w_zk, b_r, b_v, page_table, seq
     ``seq_lens`` [B] are host int32 arrays.  Returns a dict with ``recall``
     [B][Hkv] (1 where every page is selected anyway), ``attn_err`` [B][Hq],
     and their means."""
+    if k_pool.dtype == torch.int8:
+        raise ValueError("routing_recall needs the full-precision keys: exact-key routing reads them as latents")
     page_table = np.ascontiguousarray(np.where(page_table >= 0, page_table, 0), dtype=np.int32)
     seq_lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
     B, max_pages = page_table.shape
