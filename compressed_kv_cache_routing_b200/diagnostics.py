@@ -41,7 +41,8 @@ def routing_recall(*, q, z_pool, r_pool, k_pool, w_zk, b_r, b_v, page_table, seq
     error of the sketch's selection against attention over every page.
 
     Tensors as for ``BasisKV`` (device); ``page_table`` [B][max_pages] and
-    ``seq_lens`` [B] are host int32 arrays.  Returns a dict with ``recall``
+    ``seq_lens`` [B] are host int32 arrays; ``k_pool`` holds the keys in the
+    pool dtype (not int8 codes).  Returns a dict with ``recall``
     [B][Hkv] (1 where every page is selected anyway), ``attn_err`` [B][Hq],
     and their means."""
     if k_pool.dtype == torch.int8:
