@@ -580,7 +580,7 @@ int check_call(basiskv_handle* h, int batch, const void* q, int topk) {
 
 extern "C" {
 
-int basiskv_version(void) { return 100; }
+int basiskv_version(void) { return BASISKV_VERSION; }
 
 const char* basiskv_last_error(void) { return g_last_error.c_str(); }
 

@@ -308,7 +308,11 @@ BASISKV_API int basiskv_decode_attn_noalloc(const basiskv_params *p, int batch,
 /* Thread-local message for the last non-zero return of this thread. */
 BASISKV_API const char *basiskv_last_error(void);
 
-/* Library version, major * 10000 + minor * 100 + patch. */
+/* Library version, major * 10000 + minor * 100 + patch: BASISKV_VERSION
+ * of the header the library was built with.  0.2.0 added int8 key pages
+ * (k_format, k_scale in basiskv_params), basiskv_quantize_keys and
+ * basiskv_encode_tokens. */
+#define BASISKV_VERSION 200
 BASISKV_API int basiskv_version(void);
 
 #ifdef __cplusplus

@@ -32,7 +32,8 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version(lib):
-    assert bk.basiskv_version() >= 100
+    hdr = open(HEADER).read()
+    assert bk.basiskv_version() == int(re.search(r"#define BASISKV_VERSION (\d+)", hdr).group(1))
 
 
 def _params(**kw):
