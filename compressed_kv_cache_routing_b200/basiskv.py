@@ -40,7 +40,7 @@ EXPORTED = (
     "basiskv_decode_attn_host", "basiskv_route", "basiskv_get_status", "basiskv_profile_begin",
     "basiskv_profile_end", "basiskv_last_launch", "basiskv_last_error", "basiskv_version",
     "basiskv_decode_attn_noalloc", "basiskv_decode_attn_latent", "basiskv_encode_rows",
-    "basiskv_quantize_keys", "basiskv_encode_tokens",
+    "basiskv_quantize_keys", "basiskv_encode_tokens", "basiskv_append_page_copy",
 )
 
 
@@ -82,6 +82,7 @@ def load(path: str = LIB_PATH):
         "basiskv_create": [ctypes.POINTER(basiskv_params), ctypes.POINTER(ctypes.c_void_p)],
         "basiskv_destroy": [H],
         "basiskv_append_page": [H, i32, i32, i32, vp],
+        "basiskv_append_page_copy": [H, i32, i32, i32, vp, vp, vp, vp, vp],
         "basiskv_append_tokens": [H, i32, i32, vp],
         "basiskv_reset_seq": [H, i32, vp],
         "basiskv_load_page_table": [H, i32, vp, i32, vp, vp],
@@ -142,6 +143,14 @@ def basiskv_destroy(h: int) -> None:
 
 def basiskv_append_page(h, seq, slot, n_tokens, stream=None):
     _check(load().basiskv_append_page(h, seq, slot, n_tokens, _stream(stream)))
+
+
+def basiskv_append_page_copy(h, seq, slot, z, r, k, k_scale=None, stream=None):
+    """Copy one page's rows (z [Hkv][n][r], r [Hkv][n][s] or None, k
+    [Hkv][n][d], k_scale [Hkv][n] with int8 keys) into pool slot ``slot``
+    and append it to sequence ``seq`` with n valid tokens."""
+    _check(load().basiskv_append_page_copy(h, seq, slot, int(z.shape[1]), _ptr(z), _ptr(r), _ptr(k), _ptr(k_scale),
+                                           _stream(stream)))
 
 
 def basiskv_append_tokens(h, seq, n_tokens, stream=None):

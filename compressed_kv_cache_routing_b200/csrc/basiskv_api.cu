@@ -712,6 +712,40 @@ int basiskv_append_page(basiskv_handle* h, int seq, int slot, int n_tokens, basi
   return BASISKV_OK;
 }
 
+int basiskv_append_page_copy(basiskv_handle* h, int seq, int slot, int n_tokens, const void* z, const void* r,
+                             const void* k, const float* k_scale, basiskv_stream_t stream) {
+  int rc = check_handle(h);
+  if (rc) return rc;
+  const basiskv_params& p = h->p;
+  const bool int8 = p.k_format == BASISKV_KEYS_INT8;
+  if (!z || !k || (p.rank_s > 0 && !r) || (int8 && !k_scale))
+    return fail(BASISKV_ERR_INVALID_ARG, "z, k (and r when s > 0, k_scale with int8 keys) are required");
+  // the checks of basiskv_append_page, before anything is copied
+  if (seq < 0 || seq >= p.max_batch) return fail(BASISKV_ERR_INVALID_ARG, "seq %d outside [0, %d)", seq, p.max_batch);
+  if (slot < 0 || slot >= p.num_slots) return fail(BASISKV_ERR_INVALID_ARG, "slot %d outside [0, %d)", slot, p.num_slots);
+  if (n_tokens < 1 || n_tokens > p.page_size)
+    return fail(BASISKV_ERR_INVALID_ARG, "n_tokens %d outside [1, %d]", n_tokens, p.page_size);
+  const int n = h->h_npages[seq];
+  if (n > 0 && h->h_lens[seq] != n * p.page_size)
+    return fail(BASISKV_ERR_STATE, "sequence %d ends in a partial page", seq);
+  if (n >= p.max_pages_per_seq) return fail(BASISKV_ERR_CAPACITY, "sequence %d already has %d pages", seq, n);
+  // one strided copy per pool: source [Hkv][n_tokens][w], destination rows
+  // [0, n_tokens) of the slot's page of every KV head
+  cudaStream_t st = (cudaStream_t)stream;
+  auto copy = [&](void* pool, const void* src, size_t row_bytes) -> int {
+    uint8_t* dst = static_cast<uint8_t*>(pool) + (size_t)slot * p.num_kv_heads * p.page_size * row_bytes;
+    CUDA_TRY(cudaMemcpy2DAsync(dst, p.page_size * row_bytes, src, n_tokens * row_bytes, n_tokens * row_bytes,
+                               p.num_kv_heads, cudaMemcpyDeviceToDevice, st));
+    return BASISKV_OK;
+  };
+  rc = copy(const_cast<void*>(p.z_pool), z, h->elem * p.rank_r);
+  if (!rc && p.rank_s > 0) rc = copy(const_cast<void*>(p.r_pool), r, h->elem * p.rank_s);
+  if (!rc) rc = copy(const_cast<void*>(p.k_pool), k, (int8 ? 1 : h->elem) * p.head_dim);
+  if (!rc && int8) rc = copy(const_cast<float*>(p.k_scale), k_scale, sizeof(float));
+  if (rc) return rc;
+  return basiskv_append_page(h, seq, slot, n_tokens, stream);
+}
+
 int basiskv_append_tokens(basiskv_handle* h, int seq, int n_tokens, basiskv_stream_t stream) {
   int rc = check_handle(h);
   if (rc) return rc;

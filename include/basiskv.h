@@ -145,6 +145,18 @@ BASISKV_API int basiskv_destroy(basiskv_handle *h);
 BASISKV_API int basiskv_append_page(basiskv_handle *h, int seq, int slot, int n_tokens,
                         basiskv_stream_t stream);
 
+/* basiskv_append_page that first copies the page's rows into the slot:
+ * z [Hkv][n_tokens][r], r [Hkv][n_tokens][s] (NULL when s = 0) and
+ * k [Hkv][n_tokens][d], in the pool dtype (k: int8 codes with int8 keys,
+ * then also k_scale [Hkv][n_tokens] fp32; NULL otherwise), all device
+ * memory, go to rows [0, n_tokens) of slot `slot`, every KV head (one
+ * strided device-to-device copy per pool, on `stream`).  Nothing is copied
+ * when the append would fail.  Errors: those of basiskv_append_page,
+ * INVALID_ARG for a missing pointer, CUDA. */
+BASISKV_API int basiskv_append_page_copy(basiskv_handle *h, int seq, int slot, int n_tokens, const void *z,
+                             const void *r, const void *k, const float *k_scale,
+                             basiskv_stream_t stream);
+
 /* Grow the last (partial) page of `seq` by n_tokens; the new rows must
  * already be written in its slot.  Errors: INVALID_ARG, STATE (no page, or
  * the page would overflow P). */
@@ -310,8 +322,8 @@ BASISKV_API const char *basiskv_last_error(void);
 
 /* Library version, major * 10000 + minor * 100 + patch: BASISKV_VERSION
  * of the header the library was built with.  0.2.0 added int8 key pages
- * (k_format, k_scale in basiskv_params), basiskv_quantize_keys and
- * basiskv_encode_tokens. */
+ * (k_format, k_scale in basiskv_params), basiskv_quantize_keys,
+ * basiskv_encode_tokens and basiskv_append_page_copy. */
 #define BASISKV_VERSION 200
 BASISKV_API int basiskv_version(void);
 

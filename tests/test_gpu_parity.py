@@ -358,3 +358,68 @@ def test_invalid_calls_rejected():
     with pytest.raises(bk.BasisKVError):
         bk.basiskv_load_page_table(kv.handle, np.full((1, 64), 10 ** 6), np.array([1024]))
     kv.close()
+
+
+def _rebuilt_by_copy(w, k_pool, k_scale=None):
+    """A handle over empty pools filled page by page with
+    basiskv_append_page_copy from w's pools (same slots)."""
+    s = w.spec
+    z2, r2, k2 = torch.zeros_like(w.z_pool), torch.zeros_like(w.r_pool), torch.zeros_like(k_pool)
+    sc2 = torch.zeros_like(k_scale) if k_scale is not None else None
+    kv = bk.BasisKV(z_pool=z2, r_pool=r2, k_pool=k2, w_zk=w.w_zk, b_r=w.b_r, b_v=w.b_v, gqa_group=s.gqa_group,
+                    max_batch=s.batch, max_pages_per_seq=w.page_table.shape[1], max_topk=s.topk, k_scale=sc2)
+    P = s.page_size
+    for b, L in enumerate(w.seq_lens.tolist()):
+        for j in range(-(-L // P)):
+            slot, n = int(w.page_table[b, j]), min(P, L - j * P)
+            bk.basiskv_append_page_copy(kv.handle, b, slot, w.z_pool[slot, :, :n].contiguous(),
+                                        w.r_pool[slot, :, :n].contiguous(), k_pool[slot, :, :n].contiguous(),
+                                        k_scale[slot, :, :n].contiguous() if k_scale is not None else None)
+    return kv
+
+
+@pytest.mark.parametrize("int8", [False, True])
+def test_append_page_copy_matches_prefilled_pools(int8):
+    """Pages copied into empty pools by basiskv_append_page_copy decode to
+    the same bits as the same pages written in place."""
+    w = W.generate(SMALL["llama3_8b_decode"], device="cuda")
+    s = w.spec
+    if int8:
+        k_pool = torch.empty(tuple(w.k_pool.shape), dtype=torch.int8, device="cuda")
+        k_scale = torch.empty(tuple(w.k_pool.shape[:3]), device="cuda")
+        ref = bk.BasisKV(z_pool=w.z_pool, r_pool=w.r_pool, k_pool=k_pool, w_zk=w.w_zk, b_r=w.b_r, b_v=w.b_v,
+                         gqa_group=s.gqa_group, max_batch=s.batch, max_pages_per_seq=w.page_table.shape[1],
+                         max_topk=s.topk, k_scale=k_scale)
+        bk.basiskv_quantize_keys(ref.handle, w.k_pool)
+        bk.basiskv_load_page_table(ref.handle, np.where(w.page_table >= 0, w.page_table, 0), w.seq_lens)
+    else:
+        k_pool, k_scale = w.k_pool, None
+        ref = bk.BasisKV.for_workload(w)
+    kv = _rebuilt_by_copy(w, k_pool, k_scale)
+    outs = []
+    for h in (ref, kv):
+        out = torch.empty((s.batch, s.num_q_heads, s.head_dim), device="cuda")
+        sel = torch.empty((s.batch, s.num_kv_heads, s.topk), device="cuda", dtype=torch.int32)
+        bk.basiskv_decode_attn(h.handle, w.q, s.topk, s.softmax_scale, out, sel)
+        torch.cuda.synchronize()
+        assert bk.basiskv_get_status(h.handle) == 0
+        outs.append((out.cpu(), sel.cpu()))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    kv.close()
+    ref.close()
+
+
+def test_append_page_copy_refused_copies_nothing():
+    w = W.generate(SMALL["llama3_8b_decode"], device="cuda")
+    s = w.spec
+    z2, r2, k2 = torch.zeros_like(w.z_pool), torch.zeros_like(w.r_pool), torch.zeros_like(w.k_pool)
+    kv = bk.BasisKV(z_pool=z2, r_pool=r2, k_pool=k2, w_zk=w.w_zk, b_r=w.b_r, b_v=w.b_v, gqa_group=s.gqa_group,
+                    max_batch=s.batch, max_pages_per_seq=4, max_topk=s.topk)
+    zs, rs, ks = w.z_pool[0, :, :5].contiguous(), w.r_pool[0, :, :5].contiguous(), w.k_pool[0, :, :5].contiguous()
+    bk.basiskv_append_page_copy(kv.handle, 0, 1, zs, rs, ks)          # a partial page: the sequence ends here
+    with pytest.raises(bk.BasisKVError):
+        bk.basiskv_append_page_copy(kv.handle, 0, 2, zs, rs, ks)      # appending after a partial page
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(z2[2]) == 0 and torch.count_nonzero(k2[2]) == 0
+    assert torch.equal(z2[1, :, :5], zs) and torch.count_nonzero(z2[1, :, 5:]) == 0
+    kv.close()
