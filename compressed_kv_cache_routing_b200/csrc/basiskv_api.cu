@@ -48,6 +48,7 @@ constexpr int kPartsCap = kMaxSplits * kAttnWarps;  // partials per unit
 // with copies in flight) share an SM.
 constexpr size_t kRouteSmemBudget = 48 * 1024;
 constexpr size_t kAttnSmemBudget = 100 * 1024;
+constexpr size_t kAttnSmemBudgetWide = 64 * 1024;  // attention rings when r >= 64
 
 using KernelFn = void (*)(const RouteArgs);
 using AttnFn = void (*)(const AttnArgs);
@@ -244,19 +245,26 @@ void choose_kernels(basiskv_handle* h) {
     }
   }
   const bool k8 = p.k_format == BASISKV_KEYS_INT8;
-  for (int tps : {64, 32, 16}) {
-    if (p.page_size % tps) continue;
-    auto ait = attn_table().find(AttnKey{p.gqa_group, p.head_dim, p.rank_r, tps, k8});
-    if (ait == attn_table().end()) continue;
-    const size_t stage = (size_t)tps * (p.head_dim * (k8 ? 1 : es) + p.rank_r * es + (k8 ? 4 : 0));
-    int st = (int)std::min<size_t>(4, kAttnSmemBudget / (kAttnWarps * stage));
-    if (st < 1) continue;
-    if (st < 2 && tps > 16) continue;  // prefer a smaller stage with double buffering
-    h->attn_fn = ait->second;
-    h->attn_tps = tps;
-    h->attn_stages = st;
-    h->attn_smem = kAttnWarps * st * stage + sizeof(float) * kAttnWarps * p.gqa_group * p.rank_r;
-    break;
+  // Where P.Z is heavy (r >= 64) more resident warps pay for shallower
+  // rings: a 64 KB ring lets three CTAs share an SM (dense limit, r = 128:
+  // 120 us against 123 us, 111 against 115 with int8 keys); at r = 32 the
+  // deeper rings are faster.  The default budget applies when no compiled
+  // shape fits the smaller one.
+  for (size_t budget : {p.rank_r >= 64 ? kAttnSmemBudgetWide : kAttnSmemBudget, kAttnSmemBudget}) {
+    for (int tps : {64, 32, 16}) {
+      if (p.page_size % tps) continue;
+      auto ait = attn_table().find(AttnKey{p.gqa_group, p.head_dim, p.rank_r, tps, k8});
+      if (ait == attn_table().end()) continue;
+      const size_t stage = (size_t)tps * (p.head_dim * (k8 ? 1 : es) + p.rank_r * es + (k8 ? 4 : 0));
+      int st = (int)std::min<size_t>(4, budget / (kAttnWarps * stage));
+      if (st < 1) continue;
+      if (st < 2 && tps > 16) continue;  // prefer a smaller stage with double buffering
+      h->attn_fn = ait->second;
+      h->attn_tps = tps;
+      h->attn_stages = st;
+      h->attn_smem = kAttnWarps * st * stage + sizeof(float) * kAttnWarps * p.gqa_group * p.rank_r;
+      return;
+    }
   }
 }
 
