@@ -1,8 +1,11 @@
 """Writes tiny_oracle.json: the oracle's result on the seeded "tiny" workload
 (batch 1, 1 KV head, GQA 4, d 64, 1024 tokens, page 16, r 16, s 8, top-8,
-fp32, seed 0).  Calls only the generator and oracle/.  Run from the repo root:
+fp32, seed 0), and the same with the keys quantised to int8 by the oracle's
+quantiser and in latent-output mode.  Calls only the generator and oracle/.
+Run from the repo root:
     python tests/golden/make_golden.py
 """
+import dataclasses
 import hashlib
 import json
 import os
@@ -24,6 +27,11 @@ def input_digest(prob):
     return h.hexdigest()
 
 
+def int8_problem(prob):
+    codes, scales = oracle.quantize_keys(prob.k_pool)
+    return dataclasses.replace(prob, k_pool=codes, k_scale=scales)
+
+
 def main():
     w = W.generate("tiny")
     prob = to_problem(w)
@@ -38,6 +46,16 @@ def main():
         "page_scores": [float(x) for x in scores[0, 0, :n]],
         "out": [[float(x) for x in row] for row in out[0]],
     }
+    p8 = int8_problem(prob)
+    out8, sel8, _, _ = oracle.decode(p8)
+    doc["int8_keys"] = {
+        "codes_sha256": hashlib.sha256(p8.k_pool.tobytes()).hexdigest(),
+        "scales_sha256": hashlib.sha256(p8.k_scale.tobytes()).hexdigest(),
+        "sel": sel8[0, 0].tolist(),
+        "out": [[float(x) for x in row] for row in out8[0]],
+    }
+    zb, _, _, _ = oracle.decode(dataclasses.replace(prob, latent=True))
+    doc["latent"] = {"out": [[float(x) for x in row] for row in zb[0]]}
     with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "tiny_oracle.json"), "w") as f:
         json.dump(doc, f, indent=1)
 

@@ -34,6 +34,30 @@ def test_tiny_golden():
     assert np.array_equal(out[0], np.array(doc["out"]))
 
 
+def test_tiny_golden_int8_keys_and_latent():
+    """The same fixture's int8-key result (the oracle's own quantisation of
+    the keys, then decode) and latent-mode result."""
+    import dataclasses
+    import hashlib
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "make_golden", os.path.join(os.path.dirname(GOLDEN), "make_golden.py"))
+    mg = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mg)
+    with open(GOLDEN) as f:
+        doc = json.load(f)
+    prob = to_problem(W.generate("tiny"))
+    p8 = mg.int8_problem(prob)
+    g8 = doc["int8_keys"]
+    assert hashlib.sha256(p8.k_pool.tobytes()).hexdigest() == g8["codes_sha256"]
+    assert hashlib.sha256(p8.k_scale.tobytes()).hexdigest() == g8["scales_sha256"]
+    out8, sel8, _, _ = oracle.decode(p8)
+    assert sel8[0, 0].tolist() == g8["sel"]
+    assert np.array_equal(out8[0], np.array(g8["out"]))
+    zb, _, _, _ = oracle.decode(dataclasses.replace(prob, latent=True))
+    assert np.array_equal(zb[0], np.array(doc["latent"]["out"]))
+
+
 def test_unit_sampling_matches_full_run():
     """Oracle on a subset of units equals the full run on those units."""
     spec = W.shrink("high_concurrency", batch=6, len_lo=700, len_hi=1500, topk=8)
