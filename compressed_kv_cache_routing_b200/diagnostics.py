@@ -16,7 +16,15 @@ rest).  This module measures how much that approximation costs:
 Exact-key routing is the same routing step on a second handle that sees the
 key pool as its latents, with W_zk = I and no residual, so that q.Khat = q.K.
 
-    python -m compressed_kv_cache_routing_b200.diagnostics [workload ...]
+A second diagnostic measures what storing the keys as int8 codes with a
+per-token scale costs ("PackKV: Reducing KV Cache Memory Footprint through
+LLM-Aware Lossy Compression", abstract: lossy key compression at a small
+accuracy cost): the same decode step with the keys quantised on the device,
+against the step with the full-precision keys.  Routing reads no keys, so
+the selections must be identical; the output deviation is reported per
+(sequence, query head), relative to the row's largest entry.
+
+    python -m compressed_kv_cache_routing_b200.diagnostics [--int8] [workload ...]
 """
 from __future__ import annotations
 
@@ -103,13 +111,61 @@ def routing_recall_for(w, topk=None):
                           topk=s.topk if topk is None else topk, softmax_scale=s.softmax_scale)
 
 
+def key_quantization_error(w, topk=None):
+    """Output deviation caused by int8 keys on workload ``w`` (device
+    tensors): decode with w's keys and with the same keys quantised by
+    basiskv_quantize_keys.  Returns ``err`` [B][Hq] (max |y8 - y| / max |y|
+    per row), its mean and max, and whether the selections agree."""
+    s = w.spec
+    topk = s.topk if topk is None else topk
+    dev = w.q.device
+    B = len(w.seq_lens)
+    pt = np.ascontiguousarray(np.where(w.page_table >= 0, w.page_table, 0), dtype=np.int32)
+    codes = torch.empty(tuple(w.k_pool.shape), dtype=torch.int8, device=dev)
+    scales = torch.empty(tuple(w.k_pool.shape[:3]), dtype=torch.float32, device=dev)
+    common = dict(z_pool=w.z_pool, r_pool=w.r_pool, w_zk=w.w_zk, b_r=w.b_r, b_v=w.b_v, gqa_group=s.gqa_group,
+                  max_batch=B, max_pages_per_seq=max(1, pt.shape[1]), max_topk=topk)
+    native = bk.BasisKV(k_pool=w.k_pool, **common)
+    int8 = bk.BasisKV(k_pool=codes, k_scale=scales, **common)
+    try:
+        bk.basiskv_quantize_keys(int8.handle, w.k_pool)
+        res = []
+        for h in (native, int8):
+            bk.basiskv_load_page_table(h.handle, pt, w.seq_lens)
+            out = torch.empty((B, s.num_q_heads, s.head_dim), device=dev)
+            sel = torch.empty((B, s.num_kv_heads, topk), device=dev, dtype=torch.int32)
+            bk.basiskv_decode_attn(h.handle, w.q[:B], topk, s.softmax_scale, out, sel)
+            res.append((out, sel))
+        torch.cuda.synchronize(dev)
+        for h in (native, int8):
+            if bk.basiskv_get_status(h.handle, clear=True):
+                raise RuntimeError("device status set during the diagnostic")
+        (o, sl), (o8, sl8) = [(x.cpu().numpy().astype(np.float64), y.cpu().numpy()) for x, y in res]
+    finally:
+        native.close()
+        int8.close()
+    den = np.abs(o).max(axis=2)
+    err = np.where(den > 0, np.abs(o8 - o).max(axis=2) / np.where(den > 0, den, 1.0), 0.0)
+    return {"err": err, "mean_err": float(err.mean()), "max_err": float(err.max()),
+            "same_selection": bool(np.array_equal(sl, sl8))}
+
+
 def main(argv=None):
     import sys
     from . import workloads as W
-    for name in (argv if argv is not None else sys.argv[1:]) or ["llama3_8b_decode"]:
-        r = routing_recall_for(W.generate(name, device="cuda"))
-        print(f"{name:18s} mean recall {r['mean_recall']:.4f}  attention error vs every page: "
-              f"mean {r['mean_attn_err']:.3e} max {r['max_attn_err']:.3e}")
+    args = list(argv if argv is not None else sys.argv[1:])
+    int8 = "--int8" in args
+    names = [a for a in args if a != "--int8"] or ["llama3_8b_decode"]
+    for name in names:
+        w = W.generate(name, device="cuda")
+        if int8:
+            r = key_quantization_error(w)
+            print(f"{name:18s} int8 keys: same selection {r['same_selection']}  output deviation: "
+                  f"mean {r['mean_err']:.3e} max {r['max_err']:.3e}")
+        else:
+            r = routing_recall_for(w)
+            print(f"{name:18s} mean recall {r['mean_recall']:.4f}  attention error vs every page: "
+                  f"mean {r['mean_attn_err']:.3e} max {r['max_attn_err']:.3e}")
 
 
 if __name__ == "__main__":

@@ -52,3 +52,24 @@ def test_routing_recall_matches_oracle(spec, exact_recall):
         assert abs(r["mean_recall"] - recall.mean()) <= 0.02
     assert np.all((r["recall"] >= 0) & (r["recall"] <= 1))
     assert np.abs(r["attn_err"] - err).max() <= 5e-3
+
+
+def test_key_quantization_error_against_the_oracle():
+    """The int8-key deviation reported on the device equals the oracle's:
+    its decode on its own quantisation of the keys against its decode on
+    the full-precision keys (both within the parity bound of each other)."""
+    from test_gpu_int8_keys import oracle_int8
+    w = W.generate(W.shrink("llama3_8b_decode", batch=3, len_lo=2500, len_hi=5000, topk=16), device="cuda")
+    r = D.key_quantization_error(w)
+    assert r["same_selection"]
+    out, sel, _, _ = oracle.decode(to_problem(w))
+    out8, sel8, _, _ = oracle.decode(oracle_int8(w))
+    assert np.array_equal(sel, sel8)
+    den = np.abs(out).max(axis=2)
+    ref = np.abs(out8 - out).max(axis=2) / den
+    assert r["err"].shape == ref.shape
+    # the device error differs from the oracle's by at most the two paths'
+    # own parity errors (2e-3 each, relative to the same rows)
+    assert np.all(np.abs(r["err"] - ref) <= 4e-3 + 1e-6), np.abs(r["err"] - ref).max()
+    print(f"int8 keys: device mean/max deviation {r['mean_err']:.3e}/{r['max_err']:.3e}, "
+          f"oracle {ref.mean():.3e}/{ref.max():.3e}")
