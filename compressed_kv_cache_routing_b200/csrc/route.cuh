@@ -11,10 +11,12 @@
 // Page score S_j = max over the G heads and page j's valid tokens.
 //
 // Two kernels: route_mma_kernel (bf16 pools, tensor cores, persistent over a
-// flat page list, the fold done by each warp as it enters a (sequence, KV
-// head); the selection runs in the next grid) and route_generic_kernel (any
-// dtype, grid (chunks of pages, Hkv, batch), fold once per CTA, the last CTA
-// of each (sequence, KV head) runs the top-k).
+// flat page list; the fold is spread over all warps as (unit, row slice)
+// tasks written to global memory and tagged, and a warp entering a unit
+// reads it back, folding locally only if the slices are late; the
+// selection runs in the next grid) and route_generic_kernel (any dtype,
+// grid (chunks of pages, Hkv, batch), fold once per CTA, the last CTA of
+// each (sequence, KV head) runs the top-k).
 #pragma once
 
 #include "common.cuh"
