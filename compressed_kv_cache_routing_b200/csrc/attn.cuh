@@ -3,11 +3,14 @@
 // scores"); values stay rank-r latents Z, and the weighted latent is
 // expanded by B_v in the fused combine.
 //
-// Grid: (splits, Hkv, batch).  Split sp of a (sequence, KV head) handles
-// selected entries [sp*pps, min((sp+1)*pps, k_b)).  Each warp keeps an
-// online-softmax state (running max m in log2 units, sum l, latent
-// accumulator acc[r]) for the G query heads and writes it as one partial;
-// the last CTA of the unit merges all partials and applies B_v.
+// Two kernels.  attn_mma_kernel (bf16 pools, tensor cores; bf16 or int8
+// keys) is persistent over the flat list of selected-page stages and is
+// described above its definition.  attn_generic_kernel (any dtype or shape)
+// runs a grid (splits, Hkv, batch): split sp of a (sequence, KV head)
+// handles selected entries [sp*pps, min((sp+1)*pps, k_b)), keeps an online
+// softmax state (running max m in log2 units, sum l, latent accumulator
+// acc[r]) for the G query heads and writes it as one partial; the last CTA
+// of the unit merges all partials and applies B_v.
 #pragma once
 
 #include <cuda_fp16.h>
