@@ -140,9 +140,12 @@ namespace basiskv {
 
 // ---------------------------------------------------------------------------
 // Selection kernel: one CTA per (sequence, KV head) whose pages are routed.
-// The scores are staged once in shared memory (kTopkKeysMax of them), the
+// The scores are staged once in shared memory (up to keys_cap of them), the
 // radix passes and the page-ordered compaction run there; units with more
-// pages read the scores from L2 on every pass (block_topk).
+// pages read the scores from L2 on every pass (block_topk).  The passes stop
+// once the bucket holding the k-th key is taken whole: every key above the
+// leading bits fixed so far and every key of the bucket is selected, so the
+// compaction compares keys on those bits only and the set is the same.
 struct TopkArgs {
   const float* scores;     // [B][Hkv][ld_pt]
   const int32_t* seq_lens; // [B]
