@@ -23,14 +23,34 @@ Recipe (all five named workloads follow it; shapes in ``SPECS``):
 * q, Z and R are rounded to the storage dtype (round-to-nearest-even);
 * planted alignment (only when s > 0 and k < n_b): per (b, kvh), k pages are
   drawn without replacement, and in each one token t* uniformly among the
-  page's valid tokens; its residual row gets  R_t* += alpha * g,  where g is
-  the unit vector along  B_r . (sum of the group's stored queries)  and
-  alpha = (beta0 + delta) * G / |B_r . sum_h q_h|, delta ~ U(0.05, 0.5) and
-  beta0 = 20 * sqrt((1 + s/r) * mean_h |q_h|^2) -- twenty times the standard
-  deviation of one token's routing score under this distribution, far above
-  the largest unplanted score.  The planted row is re-rounded;
+  page's valid tokens, with delta ~ U(0.05, 0.5); its residual row moves
+  along a unit vector g,  R_t* += alpha * g,  and is re-rounded.  Two ways to
+  pick g and alpha:
+    - strong (no scorer given): g is the unit vector along
+      B_r . (sum of the group's stored queries) and
+      alpha = (beta0 + delta) * G / |B_r . sum_h q_h|, with
+      beta0 = 20 * sqrt((1 + s/r) * mean_h |q_h|^2), twenty times the
+      standard deviation of one token's routing score under this
+      distribution: the planted pages lead by a wide margin;
+    - near margin (``scorer`` given): the planted page is put just above
+      the best unplanted one, at tau + delta, tau being the largest page
+      score of the unit's unplanted pages.  The scores come from the caller's
+      ``scorer`` (this module computes none): ``page_scores(w)`` gives every
+      page's score in float64 from the stored values, and
+      ``token_scores(w, b, kvh, slot, tok, r_rows)`` the G per-head scores of
+      given tokens with their residual rows replaced by ``r_rows``.  A
+      token's scores are affine in its residual row, so their response to
+      each unit residual direction gives the gradient of each head's score;
+      g is the normalised sum of the heads' gradients and alpha the least
+      step that lifts the token's best head score to tau + delta.  After
+      rounding, the page scores are recomputed from the stored bits; every
+      planted page that is not at least 1e-2 above tau gets its delta
+      doubled and is planted again from its original row, until all are;
 * keys K = (Zs . W_zk + Rs . B_r + 0.05 * eps) * c from the *stored* Zs, Rs,
   rounded to the storage dtype (dense workload: K ~ N(0,1) independent of Z);
+  with the near-margin plant, K is first built from the unplanted residuals
+  and the planted rows' keys are rebuilt from their final residuals and the
+  same eps;
 * every token slot past L_b in a sequence's last page, and every unreferenced
   slot, holds JUNK (=100.0) in Z, R and K, so a missing mask changes results.
 
@@ -150,8 +170,10 @@ def _storage(dtype: str):
 
 
 def generate(spec: WorkloadSpec | str, device: str | torch.device = "cpu",
-             slot_chunk: int = 2048) -> Workload:
-    """Draw one workload following the recipe in the module docstring."""
+             slot_chunk: int = 2048, scorer=None) -> Workload:
+    """Draw one workload following the recipe in the module docstring.  With
+    ``scorer`` the planted pages sit just above the k-th boundary (the near
+    margin plant); without it they lead by a wide margin."""
     if isinstance(spec, str):
         spec = SPECS[spec]
     s = spec
@@ -198,6 +220,7 @@ def generate(spec: WorkloadSpec | str, device: str | torch.device = "cpu",
     c = torch.exp(s.outlier_sigma * randn(Hkv, d)) if s.outlier_sigma > 0 else torch.ones(Hkv, d, device=dev)
 
     planted = {}
+    rows = None  # the planted rows, one per planted page
     if not s.dense and rs > 0:
         qd = q.double().view(s.batch, Hkv, G, d)
         v = torch.einsum("ksd,bkd->bks", b_r.double(), qd.sum(2))          # [B][Hkv][s]
@@ -205,7 +228,7 @@ def generate(spec: WorkloadSpec | str, device: str | torch.device = "cpu",
         ghat = v / vnorm[..., None]
         sigma = torch.sqrt((1.0 + rs / r) * (qd * qd).sum(-1).mean(-1))      # [B][Hkv]
         beta0 = 20.0 * sigma
-        rows_slot, rows_kvh, rows_tok, rows_b, rows_alpha = [], [], [], [], []
+        rows = {k: [] for k in ("slot", "kvh", "tok", "b", "page", "delta", "alpha")}
         vnorm_h = vnorm.cpu().numpy()
         beta0_h = beta0.cpu().numpy()
         for b in range(s.batch):
@@ -220,24 +243,40 @@ def generate(spec: WorkloadSpec | str, device: str | torch.device = "cpu",
                     valid = min(P, int(lens[b]) - j * P)
                     t = int(rng.integers(0, valid))
                     delta = float(rng.uniform(0.05, 0.5))
-                    rows_slot.append(int(table[b, j]))
-                    rows_kvh.append(kvh)
-                    rows_tok.append(t)
-                    rows_b.append(b)
-                    rows_alpha.append((beta0_h[b, kvh] + delta) * G / vnorm_h[b, kvh])
-        if rows_slot:
-            si = torch.tensor(rows_slot, device=dev, dtype=torch.long)
-            ki = torch.tensor(rows_kvh, device=dev, dtype=torch.long)
-            ti = torch.tensor(rows_tok, device=dev, dtype=torch.long)
-            bi = torch.tensor(rows_b, device=dev, dtype=torch.long)
-            al = torch.tensor(rows_alpha, device=dev, dtype=torch.float64)
+                    rows["slot"].append(int(table[b, j]))
+                    rows["kvh"].append(kvh)
+                    rows["tok"].append(t)
+                    rows["b"].append(b)
+                    rows["page"].append(j)
+                    rows["delta"].append(delta)
+                    rows["alpha"].append((beta0_h[b, kvh] + delta) * G / vnorm_h[b, kvh])
+        rows = {k: np.asarray(v_) for k, v_ in rows.items()}
+        if not rows["slot"].size:
+            rows = None
+        elif scorer is None:
+            si = torch.as_tensor(rows["slot"], device=dev, dtype=torch.long)
+            ki = torch.as_tensor(rows["kvh"], device=dev, dtype=torch.long)
+            ti = torch.as_tensor(rows["tok"], device=dev, dtype=torch.long)
+            bi = torch.as_tensor(rows["b"], device=dev, dtype=torch.long)
+            al = torch.as_tensor(rows["alpha"], device=dev, dtype=torch.float64)
             add = al[:, None] * ghat[bi, ki]                                  # [n][s] f64
             rr[si, ki, ti] = (rr[si, ki, ti].double() + add).to(st)
 
+    margin = rows is not None and scorer is not None
+    eps_rows = None
+    if margin:
+        eps_rows = torch.empty((len(rows["slot"]), d), device=dev)
+        slots_t = torch.as_tensor(rows["slot"], device=dev, dtype=torch.long)
+        kvh_t = torch.as_tensor(rows["kvh"], device=dev, dtype=torch.long)
+        tok_t = torch.as_tensor(rows["tok"], device=dev, dtype=torch.long)
     k = torch.empty(num_slots, Hkv, P, d, device=dev, dtype=st)
     for s0 in range(0, num_slots, slot_chunk):
         s1 = min(num_slots, s0 + slot_chunk)
         eps = randn(s1 - s0, Hkv, P, d)
+        if margin:  # keep the noise of the rows the plant will rebuild
+            m = (slots_t >= s0) & (slots_t < s1)
+            if bool(m.any()):
+                eps_rows[m] = eps[slots_t[m] - s0, kvh_t[m], tok_t[m]]
         if s.dense:
             k[s0:s1] = eps.to(st)
             continue
@@ -264,9 +303,78 @@ def generate(spec: WorkloadSpec | str, device: str | torch.device = "cpu",
         rr[ui] = JUNK
         k[ui] = JUNK
 
-    return Workload(spec=s, seq_lens=lens, page_table=table, num_slots=num_slots, q=q,
-                    z_pool=z, r_pool=rr, k_pool=k, w_zk=w_zk.contiguous(),
-                    b_r=b_r.contiguous(), b_v=b_v.contiguous(), planted=planted)
+    w = Workload(spec=s, seq_lens=lens, page_table=table, num_slots=num_slots, q=q,
+                 z_pool=z, r_pool=rr, k_pool=k, w_zk=w_zk.contiguous(),
+                 b_r=b_r.contiguous(), b_v=b_v.contiguous(), planted=planted)
+    if margin:
+        _plant_near_margin(w, rows, eps_rows, c, scorer)
+    return w
+
+
+MARGIN = 1e-2        # the smallest gap allowed at the k boundary
+_MAX_PLANT_ROUNDS = 40
+
+
+def _plant_near_margin(w: Workload, rows: dict, eps_rows: torch.Tensor, c: torch.Tensor, scorer) -> None:
+    """Lift each planted page to tau + delta (module docstring, near-margin
+    plant).  The scores are the scorer's; this function only draws, rounds
+    and solves for the step length along the chosen direction."""
+    s = w.spec
+    dev = w.r_pool.device
+    st = w.r_pool.dtype
+    n = len(rows["slot"])
+    si = torch.as_tensor(rows["slot"], device=dev, dtype=torch.long)
+    ki = torch.as_tensor(rows["kvh"], device=dev, dtype=torch.long)
+    ti = torch.as_tensor(rows["tok"], device=dev, dtype=torch.long)
+    r0 = w.r_pool[si, ki, ti].double().cpu().numpy()                      # [n][s] stored, unplanted
+    bi, kv, pg = rows["b"], rows["kvh"], rows["page"]
+    scores = np.asarray(scorer.page_scores(w), dtype=np.float64)
+    tau = np.empty(n)
+    for (b, kvh), pages in w.planted.items():
+        nb = int(w.num_pages[b])
+        keep = np.ones(nb, bool)
+        keep[pages] = False
+        sel = (bi == b) & (kv == kvh)
+        tau[sel] = scores[b, kvh, :nb][keep].max()
+    args = (bi, kv, rows["slot"], rows["tok"])
+    u0 = np.asarray(scorer.token_scores(w, *args, r0), dtype=np.float64)   # [n][G]
+    grad = np.empty(u0.shape + (s.rank_s,))
+    for i in range(s.rank_s):
+        e = r0.copy()
+        e[:, i] += 1.0
+        grad[..., i] = np.asarray(scorer.token_scores(w, *args, e), dtype=np.float64) - u0
+    gsum = grad.sum(axis=1)
+    gdir = gsum / np.maximum(np.linalg.norm(gsum, axis=1, keepdims=True), 1e-300)
+    slope = np.einsum("ngs,ns->ng", grad, gdir)                          # [n][G]
+    delta = rows["delta"].astype(np.float64).copy()
+    todo = np.arange(n)
+    for _ in range(_MAX_PLANT_ROUNDS):
+        target = tau[todo] + delta[todo]
+        up = slope[todo] > 0
+        need = np.where(up, (target[:, None] - u0[todo]) / np.where(up, slope[todo], 1.0), np.inf)
+        alpha = np.where(u0[todo].max(axis=1) >= target, 0.0, np.maximum(need.min(axis=1), 0.0))
+        if not np.isfinite(alpha).all():
+            raise RuntimeError("a planted token's score cannot be raised along its residual")
+        idx = torch.as_tensor(todo, device=dev, dtype=torch.long)
+        r_new = torch.as_tensor(r0[todo] + alpha[:, None] * gdir[todo], device=dev).float().to(st)
+        w.r_pool[si[idx], ki[idx], ti[idx]] = r_new
+        # the planted rows' keys, from their final residual and the same noise
+        zf = w.z_pool[si[idx], ki[idx], ti[idx]].float()
+        kf = torch.empty((len(todo), s.head_dim), device=dev)
+        for h in range(s.num_kv_heads):
+            m = ki[idx] == h
+            if bool(m.any()):
+                kf[m] = zf[m] @ w.w_zk[h] + r_new[m].float() @ w.b_r[h]
+        kf += s.noise_std * eps_rows[idx]
+        kf *= c[ki[idx]]
+        w.k_pool[si[idx], ki[idx], ti[idx]] = kf.to(st)
+        scores = np.asarray(scorer.page_scores(w), dtype=np.float64)
+        short = scores[bi, kv, pg] - tau < MARGIN
+        if not short.any():
+            return
+        todo = np.nonzero(short)[0]
+        delta[todo] *= 2.0
+    raise RuntimeError("the near-margin plant did not reach the margin")
 
 
 def shrink(spec: WorkloadSpec | str, batch: int | None = None, len_lo: int | None = None,

@@ -180,3 +180,19 @@ def test_quantize_keys_rejected_without_int8_pool():
     with pytest.raises(bk.BasisKVError):
         bk.basiskv_quantize_keys(kv.handle, w.k_pool)
     kv.close()
+
+
+@pytest.mark.parametrize("name", ["llama3_8b_decode", "long_context", "high_concurrency", "gqa8", "head_dim64"])
+def test_decode_parity_near_margin(name):
+    """int8 keys on inputs whose planted pages sit just above the k-th
+    boundary (routing reads no keys, so the selection margin is the same)."""
+    from margin import OracleScorer
+    w = W.generate(SMALL[name], device="cuda", scorer=OracleScorer())
+    kv, codes, scales = int8_handle(w)
+    prob = oracle_int8(w)
+    ref_out, ref_sel, _, gap = oracle.decode(prob)
+    assert min(gap[b, h] for (b, h) in w.planted) >= W.MARGIN
+    out, sel = decode_int8(kv, w)
+    assert np.array_equal(sel, ref_sel), name
+    assert out_error(out, ref_out) <= OUT_TOL
+    kv.close()

@@ -423,3 +423,61 @@ def test_append_page_copy_refused_copies_nothing():
     assert torch.count_nonzero(z2[2]) == 0 and torch.count_nonzero(k2[2]) == 0
     assert torch.equal(z2[1, :, :5], zs) and torch.count_nonzero(z2[1, :, 5:]) == 0
     kv.close()
+
+
+# ---- near the selection margin ---------------------------------------------
+# The planted pages sit just above the best unplanted page (gap >= 1e-2 in
+# float64 on the stored bits, typically 0.05), the regime where a routing
+# score error could move a page across the k-th boundary.
+NEAR = ["tiny", "llama3_8b_decode", "long_context", "high_concurrency", "generic_bf16", "gqa8", "gqa2",
+        "gqa1", "head_dim64", "fp32_llama_shape"]
+
+
+def _near(spec):
+    from margin import OracleScorer
+    return W.generate(spec, device="cuda", scorer=OracleScorer())
+
+
+def _check_margin(w, gap):
+    n = w.num_pages
+    gaps = [gap[b, h] for (b, h) in w.planted]
+    assert gaps and min(gaps) >= W.MARGIN and max(gaps) <= 1.0, (min(gaps), max(gaps))
+    return min(gaps)
+
+
+@pytest.mark.parametrize("name", NEAR)
+def test_small_parity_near_margin(name):
+    w = _near(SMALL[name])
+    prob = to_problem(w)
+    ref_out, ref_sel, _, gap = oracle.decode(prob)
+    g = _check_margin(w, gap)
+    out, sel = gpu_decode(w)
+    assert np.array_equal(sel, ref_sel), name
+    err = out_error(out, ref_out)
+    print(f"{name}: smallest gap {g:.4f}, max row rel err {err:.3e}")
+    assert err <= OUT_TOL
+
+
+@pytest.mark.parametrize("name", ["llama3_8b_decode", "long_context", "high_concurrency"])
+def test_full_size_near_margin(name):
+    """Full workload sizes, in the benchmark's launch configuration, with the
+    planted pages just above the boundary: the selection of EVERY unit equals
+    the oracle's (which equals the planted set), every routed unit's gap lies
+    in [1e-2, 1], and sampled units' outputs match the oracle."""
+    w = _near(W.SPECS[name])
+    out, sel = gpu_decode(w)
+    s = w.spec
+    prob = to_problem(w)
+    _, ref_sel_all, gap_all = oracle.route(prob)
+    g = _check_margin(w, gap_all)
+    assert np.array_equal(sel, ref_sel_all), name
+    for (b, kvh), pages in w.planted.items():
+        assert np.array_equal(sel[b, kvh][sel[b, kvh] >= 0], pages), (name, b, kvh)
+    U = s.batch * s.num_kv_heads
+    rng = np.random.default_rng(321)
+    units = sorted(set([0, U - 1] + rng.choice(U, size=min(U, 4), replace=False).tolist()))
+    ref_out, ref_sel, _, _ = oracle.decode(prob, units=units)
+    err = out_error(out, ref_out, unit_rows(w, units))
+    print(f"{name}: smallest gap {g:.4f} over {len(w.planted)} units; sampled units {units}: "
+          f"max row rel err {err:.3e}")
+    assert err <= OUT_TOL

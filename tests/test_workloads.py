@@ -74,3 +74,50 @@ def test_algorithmic_bytes_llama_formula():
     s = w.spec
     per_unit = 2 * 4096 * (32 + 16) + 2 * 16 * 64 * (128 + 32)
     assert w.algorithmic_bytes()["total"] == per_unit * s.batch * s.num_kv_heads
+
+
+@pytest.mark.parametrize("name", ["tiny", "llama3_8b_decode", "long_context", "high_concurrency"])
+def test_near_margin_plant(name):
+    """The near-margin plant puts the planted pages just above the k-th
+    boundary: they are exactly the oracle's selection and every routed unit's
+    float64 gap lies in [1e-2, 1] (delta ~ U(0.05, 0.5), doubled only where
+    rounding left a page short)."""
+    from margin import OracleScorer
+    w = W.generate(SMALL[name], scorer=OracleScorer())
+    prob = to_problem(w)
+    _, sel, gap = oracle.route(prob)
+    n = w.num_pages
+    gaps = []
+    for b in range(w.spec.batch):
+        for kvh in range(w.spec.num_kv_heads):
+            if min(w.spec.topk, n[b]) < n[b]:
+                got = sel[b, kvh][sel[b, kvh] >= 0]
+                assert np.array_equal(got, w.planted[(b, kvh)])
+                gaps.append(gap[b, kvh])
+    assert gaps and min(gaps) >= W.MARGIN and max(gaps) <= 1.0
+    # the strong plant's margin is far wider on the same draws
+    _, _, gap_strong = oracle.route(to_problem(W.generate(SMALL[name])))
+    assert np.nanmin(gap_strong[np.isfinite(gap_strong)]) > 5 * max(gaps)
+
+
+def test_near_margin_plant_only_moves_planted_rows():
+    """Both plants draw the same lengths, tables, bases, queries and latents;
+    the residuals and keys differ only in the planted rows."""
+    from margin import OracleScorer
+    spec = SMALL["llama3_8b_decode"]
+    a = W.generate(spec)
+    b = W.generate(spec, scorer=OracleScorer())
+    for f in ("q", "z_pool", "w_zk", "b_r", "b_v"):
+        assert torch.equal(getattr(a, f), getattr(b, f)), f
+    assert np.array_equal(a.page_table, b.page_table)
+    diff_r = (a.r_pool != b.r_pool).any(-1)
+    diff_k = (a.k_pool != b.k_pool).any(-1)
+    planted_rows = torch.zeros_like(diff_r)
+    P = spec.page_size
+    for (bb, kvh), pages in b.planted.items():
+        for j in pages.tolist():
+            slot = int(b.page_table[bb, j])
+            planted_rows[slot, kvh] |= diff_r[slot, kvh]
+    assert not (diff_r & ~planted_rows).any()
+    assert int(diff_r.sum()) == sum(len(p) for p in b.planted.values())
+    assert not (diff_k & ~diff_r).any()
