@@ -26,6 +26,8 @@ BASISKV_ERR_STATE = -6
 BASISKV_STATUS_BAD_SLOT = 1
 BASISKV_STATUS_TIMEOUT = 2
 BASISKV_STATUS_BAD_PAGE = 4
+BASISKV_STATUS_PART_OVERFLOW = 8
+BASISKV_STATUS_BAD_LENGTH = 16
 
 BASISKV_DTYPE_BF16 = 0
 BASISKV_DTYPE_F32 = 1
@@ -41,6 +43,7 @@ EXPORTED = (
     "basiskv_profile_end", "basiskv_last_launch", "basiskv_last_error", "basiskv_version",
     "basiskv_decode_attn_noalloc", "basiskv_decode_attn_latent", "basiskv_encode_rows",
     "basiskv_quantize_keys", "basiskv_encode_tokens", "basiskv_append_page_copy",
+    "basiskv_noalloc_status",
 )
 
 
@@ -100,6 +103,7 @@ def load(path: str = LIB_PATH):
         "basiskv_version": [],
         "basiskv_decode_attn_noalloc": [ctypes.POINTER(basiskv_params), i32, vp, vp, vp, i32, f32, vp,
                                         vp, vp],
+        "basiskv_noalloc_status": [ctypes.POINTER(ctypes.c_uint32)],
     }
     for name, args in sigs.items():
         f = getattr(lib, name)
@@ -248,10 +252,26 @@ def basiskv_decode_attn_noalloc(params, page_table, seq_lens, q, topk, softmax_s
     for callers that may not allocate device memory.  ``page_table`` and
     ``seq_lens`` are device int32 tensors; the library's fixed scratch array
     is shared by all calls, so calls must not overlap on the GPU."""
-    _check(load().basiskv_decode_attn_noalloc(ctypes.byref(params), int(seq_lens.shape[0]),
+    import torch
+    batch = int(seq_lens.shape[0])
+    if seq_lens.dtype != torch.int32 or seq_lens.dim() != 1 or not seq_lens.is_contiguous():
+        raise ValueError("seq_lens must be a contiguous int32 vector [batch]")
+    if (page_table.dtype != torch.int32 or not page_table.is_contiguous()
+            or tuple(page_table.shape) != (batch, params.max_pages_per_seq)):
+        raise ValueError(f"page_table must be contiguous int32 [{batch}][{params.max_pages_per_seq}]"
+                         " (the row length is params.max_pages_per_seq)")
+    _check(load().basiskv_decode_attn_noalloc(ctypes.byref(params), batch,
                                               _ptr(page_table), _ptr(seq_lens), _ptr(q), topk,
                                               float(softmax_scale), _ptr(out), _ptr(sel_out),
                                               _stream(stream)))
+
+
+def basiskv_noalloc_status() -> int:
+    """Status bits of the last allocation-free call on the current device
+    (synchronises the device)."""
+    st = ctypes.c_uint32()
+    _check(load().basiskv_noalloc_status(ctypes.byref(st)))
+    return st.value
 
 
 def basiskv_version() -> int:

@@ -93,6 +93,13 @@ __device__ __forceinline__ AttnUnit attn_unit(const AttnArgs& a) {
   au.u = au.b * a.num_kv_heads + au.kvh;
   au.L = a.seq_lens[au.b];
   au.n = (au.L + a.page_size - 1) / a.page_size;
+  if (au.n > a.ld_pt || au.L < 0) {
+    // a length the page-table row cannot hold (only callers that pass
+    // device lengths unchecked can get here): clamp to the row
+    if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(a.status, kStatusBadLength);
+    au.L = au.L < 0 ? 0 : a.ld_pt * a.page_size;
+    au.n = au.L / a.page_size;
+  }
   au.routed = a.topk < au.n;
   au.kb = au.routed ? a.topk : au.n;
   au.j0 = blockIdx.x * a.pages_per_split;
@@ -336,6 +343,10 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
     tok0s[warp][i % S] = page * P + ic.ts * TPS;
     uint64_t* bar = &bars[warp][i % S];
     uint8_t* dst = ring + (size_t)(i % S) * stage_bytes;
+    if (skip_issue_for_test(wg, i)) {
+      ic.advance(a, sub);
+      return;
+    }
     mbar_arrive_expect_tx(bar, stage_bytes);
     bulk_load(dst, kpool + row0 * D * KB, kbytes, bar, pol);
     bulk_load(dst + kbytes, zpool + row0 * RR, zbytes, bar, pol);
@@ -407,7 +418,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
         }
       }
     } else if (lane == 0) {
-      atomicOr(a.status, kStatusTimeout);  // more partials than slots: result invalid
+      atomicOr(a.status, kStatusPartOverflow);  // more partials than slots: result invalid
     }
     __syncwarp();
     int last = 0;

@@ -70,10 +70,14 @@ const std::map<RouteKey, KernelFn>& route_table() {
   static const std::map<RouteKey, KernelFn> t = {
 #define RK(G, R, S, P) {RouteKey{G, R, S, P}, &route_mma_kernel<G, R, S, P>}
 #define RK2(G, R, S) RK(G, R, S, 32), RK(G, R, S, 64)
+#ifdef BASISKV_WAIT_TEST
+      RK(4, 32, 16, 64),  // the wait-expiry test build holds one shape
+#else
       RK2(4, 16, 8),  RK2(4, 24, 8),  RK2(4, 32, 8),  RK2(4, 32, 16), RK2(4, 64, 16),
       RK2(4, 64, 32), RK2(4, 128, 0), RK2(4, 32, 0),  RK2(8, 32, 16), RK2(8, 24, 8),
       RK2(8, 64, 32), RK2(2, 32, 16), RK2(1, 32, 16), RK(4, 32, 16, 16), RK(4, 32, 16, 128),
       RK(4, 24, 8, 16),
+#endif
 #undef RK2
 #undef RK
   };
@@ -84,6 +88,9 @@ const std::map<AttnKey, AttnFn>& attn_table() {
   static const std::map<AttnKey, AttnFn> t = {
 #define AK(G, D, R, T) {AttnKey{G, D, R, T, false}, &attn_mma_kernel<G, D, R, T, false>}
 #define AK8(G, D, R, T) {AttnKey{G, D, R, T, true}, &attn_mma_kernel<G, D, R, T, true>}
+#ifdef BASISKV_WAIT_TEST
+      AK(4, 128, 32, 32), AK(4, 128, 32, 64),
+#else
       AK(4, 128, 32, 64), AK(4, 128, 32, 32), AK(4, 128, 24, 32), AK(4, 128, 24, 16),
       AK(4, 128, 16, 64), AK(4, 128, 64, 32), AK(4, 128, 128, 32), AK(4, 128, 128, 16),
       AK(4, 64, 16, 16),  AK(4, 64, 32, 32),  AK(8, 128, 32, 64), AK(8, 128, 32, 32),
@@ -91,6 +98,7 @@ const std::map<AttnKey, AttnFn>& attn_table() {
       AK8(4, 128, 32, 64), AK8(4, 128, 32, 32), AK8(4, 128, 24, 32), AK8(4, 128, 24, 16),
       AK8(4, 128, 128, 32), AK8(4, 128, 128, 16), AK8(4, 64, 16, 16), AK8(4, 64, 32, 32),
       AK8(8, 128, 32, 32), AK8(1, 128, 32, 64),
+#endif
 #undef AK8
 #undef AK
   };
@@ -1072,7 +1080,12 @@ int basiskv_get_status(basiskv_handle* h, uint32_t* status, int clear) {
   if (!status) return fail(BASISKV_ERR_INVALID_ARG, "status is NULL");
   CUDA_TRY(cudaDeviceSynchronize());
   CUDA_TRY(cudaMemcpy(status, h->d_status, sizeof(uint32_t), cudaMemcpyDeviceToHost));
-  if (clear) CUDA_TRY(cudaMemset(h->d_status, 0, sizeof(uint32_t)));
+  if (clear && *status) {
+    // a call that gave up part way can leave arrival counts behind: start
+    // the next call from zero
+    CUDA_TRY(cudaMemset(h->d_counters, 0, sizeof(uint32_t) * 3 * (size_t)h->p.max_batch * h->p.num_kv_heads));
+    CUDA_TRY(cudaMemset(h->d_status, 0, sizeof(uint32_t)));
+  }
   return BASISKV_OK;
 }
 
@@ -1135,6 +1148,10 @@ std::mutex g_noalloc_mutex;
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// The status word sits at the start of the array, where every call finds it
+// whatever its shapes.
+constexpr size_t kNoAllocStatusOffset = 0;
+
 // Device address of the scratch array on the current device.  The symbol's
 // host-side name is not a device address, so it is resolved here once per
 // device with cudaGetSymbolAddress.
@@ -1167,12 +1184,12 @@ extern "C" int basiskv_decode_attn_noalloc(const basiskv_params* p, int batch, c
   if (!std::isfinite(softmax_scale)) return fail(BASISKV_ERR_INVALID_ARG, "softmax_scale must be finite");
   if (batch == 0) return BASISKV_OK;
 
-  // scratch layout: counters | status | scores | selection | partial (m, l) | partial acc
+  // scratch layout: status | counters | scores | selection | partial (m, l) | partial acc
   const size_t U = (size_t)batch * p->num_kv_heads, G = p->gqa_group;
   const int splits = std::min(kMaxSplits, std::max(1, topk));
-  const size_t off_counters = 0;
-  const size_t off_status = align256(off_counters + sizeof(uint32_t) * 2 * U);
-  const size_t off_scores = align256(off_status + sizeof(uint32_t));
+  const size_t off_status = kNoAllocStatusOffset;
+  const size_t off_counters = align256(off_status + sizeof(uint32_t));
+  const size_t off_scores = align256(off_counters + sizeof(uint32_t) * 2 * U);
   const size_t off_sel = align256(off_scores + sizeof(float) * U * p->max_pages_per_seq);
   const size_t off_ml = align256(off_sel + sizeof(int32_t) * U * topk);
   const size_t off_acc = align256(off_ml + sizeof(float) * U * splits * G * 2);
@@ -1188,7 +1205,7 @@ extern "C" int basiskv_decode_attn_noalloc(const basiskv_params* p, int batch, c
   rc = noalloc_scratch(dev, reinterpret_cast<void**>(&scratch));
   if (rc) return rc;
   cudaStream_t st = (cudaStream_t)stream;
-  // the arrival counters and the status word must start at zero
+  // the status word and the arrival counters must start at zero
   CUDA_TRY(cudaMemsetAsync(scratch, 0, off_scores, st));
 
   // routing: a grid of (page chunk, KV head, sequence) sized by the table's
@@ -1278,5 +1295,17 @@ extern "C" int basiskv_decode_attn_noalloc(const basiskv_params* p, int batch, c
     attn_generic_kernel<float><<<agrid, kAttnThreads, asmem, st>>>(aa);
   }
   CUDA_TRY(cudaGetLastError());
+  return BASISKV_OK;
+}
+
+extern "C" int basiskv_noalloc_status(uint32_t* status) {
+  if (!status) return fail(BASISKV_ERR_INVALID_ARG, "status is NULL");
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  unsigned char* scratch = nullptr;
+  int rc = noalloc_scratch(dev, reinterpret_cast<void**>(&scratch));
+  if (rc) return rc;
+  CUDA_TRY(cudaDeviceSynchronize());
+  CUDA_TRY(cudaMemcpy(status, scratch + kNoAllocStatusOffset, sizeof(uint32_t), cudaMemcpyDeviceToHost));
   return BASISKV_OK;
 }

@@ -12,13 +12,25 @@ namespace basiskv {
 constexpr uint32_t kStatusBadSlot = 1u;
 constexpr uint32_t kStatusTimeout = 2u;
 constexpr uint32_t kStatusBadPage = 4u;
+constexpr uint32_t kStatusPartOverflow = 8u;  // a unit met more partials than it has slots
+constexpr uint32_t kStatusBadLength = 16u;    // a length needs more pages than a table row holds
 
 // Largest batch whose work plan travels in the kernel parameters; larger
 // batches read the plan the prep grid writes to global memory.
 constexpr int kPlanMax = 512;
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
+#ifdef BASISKV_WAIT_TEST
+// The wait-expiry test build: short waits, and the one copy that
+// skip_issue_for_test names is never issued, so its wait must run out.
+constexpr uint64_t kWaitLimitNs = 1000000ull;
+__device__ __forceinline__ bool skip_issue_for_test(int warp_in_grid, int item) {
+  return warp_in_grid == 0 && item == 1;
+}
+#else
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+__device__ __forceinline__ bool skip_issue_for_test(int, int) { return false; }
+#endif
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

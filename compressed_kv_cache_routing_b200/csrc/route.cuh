@@ -69,6 +69,13 @@ __device__ __forceinline__ RouteUnit route_unit(const RouteArgs& a) {
   ru.u = ru.b * a.num_kv_heads + ru.kvh;
   ru.L = a.seq_lens[ru.b];
   ru.n = (ru.L + a.page_size - 1) / a.page_size;
+  if (ru.n > a.ld_pt || ru.L < 0) {
+    // a length the page-table row cannot hold (only callers that pass
+    // device lengths unchecked can get here): clamp to the row
+    if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(a.status, kStatusBadLength);
+    ru.L = ru.L < 0 ? 0 : a.ld_pt * a.page_size;
+    ru.n = ru.L / a.page_size;
+  }
   ru.first = blockIdx.x * a.pages_per_cta;
   ru.last = min(ru.n, ru.first + a.pages_per_cta);
   ru.active = ru.first < ru.n && (a.force || a.topk < ru.n);
@@ -436,6 +443,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_c
     const size_t row0 = ((size_t)slot * a.num_kv_heads + ic.kvh) * P;
     uint64_t* bar = &bars[warp][i % S];
     uint8_t* dst = ring + (size_t)(i % S) * stage_bytes;
+    if (skip_issue_for_test(wg, i)) {
+      ic.advance(a);
+      return;
+    }
     mbar_arrive_expect_tx(bar, stage_bytes);
     bulk_load(dst, zpool + row0 * RR, zbytes, bar, pol);
     if (RS > 0) bulk_load(dst + zbytes, rpool + row0 * RS, rbytes, bar, pol);

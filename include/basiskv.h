@@ -77,7 +77,13 @@ enum {
 enum {
     BASISKV_STATUS_BAD_SLOT = 1u,   /* a page-table entry outside [0, num_slots) */
     BASISKV_STATUS_TIMEOUT = 2u,    /* a bounded wait on a copy expired          */
-    BASISKV_STATUS_BAD_PAGE = 4u    /* a selected page outside [0, n_b)          */
+    BASISKV_STATUS_BAD_PAGE = 4u,   /* a selected page outside [0, n_b)          */
+    BASISKV_STATUS_PART_OVERFLOW = 8u, /* a unit met more split partials than its
+                                          slots; that unit's output is invalid  */
+    BASISKV_STATUS_BAD_LENGTH = 16u /* a sequence length needing more pages than
+                                       a page-table row holds (device lengths of
+                                       basiskv_decode_attn_noalloc only): the
+                                       sequence is cut to the row              */
 };
 
 enum { BASISKV_DTYPE_BF16 = 0, BASISKV_DTYPE_F32 = 1 };
@@ -268,7 +274,9 @@ BASISKV_API int basiskv_route(basiskv_handle *h, int batch, const void *q, int t
                   float *scores_out, int32_t *sel_out, basiskv_stream_t stream);
 
 /* Read (and optionally clear) the device status bits.  Synchronises the
- * device. */
+ * device.  Clearing a nonzero status also zeroes the handle's arrival
+ * counters, which a call that gave up part way (a wait that ran out) can
+ * leave behind, so the next call on the handle starts clean. */
 BASISKV_API int basiskv_get_status(basiskv_handle *h, uint32_t *status, int clear);
 
 /* Kernel timing: after basiskv_profile_begin(h, n), the next n decode calls
@@ -298,24 +306,37 @@ BASISKV_API int basiskv_last_launch(basiskv_handle *h, int info[6]);
  *   page_table  [batch][p->max_pages_per_seq] int32 (device), seq_lens
  *               [batch] int32 (device); q, topk, softmax_scale, out, sel_out
  *               as for basiskv_decode_attn
+ * The page table and lengths stay on the device, so they are checked there:
+ * a length needing more than p->max_pages_per_seq pages is cut to the row
+ * and sets BASISKV_STATUS_BAD_LENGTH; an entry outside [0, num_slots) reads
+ * slot 0 and sets BASISKV_STATUS_BAD_SLOT.  Those bits are read with
+ * basiskv_noalloc_status; nothing else reports them.
  * It allocates nothing.  Its scratch (page scores, selection, split
- * partials, arrival counters) lives in one 16 MiB __device__ array inside
- * the library, held by every GPU that loads the library until the process
- * exits.  A call whose scratch would exceed 16 MiB
- * (about batch * Hkv * (4 * max_pages_per_seq + 4 * topk + 32 * G * (r + 2))
- * bytes) is rejected with BASISKV_ERR_CAPACITY and a message naming the
- * size.  The first call on each device resolves the array's device address
- * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture.  Every call clears the counters it needs on
- * `stream`, then reuses the same array, which keeps the last call's
- * contents: calls that may overlap on the GPU (other streams, other host
- * threads) race on it and must be serialised by the caller.  It runs the
- * CUDA-core kernels, not the persistent tensor-core ones.  Errors:
- * INVALID_ARG, CAPACITY, CUDA, UNSUPPORTED. */
+ * partials, arrival counters, status word) lives in one 16 MiB __device__
+ * array inside the library, held by every GPU that loads the library until
+ * the process exits.  A call needs, rounded up to 256-byte pieces,
+ *   batch * Hkv * (8 + 4 * max_pages_per_seq + 4 * topk
+ *                  + 4 * min(16, topk) * G * (r + 2))  bytes,
+ * and one that would exceed 16 MiB is rejected with BASISKV_ERR_CAPACITY and
+ * a message naming the size.  The first call on each device resolves the
+ * array's device address (cudaGetSymbolAddress, with that device current);
+ * make that first call before any stream capture.  Every call clears the
+ * counters and status word it needs on `stream`, then reuses the same
+ * array, which keeps the last call's contents: calls that may overlap on the
+ * GPU (other streams, other host threads) race on it and must be serialised
+ * by the caller.  It runs the CUDA-core kernels, not the persistent
+ * tensor-core ones.  Errors: INVALID_ARG, CAPACITY, CUDA, UNSUPPORTED. */
 BASISKV_API int basiskv_decode_attn_noalloc(const basiskv_params *p, int batch,
                                             const int32_t *page_table, const int32_t *seq_lens,
                                             const void *q, int topk, float softmax_scale,
                                             float *out, int32_t *sel_out, basiskv_stream_t stream);
+
+/* Device status bits (BASISKV_STATUS_*) of the last basiskv_decode_attn_noalloc
+ * call on the current device, read from the library's scratch array without
+ * allocating.  Synchronises the device first.  The next call clears them.
+ * Before any call on this device *status is 0.  Errors: INVALID_ARG (NULL
+ * status), CUDA, UNSUPPORTED. */
+BASISKV_API int basiskv_noalloc_status(uint32_t *status);
 
 /* Thread-local message for the last non-zero return of this thread. */
 BASISKV_API const char *basiskv_last_error(void);
