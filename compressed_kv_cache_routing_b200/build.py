@@ -36,25 +36,46 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+# The wait-expiry test build: the same sources with BASISKV_WAIT_TEST, which
+# shortens every bounded wait to 1 ms and has one warp skip one copy, so a
+# test can watch a wait run out and the kernels return with a status (no
+# fault, no hang).  It holds only the Llama-3-8B decode shapes.
+WAIT_TEST_LIB = os.path.join(HERE, "libbasiskv_waittest.so")
+
+
+def _stale_lib(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + [HEADER, __file__]
     return any(os.path.getmtime(f) > t for f in deps)
+
+
+def _stale() -> bool:
+    return _stale_lib(LIB)
+
+
+def _compile(lib: str, extra: list[str], verbose: bool) -> str:
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-o", tmp, *sources()]
+    if verbose:
+        cmd.insert(1, "-Xptxas=-v")
+        print(" ".join(cmd))
+    subprocess.check_call(cmd)
+    os.replace(tmp, lib)
+    return lib
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not _stale():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, "-o", tmp, *sources()]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-        print(" ".join(cmd))
-    subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    return _compile(LIB, [], verbose)
+
+
+def build_wait_test(force: bool = False) -> str:
+    if not force and not _stale_lib(WAIT_TEST_LIB):
+        return WAIT_TEST_LIB
+    return _compile(WAIT_TEST_LIB, ["-DBASISKV_WAIT_TEST"], False)
 
 
 if __name__ == "__main__":
