@@ -47,6 +47,9 @@ def parse():
     ap.add_argument("--keys", choices=["native", "int8"], default="native",
                     help="int8: keys as int8 codes with a per-token scale")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the long-context, high-concurrency and dense-limit lines")
+    ap.add_argument("--per-workload-steps", type=int, default=300)
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     return ap.parse_args()
 
@@ -351,6 +354,86 @@ def aux_measurements(kv, w, stream, dev, int8_codes=None):
     return out
 
 
+def make_handle(w, int8, dev):
+    """A library handle over w's pools; with int8, the keys quantised on the
+    device into int8 codes and per-token scales first.  Returns (handle
+    object, codes or None)."""
+    import torch
+    from compressed_kv_cache_routing_b200 import basiskv as bk
+    if not int8:
+        return bk.BasisKV.for_workload(w), None
+    codes = torch.empty(tuple(w.k_pool.shape), dtype=torch.int8, device=dev)
+    k_scale = torch.empty(tuple(w.k_pool.shape[:3]), dtype=torch.float32, device=dev)
+    kv = bk.BasisKV(z_pool=w.z_pool, r_pool=w.r_pool, k_pool=codes, w_zk=w.w_zk, b_r=w.b_r, b_v=w.b_v,
+                    gqa_group=w.spec.gqa_group, max_batch=w.spec.batch,
+                    max_pages_per_seq=max(1, w.page_table.shape[1]), max_topk=w.spec.topk, k_scale=k_scale)
+    bk.basiskv_quantize_keys(kv.handle, w.k_pool)
+    bk.basiskv_load_page_table(kv.handle, np.where(w.page_table >= 0, w.page_table, 0), w.seq_lens)
+    torch.cuda.synchronize(dev)
+    return kv, codes
+
+
+def measure_workload(name, int8, dev, local, steps, warmup):
+    """Another workload in the same process and with the same protocol as the
+    main line (L2 flushed between steps, a CUDA event pair around each call,
+    clock samples during the timed loop, per-grid events in a second loop)."""
+    import torch
+    from compressed_kv_cache_routing_b200 import basiskv as bk
+    from compressed_kv_cache_routing_b200 import workloads as W
+    w = W.generate(name, device=dev)
+    kv, codes = make_handle(w, int8, dev)
+    s = w.spec
+    out = torch.empty((s.batch, s.num_q_heads, s.head_dim), device=dev, dtype=torch.float32)
+    sel = torch.empty((s.batch, s.num_kv_heads, s.topk), device=dev, dtype=torch.int32)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2 // 4 + 1, device=dev, dtype=torch.float32)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        bk.basiskv_decode_attn(kv.handle, w.q, s.topk, s.softmax_scale, out, sel, stream=stream)
+
+    for _ in range(max(3, warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        torch.cuda.synchronize(dev)
+        for k in range(steps):
+            flush.zero_()
+            starts[k].record(stream)
+            step()
+            ends[k].record(stream)
+        torch.cuda.synchronize(dev)
+    step_ms = np.array([a.elapsed_time(b) for a, b in zip(starts, ends)])
+    bk.basiskv_profile_begin(kv.handle, steps)
+    for _ in range(steps):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    prof = bk.basiskv_profile_end(kv.handle, steps)
+    status = bk.basiskv_get_status(kv.handle, clear=True)
+    launch = bk.basiskv_last_launch(kv.handle)
+    kv.close()
+    ms = float(np.mean(step_ms))
+    nbytes = w.algorithmic_bytes(int8)["total"]
+    hbm_peak, peak_kind = peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    res = {"ms_per_step": ms, "step_ms_p10_p50_p90": [float(np.percentile(step_ms, q)) for q in (10, 50, 90)],
+           "value": w.context_tokens / (ms * 1e-3), "unit": UNIT, "context_tokens": w.context_tokens,
+           "algorithmic_bytes": nbytes, "achieved_gbs": gbs, "frac_of_measured": gbs / hbm_peak,
+           "frac_of_8tbs": gbs / 8000.0, "peak_kind": peak_kind, "steps": steps,
+           "kernels_ms": {k: float(np.mean(v)) for k, v in prof.items()},
+           "launch": launch, "clocks": clk.summary(), "device_status": status,
+           "config": {"batch": s.batch, "page": s.page_size, "rank_r": s.rank_r, "rank_s": s.rank_s,
+                      "topk": s.topk, "keys": "int8" if int8 else s.dtype}}
+    del w, codes, out, sel, flush
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args, rank, world, local):
     import torch
     from compressed_kv_cache_routing_b200 import basiskv as bk
@@ -369,19 +452,7 @@ def run_ours(args, rank, world, local):
     spec = replica_spec(spec, rank)
     w = W.generate(spec, device=dev)
     int8 = args.keys == "int8"
-    codes = None
-    if int8:
-        # the keys as int8 codes and per-token scales, quantised on the device
-        codes = torch.empty(tuple(w.k_pool.shape), dtype=torch.int8, device=dev)
-        k_scale = torch.empty(tuple(w.k_pool.shape[:3]), dtype=torch.float32, device=dev)
-        kv = bk.BasisKV(z_pool=w.z_pool, r_pool=w.r_pool, k_pool=codes, w_zk=w.w_zk, b_r=w.b_r, b_v=w.b_v,
-                        gqa_group=w.spec.gqa_group, max_batch=w.spec.batch,
-                        max_pages_per_seq=max(1, w.page_table.shape[1]), max_topk=w.spec.topk, k_scale=k_scale)
-        bk.basiskv_quantize_keys(kv.handle, w.k_pool)
-        bk.basiskv_load_page_table(kv.handle, np.where(w.page_table >= 0, w.page_table, 0), w.seq_lens)
-        torch.cuda.synchronize(dev)
-    else:
-        kv = bk.BasisKV.for_workload(w)
+    kv, codes = make_handle(w, int8, dev)
     s = w.spec
     out = torch.empty((s.batch, s.num_q_heads, s.head_dim), device=dev, dtype=torch.float32)
     sel = torch.empty((s.batch, s.num_kv_heads, s.topk), device=dev, dtype=torch.int32)
@@ -470,6 +541,12 @@ def run_ours(args, rank, world, local):
     d2h = out_host.numel() * 4 + sel_host.numel() * 4
     aux = aux_measurements(kv, w, stream, dev, codes if int8 else None)
 
+    # the other workloads of the same family, same protocol (one GPU only)
+    per_workload = None
+    if world == 1 and not args.batch and not args.no_per_workload and args.workload == "llama3_8b_decode":
+        per_workload = {name: measure_workload(name, int8, dev, local, min(K, args.per_workload_steps), args.warmup)
+                        for name in ("long_context", "high_concurrency", "dense_limit")}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         prob = oracle_problem(w, int8)
@@ -505,6 +582,7 @@ def run_ours(args, rank, world, local):
             "device_status": status,
             "cpu_baseline": cpu,
             "aux": aux,
+            "per_workload": per_workload,
         }
         print(json.dumps(line), flush=True)
     kv.close()

@@ -24,7 +24,7 @@ namespace basiskv {
 // The same product with f16 operands (A and B both f16).
 __device__ __forceinline__ void mma_k16_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                             uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -152,6 +152,113 @@ __device__ __forceinline__ void attn_finish(const AttnArgs& a, const AttnUnit& a
   combine_unit<NT>(c, smem_f);
 }
 
+// One staged attention item of TPS tokens of one selected page: exact QK for
+// the group (heads as M, tokens as N, k permuted so each B fragment is one
+// 16-byte shared load), the online softmax in fp32 (log2 units) and the
+// latent sum P.Z with the probabilities split into bf16 hi (rows g) and lo
+// (rows g + 8).  `stage` holds the K rows (bf16, or int8 codes when K8),
+// then the Z rows, then (K8) the TPS fp32 token scales; tokens at or past
+// `valid` are masked.  qa: this lane's query fragments.
+template <int G, int D, int RR, int TPS, bool K8>
+__device__ __forceinline__ void attn_stage(const uint8_t* stage, int valid, const uint32_t (&qa)[D / 32][2][2],
+                                           float scale_log2, float& m_run, float& l_run, float (&acc)[RR / 8][4]) {
+  constexpr int DS = D / 32;
+  constexpr int RT = RR / 8;
+  constexpr int NTS = TPS / 8;
+  constexpr int KBS = TPS / 16;
+  constexpr int KB = K8 ? 1 : 2;
+  constexpr uint32_t kbytes = TPS * D * KB, zbytes = TPS * RR * 2;
+  (void)DS;
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int trow = (lane & 7) + 8 * ((lane >> 3) & 1);
+  const __nv_bfloat16* zs = reinterpret_cast<const __nv_bfloat16*>(stage + kbytes);
+
+  // exact QK for the group
+  float s[NTS][2];
+#pragma unroll
+  for (int nt = 0; nt < NTS; ++nt) {
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint8_t* krow = stage + (nt * 8 + g) * D * KB;
+    const int tok = nt * 8 + 2 * t;
+    if constexpr (K8) {
+#pragma unroll
+      for (int sp = 0; sp < D / 64; ++sp) {
+        const uint4 v = lds128(krow + 64 * sp + 16 * t);
+        uint32_t b0, b1;
+        codes_to_f16x2(v.x, b0, b1);
+        mma_k16_f16(d, qa[2 * sp][0][0], 0u, qa[2 * sp][0][1], 0u, b0, b1);
+        codes_to_f16x2(v.y, b0, b1);
+        mma_k16_f16(d, qa[2 * sp][1][0], 0u, qa[2 * sp][1][1], 0u, b0, b1);
+        codes_to_f16x2(v.z, b0, b1);
+        mma_k16_f16(d, qa[2 * sp + 1][0][0], 0u, qa[2 * sp + 1][0][1], 0u, b0, b1);
+        codes_to_f16x2(v.w, b0, b1);
+        mma_k16_f16(d, qa[2 * sp + 1][1][0], 0u, qa[2 * sp + 1][1][1], 0u, b0, b1);
+      }
+      const uint2 sc = lds64(stage + kbytes + zbytes + 4 * tok);
+      d[0] *= __uint_as_float(sc.x);
+      d[1] *= __uint_as_float(sc.y);
+    } else {
+#pragma unroll
+      for (int sp = 0; sp < D / 32; ++sp) {
+        const uint4 v = lds128(krow + 2 * (32 * sp + 8 * t));
+        mma_k16(d, qa[sp][0][0], 0u, qa[sp][0][1], 0u, v.x, v.y);
+        mma_k16(d, qa[sp][1][0], 0u, qa[sp][1][1], 0u, v.z, v.w);
+      }
+    }
+    s[nt][0] = tok < valid ? d[0] * scale_log2 : -INFINITY;
+    s[nt][1] = tok + 1 < valid ? d[1] * scale_log2 : -INFINITY;
+  }
+  // online softmax for head g (the quad 4g..4g+3 shares the row)
+  float mloc = -INFINITY;
+#pragma unroll
+  for (int nt = 0; nt < NTS; ++nt) mloc = fmaxf(mloc, fmaxf(s[nt][0], s[nt][1]));
+  mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
+  mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
+  const float m_new = fmaxf(m_run, mloc);
+  const float corr = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
+  const float base = (m_new == -INFINITY) ? 0.f : m_new;
+  float lsum = 0.f;
+#pragma unroll
+  for (int nt = 0; nt < NTS; ++nt) {
+    s[nt][0] = exp2f(s[nt][0] - base);
+    s[nt][1] = exp2f(s[nt][1] - base);
+    lsum += s[nt][0] + s[nt][1];
+  }
+  l_run = l_run * corr + lsum;
+  m_run = m_new;
+#pragma unroll
+  for (int c = 0; c < RT; ++c) {
+    acc[c][0] *= corr;
+    acc[c][1] *= corr;
+    acc[c][2] *= corr;
+    acc[c][3] *= corr;
+  }
+  // latent sum P.Z
+#pragma unroll
+  for (int kb = 0; kb < KBS; ++kb) {
+    float h0, l0, h1, l1, h2, l2, h3, l3;
+    split_bf16(s[2 * kb][0], h0, l0);
+    split_bf16(s[2 * kb][1], h1, l1);
+    split_bf16(s[2 * kb + 1][0], h2, l2);
+    split_bf16(s[2 * kb + 1][1], h3, l3);
+    const uint32_t a0 = pack_bf16(h0, h1), a1 = pack_bf16(l0, l1);
+    const uint32_t a2 = pack_bf16(h2, h3), a3 = pack_bf16(l2, l3);
+    const __nv_bfloat16* zrow = zs + (kb * 16 + trow) * RR + 8 * (lane >> 4);
+#pragma unroll
+    for (int c2 = 0; c2 < RT / 2; ++c2) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_trans(b0, b1, b2, b3, zrow + 16 * c2);
+      mma_k16(acc[2 * c2], a0, a1, a2, a3, b0, b1);
+      mma_k16(acc[2 * c2 + 1], a0, a1, a2, a3, b2, b3);
+    }
+    if (RT & 1) {
+      uint32_t b0, b1;
+      ldsm_x2_trans(b0, b1, zs + (kb * 16 + trow) * RR + 8 * (RT - 1));
+      mma_k16(acc[RT - 1], a0, a1, a2, a3, b0, b1);
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Tensor-core attention for bf16 pools, persistent over the flat list of
 // attention items (sequence-major, then KV head, selected entry, stage of
@@ -239,8 +346,6 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
   static_assert(!K8 || D % 64 == 0, "int8 keys need d % 64 == 0");
   constexpr int DS = D / 32;     // 32-wide spans of the head dim
   constexpr int RT = RR / 8;     // n8 tiles of the latent
-  constexpr int NTS = TPS / 8;   // n8 token tiles per stage
-  constexpr int KBS = TPS / 16;  // k16 token blocks per stage
   constexpr int KB = K8 ? 1 : 2; // bytes per key element
   constexpr uint32_t kbytes = TPS * D * KB, zbytes = TPS * RR * 2, sbytes = K8 ? TPS * 4 : 0;
   constexpr uint32_t stage_bytes = kbytes + zbytes + sbytes;
@@ -330,19 +435,19 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
   const uint8_t* kpool = static_cast<const uint8_t*>(a.k_pool);
   const __nv_bfloat16* zpool = static_cast<const __nv_bfloat16*>(a.z_pool);
   const uint64_t pol = policy_evict_first();
-  // lane 0 issues item i of this warp into stage i % S; the selection and
+  // lane 0 issues item i of this warp into ring position s = i mod S; the selection and
   // page-table reads for an item are made one iteration before its issue so
   // they overlap the arithmetic of the current stage
   auto slot_of = [&](int page) { return __ldg(a.page_table + (size_t)ic.b * a.ld_pt + page); };
-  auto issue = [&](int i, int page, int slot) {
+  auto issue = [&](int i, int s, int page, int slot) {
     if (slot < 0 || slot >= a.num_slots) {
       atomicOr(a.status, kStatusBadSlot);
       slot = 0;
     }
     const size_t row0 = ((size_t)slot * a.num_kv_heads + ic.kvh) * P + (size_t)ic.ts * TPS;
-    tok0s[warp][i % S] = page * P + ic.ts * TPS;
-    uint64_t* bar = &bars[warp][i % S];
-    uint8_t* dst = ring + (size_t)(i % S) * stage_bytes;
+    tok0s[warp][s] = page * P + ic.ts * TPS;
+    uint64_t* bar = &bars[warp][s];
+    uint8_t* dst = ring + (size_t)s * stage_bytes;
     if (skip_issue_for_test(wg, i)) {
       ic.advance(a, sub);
       return;
@@ -368,7 +473,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
     }
     for (int i = 0; i < first; ++i) {
       const int pgi = __shfl_sync(0xffffffffu, pg, i), sli = __shfl_sync(0xffffffffu, sl, i);
-      if (lane == 0) issue(i, pgi, sli);
+      if (lane == 0) issue(i, i, pgi, sli);
     }
   }
   if (lane == 0) {
@@ -441,7 +546,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
 
   bool ok = true;
   int i = 0;
-  const int trow = (lane & 7) + 8 * ((lane >> 3) & 1);
+  int s_i = 0;        // ring position of item i (i mod S)
+  uint32_t ph_i = 0;  // phase parity of that position's barrier for item i
   for (; i < count; ++i) {
     int next_slot = 0, page_after = 0;
     if (lane == 0) {
@@ -459,106 +565,24 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
       for (int c = 0; c < RT; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.f;
       load_q(u);
     }
-    ok = mbar_wait(&bars[warp][i % S], (uint32_t)((i / S) & 1), a.status);
+    ok = mbar_wait(&bars[warp][s_i], ph_i, a.status);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;
-    const int valid = cc.L - tok0s[warp][i % S];  // tokens of this stage inside the sequence
-    const uint8_t* stage = ring + (size_t)(i % S) * stage_bytes;
-    const __nv_bfloat16* zs = reinterpret_cast<const __nv_bfloat16*>(stage + kbytes);
-
-    // exact QK for the group
-    float s[NTS][2];
-#pragma unroll
-    for (int nt = 0; nt < NTS; ++nt) {
-      float d[4] = {0.f, 0.f, 0.f, 0.f};
-      const uint8_t* krow = stage + (nt * 8 + g) * D * KB;
-      const int tok = nt * 8 + 2 * t;
-      if constexpr (K8) {
-#pragma unroll
-        for (int sp = 0; sp < D / 64; ++sp) {
-          const uint4 v = lds128(krow + 64 * sp + 16 * t);
-          uint32_t b0, b1;
-          codes_to_f16x2(v.x, b0, b1);
-          mma_k16_f16(d, qa[2 * sp][0][0], 0u, qa[2 * sp][0][1], 0u, b0, b1);
-          codes_to_f16x2(v.y, b0, b1);
-          mma_k16_f16(d, qa[2 * sp][1][0], 0u, qa[2 * sp][1][1], 0u, b0, b1);
-          codes_to_f16x2(v.z, b0, b1);
-          mma_k16_f16(d, qa[2 * sp + 1][0][0], 0u, qa[2 * sp + 1][0][1], 0u, b0, b1);
-          codes_to_f16x2(v.w, b0, b1);
-          mma_k16_f16(d, qa[2 * sp + 1][1][0], 0u, qa[2 * sp + 1][1][1], 0u, b0, b1);
-        }
-        const uint2 sc = lds64(stage + kbytes + zbytes + 4 * tok);
-        d[0] *= __uint_as_float(sc.x);
-        d[1] *= __uint_as_float(sc.y);
-      } else {
-#pragma unroll
-        for (int sp = 0; sp < DS; ++sp) {
-          const uint4 v = lds128(krow + 2 * (32 * sp + 8 * t));
-          mma_k16(d, qa[sp][0][0], 0u, qa[sp][0][1], 0u, v.x, v.y);
-          mma_k16(d, qa[sp][1][0], 0u, qa[sp][1][1], 0u, v.z, v.w);
-        }
-      }
-      s[nt][0] = tok < valid ? d[0] * a.scale_log2 : -INFINITY;
-      s[nt][1] = tok + 1 < valid ? d[1] * a.scale_log2 : -INFINITY;
-    }
-    // online softmax for head g (the quad 4g..4g+3 shares the row)
-    float mloc = -INFINITY;
-#pragma unroll
-    for (int nt = 0; nt < NTS; ++nt) mloc = fmaxf(mloc, fmaxf(s[nt][0], s[nt][1]));
-    mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
-    mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
-    const float m_new = fmaxf(m_run, mloc);
-    const float corr = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
-    const float base = (m_new == -INFINITY) ? 0.f : m_new;
-    float lsum = 0.f;
-#pragma unroll
-    for (int nt = 0; nt < NTS; ++nt) {
-      s[nt][0] = exp2f(s[nt][0] - base);
-      s[nt][1] = exp2f(s[nt][1] - base);
-      lsum += s[nt][0] + s[nt][1];
-    }
-    l_run = l_run * corr + lsum;
-    m_run = m_new;
-#pragma unroll
-    for (int c = 0; c < RT; ++c) {
-      acc[c][0] *= corr;
-      acc[c][1] *= corr;
-      acc[c][2] *= corr;
-      acc[c][3] *= corr;
-    }
-    // latent sum P.Z
-#pragma unroll
-    for (int kb = 0; kb < KBS; ++kb) {
-      float h0, l0, h1, l1, h2, l2, h3, l3;
-      split_bf16(s[2 * kb][0], h0, l0);
-      split_bf16(s[2 * kb][1], h1, l1);
-      split_bf16(s[2 * kb + 1][0], h2, l2);
-      split_bf16(s[2 * kb + 1][1], h3, l3);
-      const uint32_t a0 = pack_bf16(h0, h1), a1 = pack_bf16(l0, l1);
-      const uint32_t a2 = pack_bf16(h2, h3), a3 = pack_bf16(l2, l3);
-      const __nv_bfloat16* zrow = zs + (kb * 16 + trow) * RR + 8 * (lane >> 4);
-#pragma unroll
-      for (int c2 = 0; c2 < RT / 2; ++c2) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_trans(b0, b1, b2, b3, zrow + 16 * c2);
-        mma_k16(acc[2 * c2], a0, a1, a2, a3, b0, b1);
-        mma_k16(acc[2 * c2 + 1], a0, a1, a2, a3, b2, b3);
-      }
-      if (RT & 1) {
-        uint32_t b0, b1;
-        ldsm_x2_trans(b0, b1, zs + (kb * 16 + trow) * RR + 8 * (RT - 1));
-        mma_k16(acc[RT - 1], a0, a1, a2, a3, b0, b1);
-      }
-    }
+    const int valid = cc.L - tok0s[warp][s_i];  // tokens of this stage inside the sequence
+    attn_stage<G, D, RR, TPS, K8>(ring + (size_t)s_i * stage_bytes, valid, qa, a.scale_log2, m_run, l_run, acc);
     ++seg;
     __syncwarp();
     if (lane == 0 && i + S < count) {
-      issue(i + S, next_page, next_slot);
+      issue(i + S, s_i, next_page, next_slot);  // (i + S) mod S = i mod S
       next_page = page_after;
       ia.advance(a, sub);
     }
     prev = cc;
     cc.advance(a, sub);
+    if (++s_i == S) {
+      s_i = 0;
+      ph_i ^= 1u;
+    }
   }
   if (!ok) {
     if (lane == 0)

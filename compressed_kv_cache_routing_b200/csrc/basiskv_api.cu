@@ -244,7 +244,8 @@ void choose_kernels(basiskv_handle* h) {
   const size_t es = 2;
   auto rit = route_table().find(RouteKey{p.gqa_group, p.rank_r, p.rank_s, p.page_size});
   if (rit != route_table().end() && p.page_size % 16 == 0 && (p.head_dim == 128 || p.head_dim == 64)) {
-    const size_t stage = (size_t)p.page_size * (p.rank_r + p.rank_s) * es;
+    const size_t stage = (size_t)route_pages_per_stage(p.page_size, p.rank_r, p.rank_s) * p.page_size *
+                         (p.rank_r + p.rank_s) * es;
     int st = (int)std::min<size_t>(4, kRouteSmemBudget / (kRouteWarps * stage));
     if (st >= 2) {
       h->route_fn = rit->second;

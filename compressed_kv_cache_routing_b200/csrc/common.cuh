@@ -171,10 +171,13 @@ __device__ __forceinline__ void ldsm_x2_trans(uint32_t& r0, uint32_t& r1, const 
 }
 
 // ---- bf16 tensor-core MMA, fp32 accumulate ----------------------------------
+// Register-only operations, so not volatile: the compiler may interleave
+// independent accumulator chains.  The shared-memory loads that feed them
+// stay volatile, in program order after the barrier waits.
 // D(16x8) += A(16x16, row) * B(16x8, col)
 __device__ __forceinline__ void mma_k16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -182,7 +185,7 @@ __device__ __forceinline__ void mma_k16(float (&d)[4], uint32_t a0, uint32_t a1,
 }
 // D(16x8) += A(16x8, row) * B(8x8, col)
 __device__ __forceinline__ void mma_k8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])

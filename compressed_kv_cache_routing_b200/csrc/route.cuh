@@ -57,6 +57,14 @@ constexpr int kRouteThreads = 128;
 constexpr int kRouteWarps = kRouteThreads / 32;
 constexpr int kMaxStages = 8;
 
+// Pages staged together by route_mma_kernel: about 6 KB per stage, so small
+// pages (P = 32 with narrow ranks) share one barrier wait and one issue.
+constexpr int route_pages_per_stage(int page_size, int rank_r, int rank_s) {
+  const int page_bytes = page_size * (rank_r + rank_s) * 2;
+  const int rps = page_bytes > 0 ? 6144 / page_bytes : 1;
+  return rps < 1 ? 1 : (rps > 4 ? 4 : rps);
+}
+
 struct RouteUnit {
   int b, kvh, u, L, n, first, last;  // pages [first, last) of this CTA
   bool active;
@@ -156,6 +164,76 @@ template <int W32, int W16>
 __device__ __forceinline__ int k16_phys(int blk, int t, int half) {
   if (blk < 2 * W32) return 32 * (blk >> 1) + 8 * t + 4 * (blk & 1) + 2 * half;
   return 32 * W32 + 4 * t + 2 * half;
+}
+
+// Routing score of one staged page: the max over the G heads and the page's
+// `valid` tokens of Z_t.qz_h + R_t.qr_h, from the page's Z rows `zs` and R
+// rows `rs` in shared memory and this lane's folded-query fragments `fr`
+// (mma tiles: tokens as M, (head, hi|lo) as N).  Returned in every lane.
+template <int G, int RR, int RS, int P, int FR>
+__device__ __forceinline__ float route_page_score(const __nv_bfloat16* zs, const __nv_bfloat16* rs, int valid,
+                                                  const uint32_t (&fr)[FR]) {
+  using Shape = RouteMma<G, RR, RS>;
+  constexpr int NT = Shape::NT;
+  constexpr int FRT = 2 * Shape::ZB + Shape::Z8 + 2 * Shape::SB + Shape::S8;
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  float best = -INFINITY;
+#pragma unroll
+  for (int mt = 0; mt < P / 16; ++mt) {
+    float acc[NT][4];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+    const __nv_bfloat16* z0 = zs + (mt * 16 + g) * RR;
+    const __nv_bfloat16* z1 = z0 + 8 * RR;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      const uint32_t* f = fr + j * FRT;
+#pragma unroll
+      for (int sp = 0; sp < Shape::Z32; ++sp) {
+        const uint4 v0 = lds128(z0 + 32 * sp + 8 * t), v1 = lds128(z1 + 32 * sp + 8 * t);
+        mma_k16(acc[j], v0.x, v1.x, v0.y, v1.y, f[4 * sp + 0], f[4 * sp + 1]);
+        mma_k16(acc[j], v0.z, v1.z, v0.w, v1.w, f[4 * sp + 2], f[4 * sp + 3]);
+      }
+      if (Shape::Z16) {
+        const uint2 v0 = lds64(z0 + 32 * Shape::Z32 + 4 * t), v1 = lds64(z1 + 32 * Shape::Z32 + 4 * t);
+        mma_k16(acc[j], v0.x, v1.x, v0.y, v1.y, f[2 * Shape::ZB - 2], f[2 * Shape::ZB - 1]);
+      }
+      if (Shape::Z8) {
+        const int o = 32 * Shape::Z32 + 16 * Shape::Z16 + 2 * t;
+        mma_k8(acc[j], lds32(z0 + o), lds32(z1 + o), f[2 * Shape::ZB]);
+      }
+      if (RS > 0) {
+        const uint32_t* fs = f + 2 * Shape::ZB + Shape::Z8;
+        const __nv_bfloat16* r0 = rs + (mt * 16 + g) * RS;
+        const __nv_bfloat16* r1 = r0 + 8 * RS;
+#pragma unroll
+        for (int sp = 0; sp < Shape::S32; ++sp) {
+          const uint4 v0 = lds128(r0 + 32 * sp + 8 * t), v1 = lds128(r1 + 32 * sp + 8 * t);
+          mma_k16(acc[j], v0.x, v1.x, v0.y, v1.y, fs[4 * sp + 0], fs[4 * sp + 1]);
+          mma_k16(acc[j], v0.z, v1.z, v0.w, v1.w, fs[4 * sp + 2], fs[4 * sp + 3]);
+        }
+        if (Shape::S16) {
+          const uint2 v0 = lds64(r0 + 32 * Shape::S32 + 4 * t), v1 = lds64(r1 + 32 * Shape::S32 + 4 * t);
+          mma_k16(acc[j], v0.x, v1.x, v0.y, v1.y, fs[2 * Shape::SB - 2], fs[2 * Shape::SB - 1]);
+        }
+        if (Shape::S8) {
+          const int o = 32 * Shape::S32 + 16 * Shape::S16 + 2 * t;
+          mma_k8(acc[j], lds32(r0 + o), lds32(r1 + o), fs[2 * Shape::SB]);
+        }
+      }
+    }
+    // D fragment: rows g, g+8 = tokens; columns 2t, 2t+1 = (hi, lo) of head 4j + t.
+    // Rows past the sequence end are dropped by selection, never by arithmetic.
+    const int tok0 = mt * 16 + g, tok1 = tok0 + 8;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      if (4 * j + t < G) {
+        if (tok0 < valid) best = fmaxf(best, acc[j][0] + acc[j][1]);
+        if (tok1 < valid) best = fmaxf(best, acc[j][2] + acc[j][3]);
+      }
+    }
+  }
+  return warp_max(best);
 }
 
 // Position in the flat list of routed pages (sequence-major, then KV head,
@@ -304,11 +382,12 @@ __device__ void warp_fold_query(const RouteArgs& a, int b, int kvh, float* qsm, 
 // (row, head) products and a butterfly reduce-scatter (31 shuffles) leaves
 // the full sum of (row, head) = (lane/G, lane%G) in the lane.
 template <int G, int RR, int RS, int CPL>
-__device__ void fold_slice(const RouteArgs& a, int u, int slice) {
+__device__ void fold_slice(const void* q_all, const float* w_zk, const float* b_r, float* qf, int num_kv_heads,
+                           int u, int slice) {
   constexpr int RPB = 32 / G, ROWS = RR + RS, d = 32 * CPL;
   const int lane = threadIdx.x & 31;
-  const int kvh = u % a.num_kv_heads;
-  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q) + (size_t)u * G * d + lane * CPL;
+  const int kvh = u % num_kv_heads;
+  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(q_all) + (size_t)u * G * d + lane * CPL;
   float qv[G][CPL];
 #pragma unroll
   for (int h = 0; h < G; ++h)
@@ -319,8 +398,8 @@ __device__ void fold_slice(const RouteArgs& a, int u, int slice) {
 #pragma unroll
   for (int rl = 0; rl < RPB; ++rl) {
     const int row = row0 + rl;
-    const float* src = row < RR ? a.w_zk + ((size_t)kvh * RR + row) * d
-                                : a.b_r + ((size_t)kvh * RS + (row - RR)) * d;
+    const float* src = row < RR ? w_zk + ((size_t)kvh * RR + row) * d
+                                : b_r + ((size_t)kvh * RS + (row - RR)) * d;
     src += lane * CPL;
     float w[CPL];
     if constexpr (CPL == 4) {
@@ -353,7 +432,12 @@ __device__ void fold_slice(const RouteArgs& a, int u, int slice) {
     }
   }
   const int row = row0 + lane / G, h = lane % G;
-  if (row < ROWS) a.qf[((size_t)u * G + h) * ROWS + row] = v[0];
+  if (row < ROWS) qf[((size_t)u * G + h) * ROWS + row] = v[0];
+}
+
+template <int G, int RR, int RS, int CPL>
+__device__ __forceinline__ void fold_slice(const RouteArgs& a, int u, int slice) {
+  fold_slice<G, RR, RS, CPL>(a.q, a.w_zk, a.b_r, a.qf, a.num_kv_heads, u, slice);
 }
 
 // This lane's routing B-fragment words for unit u, from the folded query
@@ -399,9 +483,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_c
   constexpr int NT = Shape::NT;
   static_assert(P % 16 == 0, "page size must be a multiple of 16");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g = lane >> 2, t = lane & 3;
   constexpr uint32_t zbytes = P * RR * 2, rbytes = P * RS * 2;
-  constexpr uint32_t stage_bytes = zbytes + rbytes;
+  constexpr uint32_t page_bytes = zbytes + rbytes;
+  constexpr int RPS = route_pages_per_stage(P, RR, RS);
+  constexpr uint32_t stage_bytes = RPS * page_bytes;
   const int S = a.stages;
 
   extern __shared__ __align__(128) uint8_t smem[];
@@ -424,46 +509,70 @@ __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_c
   const int W = gridDim.x * kRouteWarps, wg = blockIdx.x * kRouteWarps + warp;
   const long long T = offsets[a.batch];
   const int f0 = (int)(T * wg / W), f1 = (int)(T * (wg + 1) / W);
-  const int count = f1 - f0;
+  const int count = f1 - f0;              // pages
+  const int nst = (count + RPS - 1) / RPS;  // stages of up to RPS pages
 
   const __nv_bfloat16* zpool = static_cast<const __nv_bfloat16*>(a.z_pool);
   const __nv_bfloat16* rpool = static_cast<const __nv_bfloat16*>(a.r_pool);
   const uint64_t pol = policy_evict_first();
-  RouteCursor ic;  // issue cursor (lane 0), runs S pages ahead
+  RouteCursor ic;  // issue cursor (lane 0), runs S stages ahead
   if (count > 0) ic.seek(a, offsets, f0);
   RouteCursor cc = ic;  // compute cursor
-  // lane 0 looks the next slot up one iteration early, so the page-table
-  // read overlaps the current page's arithmetic
-  auto lookup = [&]() { return __ldg(a.page_table + (size_t)ic.b * a.ld_pt + ic.j); };
-  auto issue = [&](int i, int slot) {
-    if (slot < 0 || slot >= a.num_slots) {
-      atomicOr(a.status, kStatusBadSlot);
-      slot = 0;
+  // Stage i holds pages [i*RPS, min((i+1)*RPS, count)) of this warp's share.
+  // Lane 0 looks the slots of the next stage to issue up one iteration
+  // early, so the page-table reads overlap the current stage's arithmetic.
+  auto stage_pages = [&](int i) { return min(RPS, count - i * RPS); };
+  int nslot[RPS];
+  auto lookup = [&](int cnt) {
+    RouteCursor c = ic;
+#pragma unroll
+    for (int k = 0; k < RPS; ++k) {
+      nslot[k] = 0;
+      if (k < cnt) {
+        nslot[k] = __ldg(a.page_table + (size_t)c.b * a.ld_pt + c.j);
+        c.advance(a);
+      }
     }
-    const size_t row0 = ((size_t)slot * a.num_kv_heads + ic.kvh) * P;
-    uint64_t* bar = &bars[warp][i % S];
-    uint8_t* dst = ring + (size_t)(i % S) * stage_bytes;
+  };
+  // stage i goes to ring position s (= i mod S, tracked by the caller)
+  auto issue = [&](int i, int s) {
+    const int cnt = stage_pages(i);
+    uint64_t* bar = &bars[warp][s];
+    uint8_t* dst = ring + (size_t)s * stage_bytes;
     if (skip_issue_for_test(wg, i)) {
-      ic.advance(a);
+      for (int k = 0; k < cnt; ++k) ic.advance(a);
       return;
     }
-    mbar_arrive_expect_tx(bar, stage_bytes);
-    bulk_load(dst, zpool + row0 * RR, zbytes, bar, pol);
-    if (RS > 0) bulk_load(dst + zbytes, rpool + row0 * RS, rbytes, bar, pol);
-    ic.advance(a);
+    mbar_arrive_expect_tx(bar, cnt * page_bytes);
+#pragma unroll
+    for (int k = 0; k < RPS; ++k) {
+      if (k < cnt) {
+        int slot = nslot[k];
+        if (slot < 0 || slot >= a.num_slots) {
+          atomicOr(a.status, kStatusBadSlot);
+          slot = 0;
+        }
+        const size_t row0 = ((size_t)slot * a.num_kv_heads + ic.kvh) * P;
+        bulk_load(dst + k * page_bytes, zpool + row0 * RR, zbytes, bar, pol);
+        if (RS > 0) bulk_load(dst + k * page_bytes + zbytes, rpool + row0 * RS, rbytes, bar, pol);
+        ic.advance(a);
+      }
+    }
   };
   {
-    // the first S pages: lane j looks page j up (in parallel), lane 0 issues
-    const int first = min(S, count);
+    // the first S stages: lane j looks page j up (all reads in parallel),
+    // lane 0 issues
+    const int first = min(S * RPS, count);
     int sl = 0;
     if (lane < first) {
       RouteCursor c = ic;
       for (int k = 0; k < lane; ++k) c.advance(a);
       sl = __ldg(a.page_table + (size_t)c.b * a.ld_pt + c.j);
     }
-    for (int i = 0; i < first; ++i) {
-      const int sli = __shfl_sync(0xffffffffu, sl, i);
-      if (lane == 0) issue(i, sli);
+    for (int i = 0; i < S && i < nst; ++i) {
+#pragma unroll
+      for (int k = 0; k < RPS; ++k) nslot[k] = __shfl_sync(0xffffffffu, sl, (i * RPS + k) & 31);
+      if (lane == 0) issue(i, i);
     }
   }
   pdl_launch_dependents();
@@ -493,97 +602,49 @@ __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_c
 
   bool ok = true;
   int i = 0;
-  for (; i < count; ++i) {
-    int next_slot = 0;
-    if (lane == 0 && i + S < count) next_slot = lookup();
-    const int u = cc.unit(a);
-    if (u != cur_u) {
-      // this unit's folded query: its slices come from other warps; should
-      // they be late (their CTA not yet resident), fold it here instead
-      cur_u = u;
-      bool ready = true;
-      if (lane < NSL) ready = wait_tag(a.fold_flag + (size_t)u * 32 + lane, a.tag, kFoldWaitNs);
-      if (__all_sync(0xffffffffu, ready)) {
-        load_route_frags<G, RR, RS, FR>(a.qf + (size_t)u * G * (RR + RS), fr);
-      } else if (a.head_dim == 128) {
-        warp_fold_query<G, RR, RS, FR, 4>(a, cc.b, cc.kvh, qsm, fr);
-      } else {
-        warp_fold_query<G, RR, RS, FR, 2>(a, cc.b, cc.kvh, qsm, fr);
-      }
-    }
-    ok = mbar_wait(&bars[warp][i % S], (uint32_t)((i / S) & 1), a.status);
+  int s_i = 0;        // ring position of stage i (i mod S)
+  uint32_t ph_i = 0;  // phase parity of that position's barrier for stage i
+  for (; i < nst; ++i) {
+    if (lane == 0 && i + S < nst) lookup(stage_pages(i + S));
+    ok = mbar_wait(&bars[warp][s_i], ph_i, a.status);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;
-    const __nv_bfloat16* zs = reinterpret_cast<const __nv_bfloat16*>(ring + (size_t)(i % S) * stage_bytes);
-    const __nv_bfloat16* rs = zs + P * RR;
-    const int valid = min(P, cc.L - cc.j * P);
-    float best = -INFINITY;
+    const int cnt = stage_pages(i);
+    const uint8_t* stage = ring + (size_t)s_i * stage_bytes;
 #pragma unroll
-    for (int mt = 0; mt < P / 16; ++mt) {
-      float acc[NT][4];
-#pragma unroll
-      for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-      const __nv_bfloat16* z0 = zs + (mt * 16 + g) * RR;
-      const __nv_bfloat16* z1 = z0 + 8 * RR;
-#pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        const uint32_t* f = fr + j * (2 * Shape::ZB + Shape::Z8 + 2 * Shape::SB + Shape::S8);
-#pragma unroll
-        for (int sp = 0; sp < Shape::Z32; ++sp) {
-          const uint4 v0 = lds128(z0 + 32 * sp + 8 * t), v1 = lds128(z1 + 32 * sp + 8 * t);
-          mma_k16(acc[j], v0.x, v1.x, v0.y, v1.y, f[4 * sp + 0], f[4 * sp + 1]);
-          mma_k16(acc[j], v0.z, v1.z, v0.w, v1.w, f[4 * sp + 2], f[4 * sp + 3]);
-        }
-        if (Shape::Z16) {
-          const uint2 v0 = lds64(z0 + 32 * Shape::Z32 + 4 * t), v1 = lds64(z1 + 32 * Shape::Z32 + 4 * t);
-          mma_k16(acc[j], v0.x, v1.x, v0.y, v1.y, f[2 * Shape::ZB - 2], f[2 * Shape::ZB - 1]);
-        }
-        if (Shape::Z8) {
-          const int o = 32 * Shape::Z32 + 16 * Shape::Z16 + 2 * t;
-          mma_k8(acc[j], lds32(z0 + o), lds32(z1 + o), f[2 * Shape::ZB]);
-        }
-        if (RS > 0) {
-          const uint32_t* fs = f + 2 * Shape::ZB + Shape::Z8;
-          const __nv_bfloat16* r0 = rs + (mt * 16 + g) * RS;
-          const __nv_bfloat16* r1 = r0 + 8 * RS;
-#pragma unroll
-          for (int sp = 0; sp < Shape::S32; ++sp) {
-            const uint4 v0 = lds128(r0 + 32 * sp + 8 * t), v1 = lds128(r1 + 32 * sp + 8 * t);
-            mma_k16(acc[j], v0.x, v1.x, v0.y, v1.y, fs[4 * sp + 0], fs[4 * sp + 1]);
-            mma_k16(acc[j], v0.z, v1.z, v0.w, v1.w, fs[4 * sp + 2], fs[4 * sp + 3]);
-          }
-          if (Shape::S16) {
-            const uint2 v0 = lds64(r0 + 32 * Shape::S32 + 4 * t), v1 = lds64(r1 + 32 * Shape::S32 + 4 * t);
-            mma_k16(acc[j], v0.x, v1.x, v0.y, v1.y, fs[2 * Shape::SB - 2], fs[2 * Shape::SB - 1]);
-          }
-          if (Shape::S8) {
-            const int o = 32 * Shape::S32 + 16 * Shape::S16 + 2 * t;
-            mma_k8(acc[j], lds32(r0 + o), lds32(r1 + o), fs[2 * Shape::SB]);
+    for (int k = 0; k < RPS; ++k) {
+      if (k < cnt) {
+        const int u = cc.unit(a);
+        if (u != cur_u) {
+          // this unit's folded query: its slices come from other warps; should
+          // they be late (their CTA not yet resident), fold it here instead
+          cur_u = u;
+          bool ready = true;
+          if (lane < NSL) ready = wait_tag(a.fold_flag + (size_t)u * 32 + lane, a.tag, kFoldWaitNs);
+          if (__all_sync(0xffffffffu, ready)) {
+            load_route_frags<G, RR, RS, FR>(a.qf + (size_t)u * G * (RR + RS), fr);
+          } else if (a.head_dim == 128) {
+            warp_fold_query<G, RR, RS, FR, 4>(a, cc.b, cc.kvh, qsm, fr);
+          } else {
+            warp_fold_query<G, RR, RS, FR, 2>(a, cc.b, cc.kvh, qsm, fr);
           }
         }
-      }
-      // D fragment: rows g, g+8 = tokens; columns 2t, 2t+1 = (hi, lo) of head 4j + t.
-      // Rows past the sequence end are dropped by selection, never by arithmetic.
-      const int tok0 = mt * 16 + g, tok1 = tok0 + 8;
-#pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        if (4 * j + t < G) {
-          if (tok0 < valid) best = fmaxf(best, acc[j][0] + acc[j][1]);
-          if (tok1 < valid) best = fmaxf(best, acc[j][2] + acc[j][3]);
-        }
+        const __nv_bfloat16* zs = reinterpret_cast<const __nv_bfloat16*>(stage + k * page_bytes);
+        const float best = route_page_score<G, RR, RS, P, FR>(zs, zs + P * RR, min(P, cc.L - cc.j * P), fr);
+        if (lane == 0) a.scores[(size_t)cur_u * a.ld_pt + cc.j] = best;
+        cc.advance(a);
       }
     }
-    best = warp_max(best);
     __syncwarp();
-    if (lane == 0) {
-      a.scores[(size_t)cur_u * a.ld_pt + cc.j] = best;
-      if (i + S < count) issue(i + S, next_slot);
+    if (lane == 0 && i + S < nst) issue(i + S, s_i);  // (i + S) mod S = i mod S
+    if (++s_i == S) {
+      s_i = 0;
+      ph_i ^= 1u;
     }
-    cc.advance(a);
   }
   if (!ok) {
-    if (lane == 0)  // drain the copies still in flight, [i, min(i + S, count))
-      for (int j = i; j < count && j < i + S; ++j)
+    if (lane == 0)  // drain the copies still in flight, stages [i, min(i + S, nst))
+      for (int j = i; j < nst && j < i + S; ++j)
         mbar_wait(&bars[warp][j % S], (uint32_t)((j / S) & 1), a.status);
   }
 }
