@@ -328,9 +328,14 @@ struct AttnCursor {
     }
   }
   __device__ __forceinline__ int unit(const AttnArgs& a) const { return b * a.num_kv_heads + kvh; }
-  __device__ __forceinline__ int page(const AttnArgs& a) const {
+  __device__ __forceinline__ int page(const AttnArgs& a) const { return checked(a, page_raw(a)); }
+  // The selected page, unchecked: the load stays in flight until the value
+  // is used (check it with checked() when the item is issued).
+  __device__ __forceinline__ int page_raw(const AttnArgs& a) const {
     if (a.topk >= n) return jj;
-    int p = __ldcg(a.sel + (size_t)unit(a) * a.ld_sel + jj);
+    return __ldcg(a.sel + (size_t)unit(a) * a.ld_sel + jj);
+  }
+  __device__ __forceinline__ int checked(const AttnArgs& a, int p) const {
     if (p < 0 || p >= n) {
       atomicOr(a.status, kStatusBadPage);
       p = 0;
@@ -478,7 +483,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
   }
   if (lane == 0) {
     if (S < count) {
-      next_page = ic.page(a);
+      next_page = ic.page_raw(a);
       ia = ic;
       ia.advance(a, sub);
     }
@@ -551,8 +556,13 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
   for (; i < count; ++i) {
     int next_slot = 0, page_after = 0;
     if (lane == 0) {
-      if (i + S < count) next_slot = slot_of(next_page);
-      if (i + S + 1 < count) page_after = ia.page(a);
+      // the page of item i + S was read one iteration ago: check it and read
+      // its slot now; the page of the item after it stays in flight
+      if (i + S < count) {
+        next_page = ic.checked(a, next_page);
+        next_slot = slot_of(next_page);
+      }
+      if (i + S + 1 < count) page_after = ia.page_raw(a);
     }
     const int u = cc.unit(a);
     if (u != cur_u) {
