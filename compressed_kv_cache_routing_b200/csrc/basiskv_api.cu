@@ -44,6 +44,8 @@ int fail(int code, const char* fmt, ...) {
 constexpr int kMaxSplits = 16;
 constexpr int kProfEvents = 5;  // start, after prep, after routing, after selection, after attention
 constexpr int kPartsCap = kMaxSplits * kAttnWarps;  // partials per unit
+constexpr size_t kSchedWords = 2;  // work-claim counters of the persistent routing grid
+constexpr int kRouteStaticPct = 75;  // routing pages in static shares when units are long
 // Ring bytes per CTA: small rings let several CTAs (and so many warps, each
 // with copies in flight) share an SM.
 constexpr size_t kRouteSmemBudget = 48 * 1024;
@@ -168,9 +170,8 @@ struct basiskv_handle {
   int32_t* d_sel = nullptr;         // [max_batch][Hkv][max_topk]
   float* d_part_ml = nullptr;       // [max_batch*Hkv][kPartsCap][G][2]
   float* d_part_acc = nullptr;      // [max_batch*Hkv][kPartsCap][G][r]
-  uint32_t* d_counters = nullptr;   // [3][max_batch*Hkv]: route, attention, partial count
-  float* d_qf = nullptr;            // [max_batch*Hkv][G][r+s] folded routing queries
-  uint32_t* d_fold_flag = nullptr;  // [max_batch*Hkv][32] tag of the call that wrote each fold slice
+  uint32_t* d_counters = nullptr;   // [3][max_batch*Hkv]: route, attention, partial count; then kSchedWords
+  uint64_t* d_qf = nullptr;         // [max_batch*Hkv][G][r+s] folded routing queries, tagged with the call
   uint32_t route_tag = 0;           // tag of the last routing launch
   float* d_enc = nullptr;           // pinv(B_v) [Hkv][d][r], then pinv(B_r) [Hkv][d][s] (basiskv_encode_rows)
   bool enc_ready = false;
@@ -330,6 +331,7 @@ struct LaunchPlan {
   int attn_pps = 0, attn_splits = 0;
   // persistent kernels
   int route_ctas = 0, attn_ctas = 0;
+  int route_static_pct = 100;  // pages of the persistent routing grid handed out in static shares
   // work plans (prefix over sequences), when batch <= kPlanMax
   std::vector<int32_t> route_off, attn_off;
 };
@@ -365,6 +367,11 @@ LaunchPlan plan(const basiskv_handle* h, int batch, int topk, bool force_route) 
   }
   lp.max_unit_items = max_kb * lp.sub;
   lp.any_routed = max_routed > 0;
+  // Long units (512 pages and more): a quarter of the routed pages is left
+  // to warps that finish their static share early, which evens out the
+  // ends of the warps.  Short units gain nothing from it (each claimed
+  // chunk starts a new unit, whose folded query must be fetched first).
+  lp.route_static_pct = max_routed >= 512 ? kRouteStaticPct : 100;
 
   // generic kernels: a grid of (chunk | split, Hkv, batch)
   if (lp.any_routed) {
@@ -440,6 +447,7 @@ RouteArgs route_args(basiskv_handle* h, const LaunchPlan& lp, const void* q, int
   a.sel = h->d_sel;
   a.sel_out = sel_out;
   a.counters = h->d_counters;
+  a.sched = h->d_counters + 3 * (size_t)p.max_batch * p.num_kv_heads;
   a.status = h->d_status;
   a.ld_pt = p.max_pages_per_seq;
   a.ld_sel = p.max_topk;
@@ -453,13 +461,13 @@ RouteArgs route_args(basiskv_handle* h, const LaunchPlan& lp, const void* q, int
   a.topk = topk;
   a.pages_per_cta = lp.route_ppc;
   a.stages = h->route_stages;
+  a.static_pct = lp.route_static_pct;
   a.force = force;
   a.fill_tail = force;
   a.batch = lp.batch;
   a.route_off = h->d_route_off;
   a.qf = h->d_qf;
-  a.fold_flag = h->d_fold_flag;
-  if (++h->route_tag == 0) h->route_tag = 1;  // 0 never matches: the flags start zeroed
+  if (++h->route_tag == 0) h->route_tag = 1;  // 0 never matches: the folded queries start zeroed
   a.tag = h->route_tag;
   a.plan_n = lp.route_off.empty() ? -1 : lp.batch;
   for (size_t i = 0; i < lp.route_off.size(); ++i) a.plan_off[i] = lp.route_off[i];
@@ -634,10 +642,9 @@ int basiskv_create(const basiskv_params* p, basiskv_handle** out) {
       {(void**)&h->d_sel, sizeof(int32_t) * U * p->max_topk},
       {(void**)&h->d_part_ml, sizeof(float) * U * kPartsCap * G * 2},
       {(void**)&h->d_part_acc, sizeof(float) * U * kPartsCap * G * p->rank_r},
-      {(void**)&h->d_counters, sizeof(uint32_t) * 3 * U},
-      {(void**)&h->d_qf, sizeof(float) * U * G * (p->rank_r + p->rank_s)},
+      {(void**)&h->d_counters, sizeof(uint32_t) * (3 * U + kSchedWords)},
+      {(void**)&h->d_qf, sizeof(uint64_t) * U * G * (p->rank_r + p->rank_s)},
       {(void**)&h->d_enc, sizeof(float) * Hkv * p->head_dim * (p->rank_r + p->rank_s)},
-      {(void**)&h->d_fold_flag, sizeof(uint32_t) * U * 32},
       {(void**)&h->d_status, sizeof(uint32_t)},
       {(void**)&h->d_route_off, sizeof(int32_t) * (B + 1)},
       {(void**)&h->d_attn_off, sizeof(int32_t) * (B + 1)},
@@ -653,8 +660,8 @@ int basiskv_create(const basiskv_params* p, basiskv_handle** out) {
   }
   if (cudaMemset(h->d_page_table, 0, sizeof(int32_t) * B * p->max_pages_per_seq) != cudaSuccess ||
       cudaMemset(h->d_seq_lens, 0, sizeof(int32_t) * B) != cudaSuccess ||
-      cudaMemset(h->d_counters, 0, sizeof(uint32_t) * 3 * U) != cudaSuccess ||
-      cudaMemset(h->d_fold_flag, 0, sizeof(uint32_t) * U * 32) != cudaSuccess ||
+      cudaMemset(h->d_counters, 0, sizeof(uint32_t) * (3 * U + kSchedWords)) != cudaSuccess ||
+      cudaMemset(h->d_qf, 0, sizeof(uint64_t) * U * G * (p->rank_r + p->rank_s)) != cudaSuccess ||
       cudaMemset(h->d_status, 0, sizeof(uint32_t)) != cudaSuccess)
     return cleanup_fail(BASISKV_ERR_CUDA, "cudaMemset failed");
   h->h_table.assign(B * p->max_pages_per_seq, 0);
@@ -699,7 +706,7 @@ int basiskv_destroy(basiskv_handle* h) {
   cudaDeviceSynchronize();
   void* ptrs[] = {h->d_page_table, h->d_seq_lens, h->d_scores, h->d_sel, h->d_part_ml, h->d_part_acc,
                   h->d_counters, h->d_status, h->d_q_stage, h->d_out_stage, h->d_sel_stage,
-                  h->d_route_off, h->d_attn_off, h->d_qf, h->d_fold_flag, h->d_enc};
+                  h->d_route_off, h->d_attn_off, h->d_qf, h->d_enc};
   for (void* q : ptrs)
     if (q) cudaFree(q);
   for (cudaEvent_t e : h->events) cudaEventDestroy(e);
@@ -1084,7 +1091,8 @@ int basiskv_get_status(basiskv_handle* h, uint32_t* status, int clear) {
   if (clear && *status) {
     // a call that gave up part way can leave arrival counts behind: start
     // the next call from zero
-    CUDA_TRY(cudaMemset(h->d_counters, 0, sizeof(uint32_t) * 3 * (size_t)h->p.max_batch * h->p.num_kv_heads));
+    CUDA_TRY(cudaMemset(h->d_counters, 0,
+                        sizeof(uint32_t) * (3 * (size_t)h->p.max_batch * h->p.num_kv_heads + kSchedWords)));
     CUDA_TRY(cudaMemset(h->d_status, 0, sizeof(uint32_t)));
   }
   return BASISKV_OK;

@@ -87,23 +87,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   }
 }
 
-// Wait (acquire) until *flag == tag, for at most limit_ns; false on expiry.
-// Polls back off so that many waiters do not flood one L2 line.
+// How long a routing warp waits for a folded query written by other warps
+// before it folds the query itself.
 constexpr uint64_t kFoldWaitNs = 50000ull;
-__device__ __forceinline__ bool wait_tag(const uint32_t* flag, uint32_t tag, uint64_t limit_ns) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
-  if (v == tag) return true;
-  const uint64_t t0 = global_timer_ns();
-  uint32_t pause = 32;
-  for (;;) {
-    __nanosleep(pause);
-    pause = pause < 1024u ? 2 * pause : 1024u;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
-    if (v == tag) return true;
-    if (global_timer_ns() - t0 > limit_ns) return false;
-  }
-}
 
 // ---- bulk copy global -> shared (TMA unit, non-tensor form) -----------------
 // dst, src 16-byte aligned, bytes a multiple of 16.  Completion is reported
@@ -115,6 +101,16 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       " [%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst)),
       "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
       : "memory");
+}
+
+// 8-byte relaxed (gpu scope) accesses: each is single-copy atomic, so a
+// value and a tag packed into one word are seen together.
+__device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+// Two consecutive words (p 16-byte aligned); each word is read atomically.
+__device__ __forceinline__ void ld_relaxed_v2u64(const uint64_t* p, uint64_t& x, uint64_t& y) {
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(x), "=l"(y) : "l"(p) : "memory");
 }
 
 __device__ __forceinline__ uint64_t policy_evict_first() {

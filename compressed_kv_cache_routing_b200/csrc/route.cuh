@@ -10,13 +10,14 @@
 // token and head and reads only the r + s stored values of each token.
 // Page score S_j = max over the G heads and page j's valid tokens.
 //
-// Two kernels: route_mma_kernel (bf16 pools, tensor cores, persistent over a
-// flat page list; the fold is spread over all warps as (unit, row slice)
-// tasks written to global memory and tagged, and a warp entering a unit
-// reads it back, folding locally only if the slices are late; the
-// selection runs in the next grid) and route_generic_kernel (any dtype,
-// grid (chunks of pages, Hkv, batch), fold once per CTA, the last CTA of
-// each (sequence, KV head) runs the top-k).
+// Two kernels: route_mma_kernel (bf16 pools, tensor cores, persistent over
+// a flat page list handed out as static shares plus chunks claimed at run
+// time; the fold is spread over all warps as (unit, row slice) tasks whose
+// results are written to global memory tagged with the call, and a warp
+// entering a unit reads them back, folding locally only if they are late;
+// the selection runs in the next grid) and route_generic_kernel (any
+// dtype, grid (chunks of pages, Hkv, batch), fold once per CTA, the last
+// CTA of each (sequence, KV head) runs the top-k).
 #pragma once
 
 #include "common.cuh"
@@ -37,17 +38,18 @@ struct RouteArgs {
   int32_t* sel;             // [B][Hkv][ld_sel]
   int32_t* sel_out;         // [B][Hkv][topk] or null
   uint32_t* counters;       // [B][Hkv]
+  uint32_t* sched;          // [2] chunk claims, finished warps (persistent kernel; zero between calls)
   uint32_t* status;
   int ld_pt, ld_sel, num_slots, num_kv_heads, head_dim, page_size;
   int rank_r, rank_s, gqa_group;
   int topk, pages_per_cta, stages;
+  int static_pct;           // persistent kernel: percent of the pages handed out in static shares
   int force;                // route units whose every page would be selected
   int fill_tail;            // chunk 0 writes -inf to scores[n_b .. ld_pt)
   // persistent tensor-core kernel only
   int batch;
   const int32_t* route_off; // [B+1] prefix of routed pages x Hkv (from the prep grid)
-  float* qf;                // [B*Hkv][G][r+s] folded queries (fp32)
-  uint32_t* fold_flag;      // [B*Hkv][32] per fold slice: the tag of the call that wrote it
+  uint64_t* qf;             // [B*Hkv][G][r+s] folded queries: (tag << 32) | fp32 bits
   uint32_t tag;             // this call's tag (never 0)
   int plan_n;               // >= 0: plan_off holds route_off (batch <= kPlanMax)
   int32_t plan_off[kPlanMax + 1];
@@ -56,6 +58,7 @@ struct RouteArgs {
 constexpr int kRouteThreads = 128;
 constexpr int kRouteWarps = kRouteThreads / 32;
 constexpr int kMaxStages = 8;
+constexpr int kRouteChunkStages = 2;  // stages per claimed chunk of the persistent kernel
 
 // Pages staged together by route_mma_kernel: about 6 KB per stage, so small
 // pages (P = 32 with narrow ranks) share one barrier wait and one issue.
@@ -143,11 +146,11 @@ __device__ void route_finish(const RouteArgs& a, const RouteUnit& ru, TopkSmem& 
 // The B fragments use the same permutation, so every dot product is a sum
 // over the same index set.
 //
-// Persistent: every warp streams one contiguous share of the flat list of
-// routed pages (sequence-major, then KV head, then page) through its own
-// ring of `stages` shared buffers filled by bulk copies (cp.async.bulk, L2
-// evict-first) completing on mbarriers, and writes one score per page.  The
-// selection runs in the next grid (topk_kernel).
+// Persistent: every warp streams chunks of the flat list of routed pages
+// (sequence-major, then KV head, then page), claimed from a grid-wide
+// counter, through its own ring of `stages` shared buffers filled by bulk
+// copies (cp.async.bulk, L2 evict-first) completing on mbarriers, and writes
+// one score per page.  The selection runs in the next grid (topk_kernel).
 template <int G, int RR, int RS>
 struct RouteMma {
   static constexpr int NT = (2 * G + 7) / 8;  // n8 tiles of (hi, lo) columns
@@ -381,46 +384,70 @@ __device__ void warp_fold_query(const RouteArgs& a, int b, int kvh, float* qsm, 
 // queries: lanes own d/32 consecutive channels, each forms its 32 partial
 // (row, head) products and a butterfly reduce-scatter (31 shuffles) leaves
 // the full sum of (row, head) = (lane/G, lane%G) in the lane.
+template <int G>
+struct FoldIn {
+  float qv[G][4];       // this lane's query channels (d/32 of 4 used)
+  float w[32 / G][4];   // this lane's channels of the slice's basis rows
+};
+
 template <int G, int RR, int RS, int CPL>
-__device__ void fold_slice(const void* q_all, const float* w_zk, const float* b_r, float* qf, int num_kv_heads,
-                           int u, int slice) {
+__device__ __forceinline__ void fold_load(const RouteArgs& a, int u, int slice, FoldIn<G>& in) {
   constexpr int RPB = 32 / G, ROWS = RR + RS, d = 32 * CPL;
   const int lane = threadIdx.x & 31;
-  const int kvh = u % num_kv_heads;
-  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(q_all) + (size_t)u * G * d + lane * CPL;
-  float qv[G][CPL];
+  const int kvh = u % a.num_kv_heads;
+  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q) + (size_t)u * G * d + lane * CPL;
 #pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int j = 0; j < CPL; ++j) qv[h][j] = __bfloat162float(q[h * d + j]);
+  for (int h = 0; h < G; ++h) {
+    if constexpr (CPL == 4) {
+      const uint2 x = __ldg(reinterpret_cast<const uint2*>(q + h * d));
+      in.qv[h][0] = __uint_as_float(x.x << 16);
+      in.qv[h][1] = __uint_as_float(x.x & 0xffff0000u);
+      in.qv[h][2] = __uint_as_float(x.y << 16);
+      in.qv[h][3] = __uint_as_float(x.y & 0xffff0000u);
+    } else {
+      const uint32_t x = __ldg(reinterpret_cast<const uint32_t*>(q + h * d));
+      in.qv[h][0] = __uint_as_float(x << 16);
+      in.qv[h][1] = __uint_as_float(x & 0xffff0000u);
+    }
+  }
   const int row0 = slice * RPB;
-  float v[32];
 #pragma unroll
   for (int rl = 0; rl < RPB; ++rl) {
     const int row = row0 + rl;
-    const float* src = row < RR ? w_zk + ((size_t)kvh * RR + row) * d
-                                : b_r + ((size_t)kvh * RS + (row - RR)) * d;
+    const float* src = row < RR ? a.w_zk + ((size_t)kvh * RR + row) * d
+                                : a.b_r + ((size_t)kvh * RS + (row - RR)) * d;
     src += lane * CPL;
-    float w[CPL];
     if constexpr (CPL == 4) {
       const float4 x = row < ROWS ? __ldg(reinterpret_cast<const float4*>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
-      w[0] = x.x;
-      w[1] = x.y;
-      w[2] = x.z;
-      w[3] = x.w;
+      in.w[rl][0] = x.x;
+      in.w[rl][1] = x.y;
+      in.w[rl][2] = x.z;
+      in.w[rl][3] = x.w;
     } else {
       const float2 x = row < ROWS ? __ldg(reinterpret_cast<const float2*>(src)) : make_float2(0.f, 0.f);
-      w[0] = x.x;
-      w[1] = x.y;
+      in.w[rl][0] = x.x;
+      in.w[rl][1] = x.y;
     }
+  }
+}
+
+// The slice's sums, stored tagged with the call: word (u, h, row) of qf is
+// (tag << 32) | bits of the float, written by one 8-byte relaxed store, so a
+// reader that sees the tag sees the value (no fence, no flag).
+template <int G, int RR, int RS, int CPL>
+__device__ __forceinline__ void fold_store(const RouteArgs& a, int u, int slice, const FoldIn<G>& in) {
+  constexpr int RPB = 32 / G, ROWS = RR + RS;
+  const int lane = threadIdx.x & 31;
+  float v[32];
+#pragma unroll
+  for (int rl = 0; rl < RPB; ++rl)
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       float acc = 0.f;
 #pragma unroll
-      for (int j = 0; j < CPL; ++j) acc = fmaf(w[j], qv[h][j], acc);
+      for (int j = 0; j < CPL; ++j) acc = fmaf(in.w[rl][j], in.qv[h][j], acc);
       v[rl * G + h] = acc;
     }
-  }
 #pragma unroll
   for (int step = 16, cnt = 32; step >= 1; step >>= 1, cnt >>= 1) {
     const bool upper = (lane & step) != 0;
@@ -431,35 +458,34 @@ __device__ void fold_slice(const void* q_all, const float* w_zk, const float* b_
       v[k] = keep + __shfl_xor_sync(0xffffffffu, send, step);
     }
   }
-  const int row = row0 + lane / G, h = lane % G;
-  if (row < ROWS) qf[((size_t)u * G + h) * ROWS + row] = v[0];
+  const int row = slice * RPB + lane / G, h = lane % G;
+  if (row < ROWS)
+    st_relaxed_u64(a.qf + ((size_t)u * G + h) * ROWS + row, ((uint64_t)a.tag << 32) | __float_as_uint(v[0]));
 }
 
-template <int G, int RR, int RS, int CPL>
-__device__ __forceinline__ void fold_slice(const RouteArgs& a, int u, int slice) {
-  fold_slice<G, RR, RS, CPL>(a.q, a.w_zk, a.b_r, a.qf, a.num_kv_heads, u, slice);
-}
-
-// This lane's routing B-fragment words for unit u, from the folded query
-// (split into bf16 hi + lo columns; same order as route_mma_kernel), read
-// from global memory (written by other warps of this grid: read through L2).
+// This lane's routing B-fragment words for unit u from the tagged folded
+// query (split into bf16 hi + lo columns; same order as route_mma_kernel).
+// Returns false when a word does not carry this call's tag yet.
 template <int G, int RR, int RS, int FR>
-__device__ void load_route_frags(const float* qfu, uint32_t (&fr)[FR]) {
+__device__ bool load_route_frags(const uint64_t* qfu, uint32_t tag, uint32_t (&fr)[FR]) {
   using Shape = RouteMma<G, RR, RS>;
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  bool ready = true;
   int w = 0;
 #pragma unroll
   for (int j = 0; j < Shape::NT; ++j) {
     const int hh = 4 * j + (g >> 1);
     const bool lo = g & 1;
-    const float* qz = qfu + hh * (RR + RS);
-    const float* qr = qz + RR;
-    auto word = [&](const float* src, int e) {
+    const uint64_t* qz = qfu + hh * (RR + RS);
+    const uint64_t* qr = qz + RR;
+    auto word = [&](const uint64_t* src, int e) {
       if (hh >= G) return 0u;
-      const float2 x = __ldcg(reinterpret_cast<const float2*>(src + e));
+      uint64_t x0, x1;
+      ld_relaxed_v2u64(src + e, x0, x1);
+      ready = ready && (uint32_t)(x0 >> 32) == tag && (uint32_t)(x1 >> 32) == tag;
       float h0, l0, h1, l1;
-      split_bf16(x.x, h0, l0);
-      split_bf16(x.y, h1, l1);
+      split_bf16(__uint_as_float((uint32_t)x0), h0, l0);
+      split_bf16(__uint_as_float((uint32_t)x1), h1, l1);
       return lo ? pack_bf16(l0, l1) : pack_bf16(h0, h1);
     };
 #pragma unroll
@@ -475,7 +501,15 @@ __device__ void load_route_frags(const float* qfu, uint32_t (&fr)[FR]) {
     }
     if (Shape::S8) fr[w++] = word(qr, 32 * Shape::S32 + 16 * Shape::S16 + 2 * t);
   }
+  return ready;
 }
+
+// Stage bookkeeping of route_mma_kernel: the position of a stage's first
+// page (sequence b, KV head, page j, length L of sequence b) and its page
+// count, written by the issuing lane next to the copies.
+struct RouteStageMeta {
+  int b, kvh_cnt, j, L;  // kvh_cnt = kvh | pages << 16
+};
 
 template <int G, int RR, int RS, int P>
 __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_constant__ RouteArgs a) {
@@ -491,6 +525,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_c
 
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t bars[kRouteWarps][kMaxStages];
+  __shared__ RouteStageMeta smeta[kRouteWarps][kMaxStages];
   __shared__ float qsm_all[kRouteWarps][G * (RR + RS)];
   float* qsm = qsm_all[warp];
   uint8_t* ring = smem + (size_t)warp * S * stage_bytes;
@@ -500,49 +535,95 @@ __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_c
   }
   __syncwarp();
   // The plan comes in the parameters (small batches) or from the prep grid
-  // (then this grid waits for it first).  The query is folded by the warp
-  // itself once its first copies are in flight.
+  // (then this grid waits for it first).
   const int32_t* offsets = a.plan_n >= 0 ? a.plan_off : a.route_off;
   if (a.plan_n < 0) pdl_wait_primary();
 
-  // this warp's contiguous share of the flat routed-page list
+  // Work: the first Ts pages of the flat list go to the warps in equal
+  // contiguous shares; the rest is cut into chunks of CP pages that warps
+  // done with their share claim from a grid-wide counter, so the warps the
+  // memory system serves faster take more of it and all finish close
+  // together.  Scores land at fixed places: the order changes no result.
+  constexpr int CP = RPS * kRouteChunkStages;
   const int W = gridDim.x * kRouteWarps, wg = blockIdx.x * kRouteWarps + warp;
-  const long long T = offsets[a.batch];
-  const int f0 = (int)(T * wg / W), f1 = (int)(T * (wg + 1) / W);
-  const int count = f1 - f0;              // pages
-  const int nst = (count + RPS - 1) / RPS;  // stages of up to RPS pages
+  const int T = offsets[a.batch];
+  const int Ts = (int)((long long)T * a.static_pct / 100);
+  const int ndyn = (T - Ts + CP - 1) / CP;
+
+  // Route-prep first: tasks (unit, slice) -> warp task mod W, each writing
+  // its rows of the folded query tagged with the call.  Done before any page
+  // copy is queued, their reads do not wait behind the copies (a warp with
+  // tasks starts streaming a little later; the claimed chunks even it out).
+  constexpr int NSL = (RR + RS + 32 / G - 1) / (32 / G);
+  static_assert(NSL <= 32, "fold slices per unit must fit a warp");
+  const int U = a.batch * a.num_kv_heads;
+  auto task_routed = [&](int task) {
+    const int b = task / NSL / a.num_kv_heads;
+    return offsets[b + 1] > offsets[b];
+  };
+  for (int task = wg; task < U * NSL; task += W) {
+    if (!task_routed(task)) continue;
+    FoldIn<G> fin;
+    if (a.head_dim == 128) {
+      fold_load<G, RR, RS, 4>(a, task / NSL, task % NSL, fin);
+      fold_store<G, RR, RS, 4>(a, task / NSL, task % NSL, fin);
+    } else {
+      fold_load<G, RR, RS, 2>(a, task / NSL, task % NSL, fin);
+      fold_store<G, RR, RS, 2>(a, task / NSL, task % NSL, fin);
+    }
+  }
 
   const __nv_bfloat16* zpool = static_cast<const __nv_bfloat16*>(a.z_pool);
   const __nv_bfloat16* rpool = static_cast<const __nv_bfloat16*>(a.r_pool);
   const uint64_t pol = policy_evict_first();
-  RouteCursor ic;  // issue cursor (lane 0), runs S stages ahead
-  if (count > 0) ic.seek(a, offsets, f0);
-  RouteCursor cc = ic;  // compute cursor
-  // Stage i holds pages [i*RPS, min((i+1)*RPS, count)) of this warp's share.
-  // Lane 0 looks the slots of the next stage to issue up one iteration
-  // early, so the page-table reads overlap the current stage's arithmetic.
-  auto stage_pages = [&](int i) { return min(RPS, count - i * RPS); };
-  int nslot[RPS];
-  auto lookup = [&](int cnt) {
-    RouteCursor c = ic;
+  // Lane 0 runs the issue side: it looks the next stage up one iteration
+  // before issuing it (the page-table reads overlap the current stage's
+  // arithmetic) and claims the next chunk when it looks up the last stage
+  // of the current piece of work, one iteration before it needs it.
+  RouteCursor ic;                                      // lane 0: next page to look up
+  int lk_flat = (int)((long long)Ts * wg / W);         // its flat index
+  int lk_end = (int)((long long)Ts * (wg + 1) / W);    // end of the current piece
+  int nxt = 0;                                         // the claimed dynamic chunk
+  int nslot[RPS], nkvh[RPS];
+  RouteStageMeta nmeta;  // the looked-up stage (pages 0: none)
+  nmeta.kvh_cnt = 0;
+  if (lane == 0) {
+    if (lk_flat < lk_end) ic.seek(a, offsets, lk_flat);
+    else nxt = (int)atomicAdd(a.sched, 1u);  // no static share
+  }
+  auto lookup = [&]() {
+    nmeta.kvh_cnt = 0;
+    if (lk_flat == lk_end) {
+      if (nxt >= ndyn) return;
+      lk_flat = Ts + nxt * CP;
+      lk_end = min(T, lk_flat + CP);
+      ic.seek(a, offsets, lk_flat);
+    }
+    const int cnt = min(RPS, lk_end - lk_flat);
+    nmeta.b = ic.b;
+    nmeta.kvh_cnt = ic.kvh | (cnt << 16);
+    nmeta.j = ic.j;
+    nmeta.L = ic.L;
 #pragma unroll
     for (int k = 0; k < RPS; ++k) {
       nslot[k] = 0;
+      nkvh[k] = 0;
       if (k < cnt) {
-        nslot[k] = __ldg(a.page_table + (size_t)c.b * a.ld_pt + c.j);
-        c.advance(a);
+        nslot[k] = __ldg(a.page_table + (size_t)ic.b * a.ld_pt + ic.j);
+        nkvh[k] = ic.kvh;
+        ic.advance(a);
       }
     }
+    lk_flat += cnt;
+    if (lk_flat == lk_end) nxt = (int)atomicAdd(a.sched, 1u);  // the piece after this one
   };
-  // stage i goes to ring position s (= i mod S, tracked by the caller)
+  // issue the looked-up stage, the i-th of this warp, into ring position s
   auto issue = [&](int i, int s) {
-    const int cnt = stage_pages(i);
+    const int cnt = nmeta.kvh_cnt >> 16;
     uint64_t* bar = &bars[warp][s];
     uint8_t* dst = ring + (size_t)s * stage_bytes;
-    if (skip_issue_for_test(wg, i)) {
-      for (int k = 0; k < cnt; ++k) ic.advance(a);
-      return;
-    }
+    smeta[warp][s] = nmeta;
+    if (skip_issue_for_test(wg, i)) return;
     mbar_arrive_expect_tx(bar, cnt * page_bytes);
 #pragma unroll
     for (int k = 0; k < RPS; ++k) {
@@ -552,81 +633,110 @@ __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_c
           atomicOr(a.status, kStatusBadSlot);
           slot = 0;
         }
-        const size_t row0 = ((size_t)slot * a.num_kv_heads + ic.kvh) * P;
+        const size_t row0 = ((size_t)slot * a.num_kv_heads + nkvh[k]) * P;
         bulk_load(dst + k * page_bytes, zpool + row0 * RR, zbytes, bar, pol);
         if (RS > 0) bulk_load(dst + k * page_bytes + zbytes, rpool + row0 * RS, rbytes, bar, pol);
-        ic.advance(a);
       }
     }
   };
+  int nissued = 0;  // stages issued by this warp (uniform)
   {
-    // the first S stages: lane j looks page j up (all reads in parallel),
-    // lane 0 issues
-    const int first = min(S * RPS, count);
+    // the first stages of the static share: lane k looks page k up (all
+    // page-table reads in flight together), lane 0 issues
+    const int first = min(min(S * RPS, 32), lk_end - lk_flat);
     int sl = 0;
+    RouteStageMeta m;
+    m.b = m.kvh_cnt = m.j = m.L = 0;
     if (lane < first) {
-      RouteCursor c = ic;
+      RouteCursor c;
+      c.seek(a, offsets, lk_flat);
       for (int k = 0; k < lane; ++k) c.advance(a);
       sl = __ldg(a.page_table + (size_t)c.b * a.ld_pt + c.j);
+      m.b = c.b;
+      m.kvh_cnt = c.kvh;
+      m.j = c.j;
+      m.L = c.L;
     }
-    for (int i = 0; i < S && i < nst; ++i) {
+    for (int s = 0; s * RPS < first; ++s) {
+      const int cnt = min(RPS, first - s * RPS);
+      RouteStageMeta ms;
+      ms.b = __shfl_sync(0xffffffffu, m.b, s * RPS);
+      ms.kvh_cnt = __shfl_sync(0xffffffffu, m.kvh_cnt, s * RPS) | (cnt << 16);
+      ms.j = __shfl_sync(0xffffffffu, m.j, s * RPS);
+      ms.L = __shfl_sync(0xffffffffu, m.L, s * RPS);
 #pragma unroll
-      for (int k = 0; k < RPS; ++k) nslot[k] = __shfl_sync(0xffffffffu, sl, (i * RPS + k) & 31);
-      if (lane == 0) issue(i, i);
+      for (int k = 0; k < RPS; ++k) {
+        const int src = min(s * RPS + k, 31);
+        nslot[k] = __shfl_sync(0xffffffffu, sl, src);
+        nkvh[k] = __shfl_sync(0xffffffffu, m.kvh_cnt, src);
+      }
+      if (lane == 0) {
+        nmeta = ms;
+        issue(nissued, s);
+      }
+      ++nissued;
+    }
+    if (lane == 0) {
+      for (int k = 0; k < first; ++k) ic.advance(a);
+      lk_flat += first;
+      if (first > 0 && lk_flat == lk_end) nxt = (int)atomicAdd(a.sched, 1u);
+      for (int s = nissued; s < S; ++s) {
+        lookup();
+        if (nmeta.kvh_cnt == 0) break;
+        issue(nissued, s);
+        ++nissued;
+      }
+      nmeta.kvh_cnt = 0;
     }
   }
+  nissued = __shfl_sync(0xffffffffu, nissued, 0);
   pdl_launch_dependents();
 
-  // route-prep spread over the warps: task (unit, slice) -> warp task mod W;
-  // each writes its rows of the folded query and tags them with the call
-  constexpr int NSL = (RR + RS + 32 / G - 1) / (32 / G);
-  static_assert(NSL <= 32, "fold slices per unit must fit a warp");
-  const int U = a.batch * a.num_kv_heads;
-  for (int task = wg; task < U * NSL; task += W) {
-    const int u = task / NSL;
-    const int n = (a.seq_lens[u / a.num_kv_heads] + P - 1) / P;
-    if (n == 0 || !(a.force || a.topk < n)) continue;
-    if (a.head_dim == 128) fold_slice<G, RR, RS, 4>(a, u, task % NSL);
-    else fold_slice<G, RR, RS, 2>(a, u, task % NSL);
-    __syncwarp();
-    if (lane == 0) {
-      __threadfence();
-      *reinterpret_cast<volatile uint32_t*>(a.fold_flag + (size_t)u * 32 + task % NSL) = a.tag;
-    }
-  }
-  if (count <= 0) return;
 
   constexpr int FR = NT * (2 * Shape::ZB + Shape::Z8 + 2 * Shape::SB + Shape::S8);
   uint32_t fr[FR];
   int cur_u = -1;
+  RouteCursor cc;  // compute cursor, set from each stage's bookkeeping
 
   bool ok = true;
   int i = 0;
   int s_i = 0;        // ring position of stage i (i mod S)
   uint32_t ph_i = 0;  // phase parity of that position's barrier for stage i
-  for (; i < nst; ++i) {
-    if (lane == 0 && i + S < nst) lookup(stage_pages(i + S));
+  for (; i < nissued; ++i) {
+    if (lane == 0) lookup();  // the stage to issue at the end of this iteration
     ok = mbar_wait(&bars[warp][s_i], ph_i, a.status);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;
-    const int cnt = stage_pages(i);
+    const RouteStageMeta m = smeta[warp][s_i];
+    const int cnt = m.kvh_cnt >> 16;
+    cc.b = m.b;
+    cc.kvh = m.kvh_cnt & 0xffff;
+    cc.j = m.j;
+    cc.L = m.L;
+    cc.n = (m.L + P - 1) / P;
     const uint8_t* stage = ring + (size_t)s_i * stage_bytes;
 #pragma unroll
     for (int k = 0; k < RPS; ++k) {
       if (k < cnt) {
         const int u = cc.unit(a);
         if (u != cur_u) {
-          // this unit's folded query: its slices come from other warps; should
-          // they be late (their CTA not yet resident), fold it here instead
+          // this unit's folded query comes from other warps; should it be
+          // late (their CTA not yet resident), fold it here instead
           cur_u = u;
-          bool ready = true;
-          if (lane < NSL) ready = wait_tag(a.fold_flag + (size_t)u * 32 + lane, a.tag, kFoldWaitNs);
-          if (__all_sync(0xffffffffu, ready)) {
-            load_route_frags<G, RR, RS, FR>(a.qf + (size_t)u * G * (RR + RS), fr);
-          } else if (a.head_dim == 128) {
-            warp_fold_query<G, RR, RS, FR, 4>(a, cc.b, cc.kvh, qsm, fr);
-          } else {
-            warp_fold_query<G, RR, RS, FR, 2>(a, cc.b, cc.kvh, qsm, fr);
+          const uint64_t* qfu = a.qf + (size_t)u * G * (RR + RS);
+          bool ready = __all_sync(0xffffffffu, load_route_frags<G, RR, RS, FR>(qfu, a.tag, fr));
+          if (!ready) {
+            const uint64_t t0 = global_timer_ns();
+            uint32_t pause = 64;
+            while (!ready && global_timer_ns() - t0 < kFoldWaitNs) {
+              __nanosleep(pause);
+              pause = pause < 1024u ? 2 * pause : 1024u;
+              ready = __all_sync(0xffffffffu, load_route_frags<G, RR, RS, FR>(qfu, a.tag, fr));
+            }
+          }
+          if (!ready) {
+            if (a.head_dim == 128) warp_fold_query<G, RR, RS, FR, 4>(a, cc.b, cc.kvh, qsm, fr);
+            else warp_fold_query<G, RR, RS, FR, 2>(a, cc.b, cc.kvh, qsm, fr);
           }
         }
         const __nv_bfloat16* zs = reinterpret_cast<const __nv_bfloat16*>(stage + k * page_bytes);
@@ -636,16 +746,28 @@ __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_c
       }
     }
     __syncwarp();
-    if (lane == 0 && i + S < nst) issue(i + S, s_i);  // (i + S) mod S = i mod S
+    if (lane == 0 && nmeta.kvh_cnt != 0) {
+      issue(nissued, s_i);  // stage nissued = i + S goes where stage i was
+      ++nissued;
+    }
+    nissued = __shfl_sync(0xffffffffu, nissued, 0);
     if (++s_i == S) {
       s_i = 0;
       ph_i ^= 1u;
     }
   }
   if (!ok) {
-    if (lane == 0)  // drain the copies still in flight, stages [i, min(i + S, nst))
-      for (int j = i; j < nst && j < i + S; ++j)
-        mbar_wait(&bars[warp][j % S], (uint32_t)((j / S) & 1), a.status);
+    if (lane == 0)  // drain the copies still in flight, stages [i, nissued)
+      for (int j = i; j < nissued; ++j) mbar_wait(&bars[warp][j % S], (uint32_t)((j / S) & 1), a.status);
+  }
+  // The last warp to finish resets the claim counter for the next call (a
+  // warp's last claim has returned before it arrives here).
+  if (lane == 0) {
+    __threadfence();
+    if (atomicAdd(a.sched + 1, 1u) == (uint32_t)W - 1) {
+      a.sched[0] = 0u;
+      a.sched[1] = 0u;
+    }
   }
 }
 
