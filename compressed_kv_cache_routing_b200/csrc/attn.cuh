@@ -181,9 +181,21 @@ __device__ __forceinline__ void attn_stage(const uint8_t* stage, int valid, cons
     const uint8_t* krow = stage + (nt * 8 + g) * D * KB;
     const int tok = nt * 8 + 2 * t;
     if constexpr (K8) {
+      // 128-byte code rows: odd rows take their two 64-channel spans in the
+      // other order, so a quarter-warp's two rows fall on disjoint banks
+      uint4 kv[D / 64];
+      if constexpr (D / 64 == 2) {
+        const int odd = g & 1;
+        const uint4 u0 = lds128(krow + 64 * odd + 16 * t), u1 = lds128(krow + 64 * (1 - odd) + 16 * t);
+        kv[0] = odd ? u1 : u0;
+        kv[1] = odd ? u0 : u1;
+      } else {
+#pragma unroll
+        for (int sp = 0; sp < D / 64; ++sp) kv[sp] = lds128(krow + 64 * sp + 16 * t);
+      }
 #pragma unroll
       for (int sp = 0; sp < D / 64; ++sp) {
-        const uint4 v = lds128(krow + 64 * sp + 16 * t);
+        const uint4 v = kv[sp];
         uint32_t b0, b1;
         codes_to_f16x2(v.x, b0, b1);
         mma_k16_f16(d, qa[2 * sp][0][0], 0u, qa[2 * sp][0][1], 0u, b0, b1);
@@ -198,11 +210,20 @@ __device__ __forceinline__ void attn_stage(const uint8_t* stage, int valid, cons
       d[0] *= __uint_as_float(sc.x);
       d[1] *= __uint_as_float(sc.y);
     } else {
+      // 64-channel halves: thread t holds channels 16t .. 16t+15 of each
+      // (16-byte chunks 2t and 2t+1); odd rows read the two chunks in the
+      // other order, so the even and odd rows of a quarter-warp use even and
+      // odd chunks (disjoint banks), and a select puts them back in place
 #pragma unroll
-      for (int sp = 0; sp < D / 32; ++sp) {
-        const uint4 v = lds128(krow + 2 * (32 * sp + 8 * t));
-        mma_k16(d, qa[sp][0][0], 0u, qa[sp][0][1], 0u, v.x, v.y);
-        mma_k16(d, qa[sp][1][0], 0u, qa[sp][1][1], 0u, v.z, v.w);
+      for (int h = 0; h < D / 64; ++h) {
+        const int odd = g & 1;
+        const uint4 u0 = lds128(krow + 2 * (64 * h + 16 * t + 8 * odd));
+        const uint4 u1 = lds128(krow + 2 * (64 * h + 16 * t + 8 * (1 - odd)));
+        const uint4 v0 = odd ? u1 : u0, v1 = odd ? u0 : u1;
+        mma_k16(d, qa[2 * h][0][0], 0u, qa[2 * h][0][1], 0u, v0.x, v0.y);
+        mma_k16(d, qa[2 * h][1][0], 0u, qa[2 * h][1][1], 0u, v0.z, v0.w);
+        mma_k16(d, qa[2 * h + 1][0][0], 0u, qa[2 * h + 1][0][1], 0u, v1.x, v1.y);
+        mma_k16(d, qa[2 * h + 1][1][0], 0u, qa[2 * h + 1][1][1], 0u, v1.z, v1.w);
       }
     }
     s[nt][0] = tok < valid ? d[0] * scale_log2 : -INFINITY;
@@ -266,8 +287,11 @@ __device__ __forceinline__ void attn_stage(const uint8_t* stage, int valid, cons
 //
 // QK: S(16 x 8 tokens) = Qg(16 x d) . K^T, rows 0..G-1 of Qg hold the group's
 // queries (rows G..15 zero), K rows come from shared memory; the k index is
-// permuted exactly as in the routing kernel so each thread's B fragment is a
-// 16-byte load.  The S fragment (row g = head, columns 2t, 2t+1 = tokens) is
+// permuted so that thread t holds channels 16t .. 16t+15 of each 64-channel
+// half of a key row (two 16-byte loads; MMA j of half h takes channels
+// 64h + 16t + 4j .. +3 on both operands), and odd rows load the two chunks
+// in swapped order, so the two rows a quarter-warp reads use disjoint
+// banks.  The S fragment (row g = head, columns 2t, 2t+1 = tokens) is
 // already the A fragment layout of the next product, so the probabilities
 // never leave registers.
 // PV: acc(16 x r) += Pg(16 x 16 tokens) . Z(16 tokens x r); row g of Pg holds
@@ -348,7 +372,7 @@ template <int G, int D, int RR, int TPS, bool K8 = false>
 __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_constant__ AttnArgs a) {
   static_assert(G >= 1 && G <= 8, "GQA group must be 1..8");
   static_assert(D % 32 == 0 && RR % 8 == 0 && TPS % 16 == 0, "shape");
-  static_assert(!K8 || D % 64 == 0, "int8 keys need d % 64 == 0");
+  static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
   constexpr int DS = D / 32;     // 32-wide spans of the head dim
   constexpr int RT = RR / 8;     // n8 tiles of the latent
   constexpr int KB = K8 ? 1 : 2; // bytes per key element
@@ -418,14 +442,23 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
         qa[2 * sp + 1][1][1] = h2(v1.w);
       }
     } else {
+      // bf16 pairs of channels 64*h + 16*t + [0, 16): MMA j of half h takes
+      // (c, c+1) and (c+2, c+3) with c = 64*h + 16*t + 4*j, as the keys do
 #pragma unroll
-      for (int s = 0; s < DS; ++s) {
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (g < G) v = __ldg(reinterpret_cast<const uint4*>(qrow + 32 * s + 8 * t));
-        qa[s][0][0] = v.x;
-        qa[s][0][1] = v.y;
-        qa[s][1][0] = v.z;
-        qa[s][1][1] = v.w;
+      for (int h = 0; h < D / 64; ++h) {
+        uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
+        if (g < G) {
+          v0 = __ldg(reinterpret_cast<const uint4*>(qrow + 64 * h + 16 * t));
+          v1 = __ldg(reinterpret_cast<const uint4*>(qrow + 64 * h + 16 * t + 8));
+        }
+        qa[2 * h][0][0] = v0.x;
+        qa[2 * h][0][1] = v0.y;
+        qa[2 * h][1][0] = v0.z;
+        qa[2 * h][1][1] = v0.w;
+        qa[2 * h + 1][0][0] = v1.x;
+        qa[2 * h + 1][0][1] = v1.y;
+        qa[2 * h + 1][1][0] = v1.z;
+        qa[2 * h + 1][1][1] = v1.w;
       }
     }
   };
