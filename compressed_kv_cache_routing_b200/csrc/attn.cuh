@@ -573,11 +573,12 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
     }
     last = __shfl_sync(0xffffffffu, last, 0);
     if (last) {
+      const float* bv = a.b_v + (size_t)at.kvh * RR * D;
       MergeOut<G, RR> mo;
       merge_all<G, RR>(a.part_ml + (size_t)u * a.np_cap * G * 2, a.part_acc + (size_t)u * a.np_cap * G * RR,
                        min(np, a.np_cap), mo);
       if (a.latent) finish_unit_latent<G, RR>(mo, a.out + (size_t)u * G * RR);
-      else finish_unit<G, RR, D>(mo, a.b_v + (size_t)at.kvh * RR * D, a.out + (size_t)u * G * D, zbar);
+      else finish_unit<G, RR, D>(mo, bv, a.out + (size_t)u * G * D, zbar);
       if (lane == 0) a.counters[u] = 0u;
     }
   };

@@ -115,6 +115,21 @@ __device__ void merge_partials(const float* ml, const float* acc, int cnt, Merge
   static_assert(RR % 4 == 0 && 32 % G == 0, "shape");
   constexpr int V = MergeOut<G, RR>::V, VPL = MergeOut<G, RR>::VPL;
   const int lane = threadIdx.x & 31;
+  constexpr int JB = VPL >= 4 ? 4 : 8;  // chunks whose slices are loaded together (<= 16 float4 in flight)
+  // the first group's latent slices are requested before the (m, l) pairs,
+  // so both arrive in one L2 round trip
+  float4 x[JB][VPL];
+  auto load_group = [&](int j0) {
+#pragma unroll
+    for (int jj = 0; jj < JB; ++jj)
+#pragma unroll
+      for (int k = 0; k < VPL; ++k) {
+        const int j = j0 + jj, v = lane + 32 * k;
+        x[jj][k] = (j < cnt && v < V) ? __ldcg(reinterpret_cast<const float4*>(acc + (size_t)j * G * RR) + v)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+  };
+  load_group(0);
   // pairs q = lane and lane + 32: chunk q / G, head q % G (= lane % G)
   float mA = -INFINITY, lA = 0.f, mB = -INFINITY, lB = 0.f;
   if (lane < cnt * G) {
@@ -138,19 +153,10 @@ __device__ void merge_partials(const float* ml, const float* acc, int cnt, Merge
   o.L = L;
 #pragma unroll
   for (int k = 0; k < VPL; ++k) o.acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-  constexpr int JB = VPL >= 4 ? 4 : 8;  // chunks whose slices are loaded together (<= 16 float4 in flight)
 #pragma unroll
   for (int j0 = 0; j0 < 8; j0 += JB) {
     if (j0 >= cnt) break;
-    float4 x[JB][VPL];
-#pragma unroll
-    for (int jj = 0; jj < JB; ++jj)
-#pragma unroll
-      for (int k = 0; k < VPL; ++k) {
-        const int j = j0 + jj, v = lane + 32 * k;
-        x[jj][k] = (j < cnt && v < V) ? __ldcg(reinterpret_cast<const float4*>(acc + (size_t)j * G * RR) + v)
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+    if (j0 > 0) load_group(j0);
 #pragma unroll
     for (int jj = 0; jj < JB; ++jj) {
       const int j = j0 + jj;
