@@ -142,6 +142,37 @@ def test_small_parity(name):
         assert np.all(np.isneginf(sc[b, :, n[b]:]))
 
 
+def test_claimed_routing_chunks_score_every_page():
+    """Units of 512 pages and more: the routing grid hands out a quarter of
+    the pages in chunks claimed at run time.  Every page's score must be
+    written on every call, whichever warp claims it: the score buffer is
+    poisoned before each call, and two calls with different queries on one
+    handle must each match the oracle's scores page for page."""
+    spec = W.shrink("llama3_8b_decode", batch=3, len_lo=560 * 64, len_hi=700 * 64, topk=16)
+    w = W.generate(spec, device="cuda")
+    assert w.num_pages.max() >= 512
+    kv = bk.BasisKV.for_workload(w, max_topk=16)
+    B, n = len(w.seq_lens), w.num_pages
+    for call in range(2):
+        if call == 1:
+            w.q = (w.q * 0.5).contiguous()  # exact in bf16: every score halves, the order stays
+        sc = torch.full((B, w.spec.num_kv_heads, w.page_table.shape[1]), float("nan"), device="cuda")
+        sel = torch.full((B, w.spec.num_kv_heads, 16), -7, device="cuda", dtype=torch.int32)
+        bk.basiskv_route(kv.handle, w.q, 16, sc, sel)
+        torch.cuda.synchronize()
+        assert bk.basiskv_get_status(kv.handle) == 0
+        got = sc.cpu().numpy()
+        _, ref_sel, ref_sc, _ = oracle.decode(to_problem(w, topk=16), want_scores=True)
+        for b in range(B):
+            a, r = got[b, :, :n[b]], ref_sc[b, :, :n[b]]
+            assert np.isfinite(a).all(), (call, b)
+            assert np.all(np.abs(a - r) <= SCORE_TOL * np.maximum(1.0, np.abs(r))), (call, b)
+        assert np.array_equal(sel.cpu().numpy(), ref_sel), call
+        out, dsel = gpu_decode(w, kv=kv)
+        assert np.array_equal(dsel, ref_sel), call
+    kv.close()
+
+
 FULL = ["tiny", "llama3_8b_decode", "long_context", "high_concurrency", "dense_limit"]
 
 
