@@ -187,10 +187,16 @@ BASISKV_API int basiskv_load_page_table(basiskv_handle *h, int batch, const int3
  *            is skipped
  *   out      [batch][Hkv*G][d] fp32 (device)
  *   sel_out  [batch][Hkv][topk] int32 or NULL (device)
- * Enqueues the routing kernel (scores, fused top-k) and the attention
- * kernel (split exact QK + softmax + latent sum, fused combine and B_v) on
- * `stream`; no allocation, no host synchronisation.  A sequence of length 0
- * gets out = 0 and sel = -1.  Device-detected faults set status bits.
+ * Enqueues the routing grid (page scores), the selection grid (top-k; on
+ * the CUDA-core path the routing grid selects itself) and the attention
+ * grid (exact QK on the selected pages, softmax, latent sum, merge of the
+ * split partials and B_v) on `stream`, the later grids by programmatic
+ * dependent launch; no allocation, no host synchronisation.  A sequence of
+ * length 0 gets out = 0 and sel = -1.  Device-detected faults set status
+ * bits.  Calls on one handle share its scratch: keep them in one stream
+ * order (one stream, or events between streams).  A call is not meant for
+ * CUDA-graph capture: its work plan and a per-call tag travel in the kernel
+ * parameters, which a replayed graph would repeat unchanged.
  * Errors: INVALID_ARG. */
 BASISKV_API int basiskv_decode_attn(basiskv_handle *h, int batch, const void *q, int topk,
                         float softmax_scale, float *out, int32_t *sel_out,

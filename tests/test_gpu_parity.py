@@ -346,6 +346,33 @@ def test_deterministic_and_host_entry_point():
     kv.close()
 
 
+def test_two_handles_on_two_streams():
+    """Handles keep their own scratch and claim counters: two handles
+    decoding on two streams at the same time, several calls each with no
+    synchronisation in between, both stay equal to the oracle."""
+    ws = [W.generate(W.shrink("llama3_8b_decode", batch=4, len_lo=40000, len_hi=42000, topk=24), device="cuda"),
+          W.generate(SMALL["high_concurrency"], device="cuda")]
+    kvs = [bk.BasisKV.for_workload(w) for w in ws]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs, sels = [], []
+    for w in ws:
+        s = w.spec
+        outs.append(torch.full((s.batch, s.num_q_heads, s.head_dim), float("nan"), device="cuda"))
+        sels.append(torch.full((s.batch, s.num_kv_heads, s.topk), -7, device="cuda", dtype=torch.int32))
+    torch.cuda.synchronize()
+    for _ in range(5):
+        for w, kv, st, o, sl in zip(ws, kvs, streams, outs, sels):
+            bk.basiskv_decode_attn(kv.handle, w.q, w.spec.topk, w.spec.softmax_scale, o, sl,
+                                   stream=st.cuda_stream)
+    torch.cuda.synchronize()
+    for w, kv, o, sl in zip(ws, kvs, outs, sels):
+        assert bk.basiskv_get_status(kv.handle) == 0
+        ref_out, ref_sel, _, _ = oracle.decode(to_problem(w))
+        assert np.array_equal(sl.cpu().numpy(), ref_sel)
+        assert out_error(o.cpu().numpy(), ref_out) <= OUT_TOL
+        kv.close()
+
+
 def test_incremental_page_table_matches_bulk_load():
     w = W.generate(SMALL["high_concurrency"], device="cuda")
     s = w.spec
