@@ -167,6 +167,7 @@ struct basiskv_handle {
   int32_t* d_page_table = nullptr;  // [max_batch][max_pages]
   int32_t* d_seq_lens = nullptr;    // [max_batch]
   float* d_scores = nullptr;        // [max_batch][Hkv][max_pages]
+  uint64_t* d_scores64 = nullptr;   // [max_batch][Hkv][max_pages] scores tagged with the routing call
   int32_t* d_sel = nullptr;         // [max_batch][Hkv][max_topk]
   float* d_part_ml = nullptr;       // [max_batch*Hkv][kPartsCap][G][2]
   float* d_part_acc = nullptr;      // [max_batch*Hkv][kPartsCap][G][r]
@@ -332,6 +333,7 @@ struct LaunchPlan {
   // persistent kernels
   int route_ctas = 0, attn_ctas = 0;
   int route_static_pct = 100;  // pages of the persistent routing grid handed out in static shares
+  int max_routed = 0;          // pages of the longest routed sequence
   // work plans (prefix over sequences), when batch <= kPlanMax
   std::vector<int32_t> route_off, attn_off;
 };
@@ -372,6 +374,7 @@ LaunchPlan plan(const basiskv_handle* h, int batch, int topk, bool force_route) 
   // ends of the warps.  Short units gain nothing from it (each claimed
   // chunk starts a new unit, whose folded query must be fetched first).
   lp.route_static_pct = max_routed >= 512 ? kRouteStaticPct : 100;
+  lp.max_routed = max_routed;
 
   // generic kernels: a grid of (chunk | split, Hkv, batch)
   if (lp.any_routed) {
@@ -444,6 +447,8 @@ RouteArgs route_args(basiskv_handle* h, const LaunchPlan& lp, const void* q, int
   a.page_table = h->d_page_table;
   a.seq_lens = h->d_seq_lens;
   a.scores = scores;
+  a.scores64 = h->d_scores64;
+  a.tagged_scores = 0;
   a.sel = h->d_sel;
   a.sel_out = sel_out;
   a.counters = h->d_counters;
@@ -509,10 +514,14 @@ int launch_route(basiskv_handle* h, const LaunchPlan& lp, const RouteArgs& a, bo
 
 // Selection for the persistent routing kernel (PDL behind it).
 int launch_topk(basiskv_handle* h, const LaunchPlan& lp, int topk, const float* scores, int32_t* sel_out,
-                int force, bool pdl, cudaStream_t stream) {
+                int force, bool pdl, bool poll, cudaStream_t stream) {
   const basiskv_params& p = h->p;
   TopkArgs a;
   a.scores = scores;
+  a.scores64 = h->d_scores64;
+  a.poll = poll;
+  a.tag = h->route_tag;
+  a.status = h->d_status;
   a.seq_lens = h->d_seq_lens;
   a.sel = h->d_sel;
   a.sel_out = sel_out;
@@ -639,6 +648,7 @@ int basiskv_create(const basiskv_params* p, basiskv_handle** out) {
       {(void**)&h->d_page_table, sizeof(int32_t) * B * p->max_pages_per_seq},
       {(void**)&h->d_seq_lens, sizeof(int32_t) * B},
       {(void**)&h->d_scores, sizeof(float) * U * p->max_pages_per_seq},
+      {(void**)&h->d_scores64, sizeof(uint64_t) * U * p->max_pages_per_seq},
       {(void**)&h->d_sel, sizeof(int32_t) * U * p->max_topk},
       {(void**)&h->d_part_ml, sizeof(float) * U * kPartsCap * G * 2},
       {(void**)&h->d_part_acc, sizeof(float) * U * kPartsCap * G * p->rank_r},
@@ -662,6 +672,7 @@ int basiskv_create(const basiskv_params* p, basiskv_handle** out) {
       cudaMemset(h->d_seq_lens, 0, sizeof(int32_t) * B) != cudaSuccess ||
       cudaMemset(h->d_counters, 0, sizeof(uint32_t) * (3 * U + kSchedWords)) != cudaSuccess ||
       cudaMemset(h->d_qf, 0, sizeof(uint64_t) * U * G * (p->rank_r + p->rank_s)) != cudaSuccess ||
+      cudaMemset(h->d_scores64, 0, sizeof(uint64_t) * U * p->max_pages_per_seq) != cudaSuccess ||
       cudaMemset(h->d_status, 0, sizeof(uint32_t)) != cudaSuccess)
     return cleanup_fail(BASISKV_ERR_CUDA, "cudaMemset failed");
   h->h_table.assign(B * p->max_pages_per_seq, 0);
@@ -706,7 +717,7 @@ int basiskv_destroy(basiskv_handle* h) {
   cudaDeviceSynchronize();
   void* ptrs[] = {h->d_page_table, h->d_seq_lens, h->d_scores, h->d_sel, h->d_part_ml, h->d_part_acc,
                   h->d_counters, h->d_status, h->d_q_stage, h->d_out_stage, h->d_sel_stage,
-                  h->d_route_off, h->d_attn_off, h->d_qf, h->d_enc};
+                  h->d_route_off, h->d_attn_off, h->d_qf, h->d_scores64, h->d_enc};
   for (void* q : ptrs)
     if (q) cudaFree(q);
   for (cudaEvent_t e : h->events) cudaEventDestroy(e);
@@ -856,14 +867,19 @@ static int decode_step(basiskv_handle* h, int batch, const void* q, int topk, fl
   }
   if (prof) CUDA_TRY(cudaEventRecord(ev[1], st));
   // the first grid of a call never overlaps the caller's previous work
+  // The tensor-core routing grid tags its scores with the call, and the
+  // selection grid then takes each unit as soon as its scores are all
+  // there (the selection kernel's shared memory holds the longest unit).
+  const bool poll = route_tc && lp.max_routed <= h->topk_keys;
   if (lp.any_routed) {
     RouteArgs ra = route_args(h, lp, q, topk, h->d_scores, sel_out, 0);
+    ra.tagged_scores = poll;
     rc = launch_route(h, lp, ra, use_prep && !prof, st);
     if (rc) return rc;
   }
   if (prof) CUDA_TRY(cudaEventRecord(ev[2], st));
   if (route_tc) {
-    rc = launch_topk(h, lp, topk, h->d_scores, sel_out, 0, !prof, st);
+    rc = launch_topk(h, lp, topk, h->d_scores, sel_out, 0, !prof, poll, st);
     if (rc) return rc;
   }
   if (prof) CUDA_TRY(cudaEventRecord(ev[3], st));
@@ -1079,7 +1095,7 @@ int basiskv_route(basiskv_handle* h, int batch, const void* q, int topk, float* 
   RouteArgs ra = route_args(h, lp, q, topk, scores, sel_out, 1);
   rc = launch_route(h, lp, ra, true, st);
   if (rc || !h->route_fn) return rc;
-  return launch_topk(h, lp, topk, scores, sel_out, 1, true, st);
+  return launch_topk(h, lp, topk, scores, sel_out, 1, true, false, st);
 }
 
 int basiskv_get_status(basiskv_handle* h, uint32_t* status, int clear) {

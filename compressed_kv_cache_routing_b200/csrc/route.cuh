@@ -35,6 +35,8 @@ struct RouteArgs {
   const int32_t* page_table;  // [B][ld_pt]
   const int32_t* seq_lens;  // [B]
   float* scores;            // [B][Hkv][ld_pt]
+  uint64_t* scores64;       // [B][Hkv][ld_pt] (tag << 32) | fp32 bits, when tagged_scores
+  int tagged_scores;        // persistent kernel: write scores64 instead of scores
   int32_t* sel;             // [B][Hkv][ld_sel]
   int32_t* sel_out;         // [B][Hkv][topk] or null
   uint32_t* counters;       // [B][Hkv]
@@ -150,7 +152,9 @@ __device__ void route_finish(const RouteArgs& a, const RouteUnit& ru, TopkSmem& 
 // (sequence-major, then KV head, then page), claimed from a grid-wide
 // counter, through its own ring of `stages` shared buffers filled by bulk
 // copies (cp.async.bulk, L2 evict-first) completing on mbarriers, and writes
-// one score per page.  The selection runs in the next grid (topk_kernel).
+// one score per page (tagged with the call, so the selection grid can take
+// a unit as soon as its pages are scored).  The selection runs in the next
+// grid (topk_kernel).
 template <int G, int RR, int RS>
 struct RouteMma {
   static constexpr int NT = (2 * G + 7) / 8;  // n8 tiles of (hi, lo) columns
@@ -741,7 +745,13 @@ __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_c
         }
         const __nv_bfloat16* zs = reinterpret_cast<const __nv_bfloat16*>(stage + k * page_bytes);
         const float best = route_page_score<G, RR, RS, P, FR>(zs, zs + P * RR, min(P, cc.L - cc.j * P), fr);
-        if (lane == 0) a.scores[(size_t)cur_u * a.ld_pt + cc.j] = best;
+        if (lane == 0) {
+          if (a.tagged_scores)
+            st_relaxed_u64(a.scores64 + (size_t)cur_u * a.ld_pt + cc.j,
+                           ((uint64_t)a.tag << 32) | __float_as_uint(best));
+          else
+            a.scores[(size_t)cur_u * a.ld_pt + cc.j] = best;
+        }
         cc.advance(a);
       }
     }

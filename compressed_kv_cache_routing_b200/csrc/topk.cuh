@@ -148,10 +148,14 @@ namespace basiskv {
 // compaction compares keys on those bits only and the set is the same.
 struct TopkArgs {
   const float* scores;     // [B][Hkv][ld_pt]
+  const uint64_t* scores64;  // [B][Hkv][ld_pt] (tag << 32) | fp32 bits, when poll
   const int32_t* seq_lens; // [B]
   int32_t* sel;            // [B][Hkv][ld_sel]
   int32_t* sel_out;        // [B][Hkv][topk] or null
+  uint32_t* status;
   int num_kv_heads, page_size, ld_pt, ld_sel, topk, force, keys_cap;
+  int poll;                // read tagged scores as they come, without waiting for the routing grid
+  uint32_t tag;            // the routing call's tag (poll)
 };
 
 constexpr int kTopkThreads = 256;
@@ -163,7 +167,13 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkArgs a) {
   const int b = blockIdx.y, kvh = blockIdx.x, u = b * a.num_kv_heads + kvh;
   const int n = (a.seq_lens[b] + a.page_size - 1) / a.page_size;
   if (n == 0 || !(a.force || a.topk < n)) return;
-  pdl_wait_primary();  // the scores come from the routing grid
+  // The scores come from the routing grid.  When they carry the call's tag
+  // (poll) a CTA does not wait for the whole routing grid: it reads its
+  // unit's scores until every one carries the tag, so units whose pages
+  // are all scored are selected while the routing grid still streams
+  // others.  Each 8-byte word is written and read atomically, so a tagged
+  // word holds this call's score.
+  if (!a.poll) pdl_wait_primary();
   const float* sc = a.scores + (size_t)u * a.ld_pt;
   int32_t* sel = a.sel + (size_t)u * a.ld_sel;
   int32_t* so = a.sel_out ? a.sel_out + (size_t)u * a.topk : nullptr;
@@ -172,7 +182,26 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkArgs a) {
     return;
   }
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int i = tid; i < n; i += kTopkThreads) keys[i] = score_key(__ldcg(sc + i));
+  if (a.poll) {
+    const uint64_t* sc64 = a.scores64 + (size_t)u * a.ld_pt;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+      bool ok = true;
+      for (int i = tid; i < n; i += kTopkThreads) {
+        const uint64_t w = ld_relaxed_u64(sc64 + i);
+        ok = ok && (uint32_t)(w >> 32) == a.tag;
+        keys[i] = score_key(__uint_as_float((uint32_t)w));
+      }
+      if (__syncthreads_and(ok)) break;
+      if (__syncthreads_or(global_timer_ns() - t0 > kWaitLimitNs)) {
+        if (tid == 0) atomicOr(a.status, kStatusTimeout);
+        break;
+      }
+      __nanosleep(512);
+    }
+  } else {
+    for (int i = tid; i < n; i += kTopkThreads) keys[i] = score_key(__ldcg(sc + i));
+  }
   __syncthreads();
   const int kb = a.topk < n ? a.topk : n;
   uint32_t thr = 0u, tmask = 0xFFFFFFFFu;  // keys compare on their bits under tmask
