@@ -60,6 +60,8 @@ struct AttnArgs {
   const int32_t* page_table; // [B][ld_pt]
   const int32_t* seq_lens;   // [B]
   const int32_t* sel;        // [B][Hkv][ld_sel] (routed units)
+  const uint64_t* sel64;     // [B][Hkv][ld_sel] (tag << 32) | page, or null (persistent kernel)
+  uint32_t sel_tag;          // the tag of this call's selection (sel64)
   int32_t* sel_out;          // [B][Hkv][topk] or null
   float* part_ml;            // [B*Hkv][np_cap][G][2]
   float* part_acc;           // [B*Hkv][np_cap][G][r]
@@ -308,6 +310,21 @@ __device__ __forceinline__ void attn_stage(const uint8_t* stage, int valid, cons
 // scale multiplies its dot product before the softmax.  At the end of its segment of a unit a
 // warp writes one partial (m, l, acc); the warp that completes the unit
 // merges the partials and applies B_v.
+// A tagged selection entry whose unit is still being selected: wait for it
+// (bounded; on expiry the status says TIMEOUT and entry 0 is used).
+__device__ __noinline__ uint64_t wait_selected(const uint64_t* src, uint32_t tag, uint32_t* status) {
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    __nanosleep(256);
+    const uint64_t w = ld_relaxed_u64(src);
+    if ((uint32_t)(w >> 32) == tag) return w;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(status, kStatusTimeout);
+      return 0;
+    }
+  }
+}
+
 struct AttnCursor {
   int b, kvh, jj, ts, n, kb, L;
   int uoff;            // flat index of the unit's first item
@@ -352,14 +369,28 @@ struct AttnCursor {
     }
   }
   __device__ __forceinline__ int unit(const AttnArgs& a) const { return b * a.num_kv_heads + kvh; }
-  __device__ __forceinline__ int page(const AttnArgs& a) const { return checked(a, page_raw(a)); }
-  // The selected page, unchecked: the load stays in flight until the value
-  // is used (check it with checked() when the item is issued).
-  __device__ __forceinline__ int page_raw(const AttnArgs& a) const {
-    if (a.topk >= n) return jj;
-    return __ldcg(a.sel + (size_t)unit(a) * a.ld_sel + jj);
+  template <bool TS>
+  __device__ __forceinline__ int page(const AttnArgs& a) const { return checked<TS>(a, page_raw<TS>(a)); }
+  // The selected entry, unchecked: the load stays in flight until the value
+  // is used (check it with checked() when the item is issued).  A tagged
+  // entry (TS: sel64) carries the tag of the call whose selection wrote it.
+  template <bool TS>
+  __device__ __forceinline__ auto page_raw(const AttnArgs& a) const {
+    if constexpr (TS) {
+      if (a.topk >= n) return (uint64_t)jj;
+      return ld_relaxed_u64(a.sel64 + (size_t)unit(a) * a.ld_sel + jj);
+    } else {
+      if (a.topk >= n) return jj;
+      return __ldcg(a.sel + (size_t)unit(a) * a.ld_sel + jj);
+    }
   }
-  __device__ __forceinline__ int checked(const AttnArgs& a, int p) const {
+  template <bool TS, typename Word>
+  __device__ __forceinline__ int checked(const AttnArgs& a, Word w) const {
+    if constexpr (TS) {
+      if (a.topk < n && (uint32_t)(w >> 32) != a.sel_tag)
+        w = wait_selected(a.sel64 + (size_t)unit(a) * a.ld_sel + jj, a.sel_tag, a.status);
+    }
+    int p = (int)(uint32_t)w;
     if (p < 0 || p >= n) {
       atomicOr(a.status, kStatusBadPage);
       p = 0;
@@ -368,7 +399,9 @@ struct AttnCursor {
   }
 };
 
-template <int G, int D, int RR, int TPS, bool K8 = false>
+// TS: the selection comes as tagged entries (sel64) from a selection grid
+// that this grid does not wait for as a whole.
+template <int G, int D, int RR, int TPS, bool K8 = false, bool TS = false>
 __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_constant__ AttnArgs a) {
   static_assert(G >= 1 && G <= 8, "GQA group must be 1..8");
   static_assert(D % 32 == 0 && RR % 8 == 0 && TPS % 16 == 0, "shape");
@@ -467,7 +500,9 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
     cur_u = cc.unit(a);
     load_q(cur_u);
   }
-  pdl_wait_primary();  // the selection is written by the previous grid
+  // The selection is written by the previous grid: wait for that grid, or,
+  // with a tagged selection, for each unit's entries as they are needed.
+  if constexpr (!TS) pdl_wait_primary();
   if (count <= 0) return;
 
   const uint8_t* kpool = static_cast<const uint8_t*>(a.k_pool);
@@ -497,7 +532,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
     ic.advance(a, sub);
   };
   AttnCursor ia;       // lane 0: the item after the next one to issue
-  int next_page = 0;   // lane 0: page of the next item to issue
+  using SelWord = decltype(ic.page_raw<TS>(a));
+  SelWord next_page = 0;  // lane 0: selected entry of the next item to issue (loaded, unchecked)
   {
     // the first S items: lane j looks item j up (all lookups in parallel),
     // lane 0 issues them in order
@@ -506,7 +542,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
     if (lane < first) {
       AttnCursor c = ic;
       for (int k = 0; k < lane; ++k) c.advance(a, sub);
-      pg = c.page(a);
+      pg = c.page<TS>(a);
       sl = __ldg(a.page_table + (size_t)c.b * a.ld_pt + pg);
     }
     for (int i = 0; i < first; ++i) {
@@ -516,7 +552,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
   }
   if (lane == 0) {
     if (S < count) {
-      next_page = ic.page_raw(a);
+      next_page = ic.page_raw<TS>(a);
       ia = ic;
       ia.advance(a, sub);
     }
@@ -588,15 +624,16 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
   int s_i = 0;        // ring position of item i (i mod S)
   uint32_t ph_i = 0;  // phase parity of that position's barrier for item i
   for (; i < count; ++i) {
-    int next_slot = 0, page_after = 0;
+    int next_pg = 0, next_slot = 0;
+    SelWord page_after = 0;
     if (lane == 0) {
       // the page of item i + S was read one iteration ago: check it and read
       // its slot now; the page of the item after it stays in flight
       if (i + S < count) {
-        next_page = ic.checked(a, next_page);
-        next_slot = slot_of(next_page);
+        next_pg = ic.checked<TS>(a, next_page);
+        next_slot = slot_of(next_pg);
       }
-      if (i + S + 1 < count) page_after = ia.page_raw(a);
+      if (i + S + 1 < count) page_after = ia.page_raw<TS>(a);
     }
     const int u = cc.unit(a);
     if (u != cur_u) {
@@ -617,7 +654,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
     ++seg;
     __syncwarp();
     if (lane == 0 && i + S < count) {
-      issue(i + S, s_i, next_page, next_slot);  // (i + S) mod S = i mod S
+      issue(i + S, s_i, next_pg, next_slot);  // (i + S) mod S = i mod S
       next_page = page_after;
       ia.advance(a, sub);
     }

@@ -54,6 +54,10 @@ constexpr size_t kAttnSmemBudgetWide = 64 * 1024;  // attention rings when r >= 
 
 using KernelFn = void (*)(const RouteArgs);
 using AttnFn = void (*)(const AttnArgs);
+struct AttnFns {
+  AttnFn plain;   // waits for the selection grid
+  AttnFn tagged;  // reads tagged selection entries as they come
+};
 
 // ---- compiled tensor-core shapes ------------------------------------------
 struct RouteKey {
@@ -86,10 +90,12 @@ const std::map<RouteKey, KernelFn>& route_table() {
   return t;
 }
 
-const std::map<AttnKey, AttnFn>& attn_table() {
-  static const std::map<AttnKey, AttnFn> t = {
-#define AK(G, D, R, T) {AttnKey{G, D, R, T, false}, &attn_mma_kernel<G, D, R, T, false>}
-#define AK8(G, D, R, T) {AttnKey{G, D, R, T, true}, &attn_mma_kernel<G, D, R, T, true>}
+const std::map<AttnKey, AttnFns>& attn_table() {
+  static const std::map<AttnKey, AttnFns> t = {
+#define AK(G, D, R, T) \
+  {AttnKey{G, D, R, T, false}, AttnFns{&attn_mma_kernel<G, D, R, T, false, false>, &attn_mma_kernel<G, D, R, T, false, true>}}
+#define AK8(G, D, R, T) \
+  {AttnKey{G, D, R, T, true}, AttnFns{&attn_mma_kernel<G, D, R, T, true, false>, &attn_mma_kernel<G, D, R, T, true, true>}}
 #ifdef BASISKV_WAIT_TEST
       AK(4, 128, 32, 32), AK(4, 128, 32, 64),
 #else
@@ -168,6 +174,7 @@ struct basiskv_handle {
   int32_t* d_seq_lens = nullptr;    // [max_batch]
   float* d_scores = nullptr;        // [max_batch][Hkv][max_pages]
   uint64_t* d_scores64 = nullptr;   // [max_batch][Hkv][max_pages] scores tagged with the routing call
+  uint64_t* d_sel64 = nullptr;      // [max_batch][Hkv][max_topk] selection tagged with the routing call
   int32_t* d_sel = nullptr;         // [max_batch][Hkv][max_topk]
   float* d_part_ml = nullptr;       // [max_batch*Hkv][kPartsCap][G][2]
   float* d_part_acc = nullptr;      // [max_batch*Hkv][kPartsCap][G][r]
@@ -189,7 +196,8 @@ struct basiskv_handle {
   std::vector<int32_t> h_npages;
   // kernels chosen at create
   KernelFn route_fn = nullptr;
-  AttnFn attn_fn = nullptr;
+  AttnFn attn_fn = nullptr;         // persistent attention, waiting for the selection grid
+  AttnFn attn_fn_ts = nullptr;      // the same reading tagged selection entries
   int attn_tps = 0;
   int route_stages = 0, attn_stages = 0;
   size_t route_smem = 0, attn_smem = 0;
@@ -270,7 +278,8 @@ void choose_kernels(basiskv_handle* h) {
       int st = (int)std::min<size_t>(4, budget / (kAttnWarps * stage));
       if (st < 1) continue;
       if (st < 2 && tps > 16) continue;  // prefer a smaller stage with double buffering
-      h->attn_fn = ait->second;
+      h->attn_fn = ait->second.plain;
+      h->attn_fn_ts = ait->second.tagged;
       h->attn_tps = tps;
       h->attn_stages = st;
       h->attn_smem = kAttnWarps * st * stage + sizeof(float) * kAttnWarps * p.gqa_group * p.rank_r;
@@ -520,6 +529,7 @@ int launch_topk(basiskv_handle* h, const LaunchPlan& lp, int topk, const float* 
   a.scores = scores;
   a.scores64 = h->d_scores64;
   a.poll = poll;
+  a.sel64 = poll ? h->d_sel64 : nullptr;
   a.tag = h->route_tag;
   a.status = h->d_status;
   a.seq_lens = h->d_seq_lens;
@@ -540,7 +550,7 @@ int launch_topk(basiskv_handle* h, const LaunchPlan& lp, int topk, const float* 
 }
 
 int launch_attn(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk, float scale, int latent,
-                float* out, int32_t* sel_out, bool pdl, cudaStream_t stream) {
+                float* out, int32_t* sel_out, bool pdl, bool tagged_sel, cudaStream_t stream) {
   const basiskv_params& p = h->p;
   const size_t U = (size_t)p.max_batch * p.num_kv_heads;
   AttnArgs a;
@@ -553,6 +563,8 @@ int launch_attn(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk
   a.page_table = h->d_page_table;
   a.seq_lens = h->d_seq_lens;
   a.sel = h->d_sel;
+  a.sel64 = tagged_sel ? h->d_sel64 : nullptr;
+  a.sel_tag = h->route_tag;
   a.sel_out = sel_out;
   a.part_ml = h->d_part_ml;
   a.part_acc = h->d_part_acc;
@@ -581,7 +593,7 @@ int launch_attn(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk
   cudaLaunchAttribute attr[1];
   if (h->attn_fn) {
     cudaLaunchConfig_t cfg = launch_cfg(dim3(lp.attn_ctas), kAttnThreads, h->attn_smem, stream, pdl, attr);
-    CUDA_TRY(cudaLaunchKernelEx(&cfg, h->attn_fn, a));
+    CUDA_TRY(cudaLaunchKernelEx(&cfg, tagged_sel ? h->attn_fn_ts : h->attn_fn, a));
     return BASISKV_OK;
   }
   cudaLaunchConfig_t cfg = launch_cfg(dim3(lp.attn_splits, p.num_kv_heads, lp.batch), kAttnThreads,
@@ -649,6 +661,7 @@ int basiskv_create(const basiskv_params* p, basiskv_handle** out) {
       {(void**)&h->d_seq_lens, sizeof(int32_t) * B},
       {(void**)&h->d_scores, sizeof(float) * U * p->max_pages_per_seq},
       {(void**)&h->d_scores64, sizeof(uint64_t) * U * p->max_pages_per_seq},
+      {(void**)&h->d_sel64, sizeof(uint64_t) * U * p->max_topk},
       {(void**)&h->d_sel, sizeof(int32_t) * U * p->max_topk},
       {(void**)&h->d_part_ml, sizeof(float) * U * kPartsCap * G * 2},
       {(void**)&h->d_part_acc, sizeof(float) * U * kPartsCap * G * p->rank_r},
@@ -673,6 +686,7 @@ int basiskv_create(const basiskv_params* p, basiskv_handle** out) {
       cudaMemset(h->d_counters, 0, sizeof(uint32_t) * (3 * U + kSchedWords)) != cudaSuccess ||
       cudaMemset(h->d_qf, 0, sizeof(uint64_t) * U * G * (p->rank_r + p->rank_s)) != cudaSuccess ||
       cudaMemset(h->d_scores64, 0, sizeof(uint64_t) * U * p->max_pages_per_seq) != cudaSuccess ||
+      cudaMemset(h->d_sel64, 0, sizeof(uint64_t) * U * p->max_topk) != cudaSuccess ||
       cudaMemset(h->d_status, 0, sizeof(uint32_t)) != cudaSuccess)
     return cleanup_fail(BASISKV_ERR_CUDA, "cudaMemset failed");
   h->h_table.assign(B * p->max_pages_per_seq, 0);
@@ -683,15 +697,24 @@ int basiskv_create(const basiskv_params* p, basiskv_handle** out) {
   choose_kernels(h);
   int arc = h->route_fn ? set_smem_attr((const void*)h->route_fn, h->route_smem) : BASISKV_OK;
   if (!arc && h->attn_fn) arc = set_smem_attr((const void*)h->attn_fn, h->attn_smem);
+  if (!arc && h->attn_fn_ts) arc = set_smem_attr((const void*)h->attn_fn_ts, h->attn_smem);
   if (!arc)
     arc = set_smem_attr((const void*)&prep_kernel, 0);
   if (!arc) arc = set_smem_attr((const void*)&topk_kernel, sizeof(uint32_t) * (size_t)h->topk_keys);
   if (!arc && h->route_fn &&
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&h->route_occ, h->route_fn, kRouteThreads, h->route_smem) != cudaSuccess)
     arc = fail(BASISKV_ERR_CUDA, "occupancy query failed");
-  if (!arc && h->attn_fn &&
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&h->attn_occ, h->attn_fn, kAttnThreads, h->attn_smem) != cudaSuccess)
-    arc = fail(BASISKV_ERR_CUDA, "occupancy query failed");
+  if (!arc && h->attn_fn) {
+    // one grid size for both variants: the smaller residency of the two
+    int occ_ts = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&h->attn_occ, h->attn_fn, kAttnThreads, h->attn_smem) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_ts, h->attn_fn_ts, kAttnThreads, h->attn_smem) !=
+            cudaSuccess)
+      arc = fail(BASISKV_ERR_CUDA, "occupancy query failed");
+    else
+      h->attn_occ = std::min(h->attn_occ, occ_ts);
+  }
   h->route_occ = std::max(1, h->route_occ);
   h->attn_occ = std::max(1, h->attn_occ);
   if (!arc)
@@ -717,7 +740,7 @@ int basiskv_destroy(basiskv_handle* h) {
   cudaDeviceSynchronize();
   void* ptrs[] = {h->d_page_table, h->d_seq_lens, h->d_scores, h->d_sel, h->d_part_ml, h->d_part_acc,
                   h->d_counters, h->d_status, h->d_q_stage, h->d_out_stage, h->d_sel_stage,
-                  h->d_route_off, h->d_attn_off, h->d_qf, h->d_scores64, h->d_enc};
+                  h->d_route_off, h->d_attn_off, h->d_qf, h->d_scores64, h->d_sel64, h->d_enc};
   for (void* q : ptrs)
     if (q) cudaFree(q);
   for (cudaEvent_t e : h->events) cudaEventDestroy(e);
@@ -885,7 +908,7 @@ static int decode_step(basiskv_handle* h, int batch, const void* q, int topk, fl
   if (prof) CUDA_TRY(cudaEventRecord(ev[3], st));
   // PDL only behind a routing grid (which signals after any prep grid has
   // finished, so the plan is complete when this grid starts)
-  rc = launch_attn(h, lp, q, topk, softmax_scale, latent, out, sel_out, lp.any_routed && !prof, st);
+  rc = launch_attn(h, lp, q, topk, softmax_scale, latent, out, sel_out, lp.any_routed && !prof, poll, st);
   if (rc) return rc;
   if (prof) {
     CUDA_TRY(cudaEventRecord(ev[4], st));

@@ -152,6 +152,7 @@ struct TopkArgs {
   const int32_t* seq_lens; // [B]
   int32_t* sel;            // [B][Hkv][ld_sel]
   int32_t* sel_out;        // [B][Hkv][topk] or null
+  uint64_t* sel64;         // [B][Hkv][ld_sel] the selection tagged with the call, or null
   uint32_t* status;
   int num_kv_heads, page_size, ld_pt, ld_sel, topk, force, keys_cap;
   int poll;                // read tagged scores as they come, without waiting for the routing grid
@@ -176,6 +177,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkArgs a) {
   if (!a.poll) pdl_wait_primary();
   const float* sc = a.scores + (size_t)u * a.ld_pt;
   int32_t* sel = a.sel + (size_t)u * a.ld_sel;
+  uint64_t* sel64 = a.sel64 ? a.sel64 + (size_t)u * a.ld_sel : nullptr;
   int32_t* so = a.sel_out ? a.sel_out + (size_t)u * a.topk : nullptr;
   if (n > a.keys_cap) {
     block_topk<kTopkThreads>(sc, n, a.topk, sel, so, a.topk, sm);
@@ -284,6 +286,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkArgs a) {
       const uint32_t key = keys[i] & tmask;
       if (kb >= n || key > thr || (key == thr && e < need)) {
         sel[pos] = i;
+        if (sel64) st_relaxed_u64(sel64 + pos, ((uint64_t)a.tag << 32) | (uint32_t)i);
         if (so) so[pos] = i;
         ++pos;
       }
