@@ -76,6 +76,7 @@ struct AttnArgs {
   // persistent tensor-core kernel only
   int batch;
   const int32_t* attn_off;   // [B+1] prefix of attention items x Hkv (from the prep grid)
+  int chunk_items;           // cooperative kernel: items per chunk (0: one chunk per CTA)
   int plan_n;                // >= 0: plan_off holds attn_off (batch <= kPlanMax)
   int32_t plan_off[kPlanMax + 1];
 };
@@ -310,6 +311,37 @@ __device__ __forceinline__ void attn_stage(const uint8_t* stage, int valid, cons
 // scale multiplies its dot product before the softmax.  At the end of its segment of a unit a
 // warp writes one partial (m, l, acc); the warp that completes the unit
 // merges the partials and applies B_v.
+// This lane's query fragments for unit u (the group's G heads as rows g < G
+// of the A operand, zero rows for g >= G), in the k order of the key loads:
+// MMA j of 64-channel span h takes channels (c, c+1) and (c+2, c+3) with
+// c = 64*h + 16*t + 4*j.  Int8 keys meet the query rounded to f16.
+template <int G, int D, bool K8>
+__device__ __forceinline__ void load_q_frags(const AttnArgs& a, int u, uint32_t (&qa)[D / 32][2][2]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)u * G + (g < G ? g : 0)) * D;
+#pragma unroll
+  for (int h = 0; h < D / 64; ++h) {
+    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
+    if (g < G) {
+      v0 = __ldg(reinterpret_cast<const uint4*>(qrow + 64 * h + 16 * t));
+      v1 = __ldg(reinterpret_cast<const uint4*>(qrow + 64 * h + 16 * t + 8));
+    }
+    if constexpr (K8) {
+      auto h2 = [](uint32_t w) { return pack_f16(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
+      v0 = make_uint4(h2(v0.x), h2(v0.y), h2(v0.z), h2(v0.w));
+      v1 = make_uint4(h2(v1.x), h2(v1.y), h2(v1.z), h2(v1.w));
+    }
+    qa[2 * h][0][0] = v0.x;
+    qa[2 * h][0][1] = v0.y;
+    qa[2 * h][1][0] = v0.z;
+    qa[2 * h][1][1] = v0.w;
+    qa[2 * h + 1][0][0] = v1.x;
+    qa[2 * h + 1][0][1] = v1.y;
+    qa[2 * h + 1][1][0] = v1.z;
+    qa[2 * h + 1][1][1] = v1.w;
+  }
+}
+
 // A tagged selection entry whose unit is still being selected: wait for it
 // (bounded; on expiry the status says TIMEOUT and entry 0 is used).
 __device__ __noinline__ uint64_t wait_selected(const uint64_t* src, uint32_t tag, uint32_t* status) {
@@ -452,49 +484,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
   AttnCursor cc = ic;
 
   uint32_t qa[DS][2][2];
-  auto load_q = [&](int u) {
-    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)u * G + (g < G ? g : 0)) * D;
-    if constexpr (K8) {
-      // f16 pairs of channels 64*sp + 16*t + [0, 16): MMA j of span sp
-      // takes (c, c+1) and (c+2, c+3) with c = 64*sp + 16*t + 4*j
-      auto h2 = [](uint32_t w) { return pack_f16(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); };
-#pragma unroll
-      for (int sp = 0; sp < D / 64; ++sp) {
-        uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
-        if (g < G) {
-          v0 = __ldg(reinterpret_cast<const uint4*>(qrow + 64 * sp + 16 * t));
-          v1 = __ldg(reinterpret_cast<const uint4*>(qrow + 64 * sp + 16 * t + 8));
-        }
-        qa[2 * sp][0][0] = h2(v0.x);
-        qa[2 * sp][0][1] = h2(v0.y);
-        qa[2 * sp][1][0] = h2(v0.z);
-        qa[2 * sp][1][1] = h2(v0.w);
-        qa[2 * sp + 1][0][0] = h2(v1.x);
-        qa[2 * sp + 1][0][1] = h2(v1.y);
-        qa[2 * sp + 1][1][0] = h2(v1.z);
-        qa[2 * sp + 1][1][1] = h2(v1.w);
-      }
-    } else {
-      // bf16 pairs of channels 64*h + 16*t + [0, 16): MMA j of half h takes
-      // (c, c+1) and (c+2, c+3) with c = 64*h + 16*t + 4*j, as the keys do
-#pragma unroll
-      for (int h = 0; h < D / 64; ++h) {
-        uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
-        if (g < G) {
-          v0 = __ldg(reinterpret_cast<const uint4*>(qrow + 64 * h + 16 * t));
-          v1 = __ldg(reinterpret_cast<const uint4*>(qrow + 64 * h + 16 * t + 8));
-        }
-        qa[2 * h][0][0] = v0.x;
-        qa[2 * h][0][1] = v0.y;
-        qa[2 * h][1][0] = v0.z;
-        qa[2 * h][1][1] = v0.w;
-        qa[2 * h + 1][0][0] = v1.x;
-        qa[2 * h + 1][0][1] = v1.y;
-        qa[2 * h + 1][1][0] = v1.z;
-        qa[2 * h + 1][1][1] = v1.w;
-      }
-    }
-  };
+  auto load_q = [&](int u) { load_q_frags<G, D, K8>(a, u, qa); };
   int cur_u = -1;
   if (count > 0) {
     cur_u = cc.unit(a);

@@ -15,6 +15,7 @@
 
 #include "../../include/basiskv.h"
 #include "attn.cuh"
+#include "attn_coop.cuh"
 #include "encode.cuh"
 #include "plan.cuh"
 #include "route.cuh"
@@ -51,6 +52,10 @@ constexpr int kRouteStaticPct = 75;  // routing pages in static shares when unit
 constexpr size_t kRouteSmemBudget = 48 * 1024;
 constexpr size_t kAttnSmemBudget = 100 * 1024;
 constexpr size_t kAttnSmemBudgetWide = 64 * 1024;  // attention rings when r >= 64
+// Cooperative attention: one CTA per SM; its ring takes what is left of the
+// SM's shared memory after the merge buffers.
+constexpr size_t kCoopSmemPerSm = 212 * 1024;
+constexpr long long kCoopMinItems = 8;  // items per CTA at least
 
 using KernelFn = void (*)(const RouteArgs);
 using AttnFn = void (*)(const AttnArgs);
@@ -109,6 +114,24 @@ const std::map<AttnKey, AttnFns>& attn_table() {
 #endif
 #undef AK8
 #undef AK
+  };
+  return t;
+}
+
+// Cooperative attention kernels: key (G, d, r, tokens per stage, int8 keys).
+const std::map<AttnKey, AttnFns>& coop_table() {
+  static const std::map<AttnKey, AttnFns> t = {
+#define CK(G, D, R, T, K8) \
+  {AttnKey{G, D, R, T, K8}, AttnFns{&attn_coop_kernel<G, D, R, T, K8, false>, &attn_coop_kernel<G, D, R, T, K8, true>}}
+#ifdef BASISKV_WAIT_TEST
+      CK(4, 128, 32, 64, false), CK(4, 128, 32, 32, false),
+#else
+      CK(4, 128, 32, 64, false), CK(4, 128, 32, 32, false), CK(4, 128, 24, 32, false),
+      CK(4, 128, 128, 64, false), CK(4, 128, 128, 32, false), CK(4, 64, 16, 16, false),
+      CK(4, 128, 32, 64, true), CK(4, 128, 32, 32, true), CK(4, 128, 24, 32, true),
+      CK(4, 128, 128, 64, true), CK(4, 128, 128, 32, true), CK(4, 64, 16, 16, true),
+#endif
+#undef CK
   };
   return t;
 }
@@ -198,6 +221,8 @@ struct basiskv_handle {
   KernelFn route_fn = nullptr;
   AttnFn attn_fn = nullptr;         // persistent attention, waiting for the selection grid
   AttnFn attn_fn_ts = nullptr;      // the same reading tagged selection entries
+  bool attn_coop = false;           // attn_fn is attn_coop_kernel
+  int attn_threads = kAttnThreads;
   int attn_tps = 0;
   int route_stages = 0, attn_stages = 0;
   size_t route_smem = 0, attn_smem = 0;
@@ -264,6 +289,28 @@ void choose_kernels(basiskv_handle* h) {
     }
   }
   const bool k8 = p.k_format == BASISKV_KEYS_INT8;
+  // the cooperative kernel where a shape of it is compiled: 32-token stages
+  // where pages allow (about twenty stages in flight per SM), one CTA per SM
+  for (int tps : {32, 64, 16}) {
+    if (p.page_size % tps) continue;
+    auto cit = coop_table().find(AttnKey{p.gqa_group, p.head_dim, p.rank_r, tps, k8});
+    if (cit == coop_table().end()) continue;
+    const size_t stage = (size_t)tps * (p.head_dim * (k8 ? 1 : es) + p.rank_r * es + (k8 ? 4 : 0));
+    const size_t gr = (size_t)p.gqa_group * p.rank_r;
+    const size_t extra =
+        sizeof(float) * ((size_t)coop_bufs(p.gqa_group, p.rank_r) * kCoopWarps * (gr + 16) + kCoopMergeWarps * gr);
+    if (kCoopSmemPerSm < extra + 2 * kCoopWarps * stage) continue;
+    // a multiple of the consumer warps (each warp's stages keep their slots)
+    const int st = (int)std::min<size_t>(kCoopMaxStages, (kCoopSmemPerSm - extra) / stage) / kCoopWarps * kCoopWarps;
+    h->attn_fn = cit->second.plain;
+    h->attn_fn_ts = cit->second.tagged;
+    h->attn_coop = true;
+    h->attn_threads = kCoopThreads;
+    h->attn_tps = tps;
+    h->attn_stages = st;
+    h->attn_smem = st * stage + extra;
+    return;
+  }
   // Where P.Z is heavy (r >= 64) more resident warps pay for shallower
   // rings: a 64 KB ring lets three CTAs share an SM (dense limit, r = 128:
   // 120 us against 123 us, 111 against 115 with int8 keys); at r = 32 the
@@ -341,6 +388,7 @@ struct LaunchPlan {
   int attn_pps = 0, attn_splits = 0;
   // persistent kernels
   int route_ctas = 0, attn_ctas = 0;
+  long long attn_chunk = 0;   // cooperative attention: items per CTA
   int route_static_pct = 100;  // pages of the persistent routing grid handed out in static shares
   int max_routed = 0;          // pages of the longest routed sequence
   // work plans (prefix over sequences), when batch <= kPlanMax
@@ -406,6 +454,19 @@ LaunchPlan plan(const basiskv_handle* h, int batch, int topk, bool force_route) 
   lp.route_ctas = (int)std::max<long long>(1, std::min<long long>(
       (long long)h->num_sms * h->route_occ, (lp.route_pages + kRouteWarps * min_per_warp - 1) /
                                                 (kRouteWarps * min_per_warp)));
+  if (h->attn_coop) {
+    // one chunk of consecutive items per CTA; a unit must meet at most
+    // kPartsCap - 2 chunks
+    long long ctas = std::min<long long>((long long)h->num_sms * h->attn_occ,
+                                         std::max<long long>(1, lp.attn_items / kCoopMinItems));
+    if (lp.max_unit_items > 0) {
+      const long long per = (lp.max_unit_items + kPartsCap - 3) / (kPartsCap - 2);
+      ctas = std::min<long long>(ctas, std::max<long long>(1, lp.attn_items / per));
+    }
+    lp.attn_ctas = (int)std::max<long long>(1, ctas);
+    lp.attn_chunk = std::max<long long>(1, (lp.attn_items + lp.attn_ctas - 1) / lp.attn_ctas);
+    return lp;
+  }
   long long attn_warps = std::min<long long>((long long)h->num_sms * h->attn_occ * kAttnWarps,
                                              std::max<long long>(1, lp.attn_items));
   if (lp.max_unit_items > 0) {
@@ -588,11 +649,12 @@ int launch_attn(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk
   a.batch = lp.batch;
   a.attn_off = h->d_attn_off;
   a.plan_n = lp.attn_off.empty() ? -1 : lp.batch;
+  a.chunk_items = (int)lp.attn_chunk;
   for (size_t i = 0; i < lp.attn_off.size(); ++i) a.plan_off[i] = lp.attn_off[i];
 
   cudaLaunchAttribute attr[1];
   if (h->attn_fn) {
-    cudaLaunchConfig_t cfg = launch_cfg(dim3(lp.attn_ctas), kAttnThreads, h->attn_smem, stream, pdl, attr);
+    cudaLaunchConfig_t cfg = launch_cfg(dim3(lp.attn_ctas), h->attn_threads, h->attn_smem, stream, pdl, attr);
     CUDA_TRY(cudaLaunchKernelEx(&cfg, tagged_sel ? h->attn_fn_ts : h->attn_fn, a));
     return BASISKV_OK;
   }
@@ -707,9 +769,9 @@ int basiskv_create(const basiskv_params* p, basiskv_handle** out) {
   if (!arc && h->attn_fn) {
     // one grid size for both variants: the smaller residency of the two
     int occ_ts = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&h->attn_occ, h->attn_fn, kAttnThreads, h->attn_smem) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&h->attn_occ, h->attn_fn, h->attn_threads, h->attn_smem) !=
             cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_ts, h->attn_fn_ts, kAttnThreads, h->attn_smem) !=
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_ts, h->attn_fn_ts, h->attn_threads, h->attn_smem) !=
             cudaSuccess)
       arc = fail(BASISKV_ERR_CUDA, "occupancy query failed");
     else

@@ -87,6 +87,41 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   }
 }
 
+// Wait like mbar_wait, and also give up (without a status) once another
+// warp of the CTA has set *abort; on expiry set both.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity, uint32_t* status,
+                                                   volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 15u) == 0) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        atomicOr(status, kStatusTimeout);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Atomic add with release and acquire semantics at gpu scope: the caller's
+// earlier writes (and those ordered before them) are visible to whoever
+// reads the new count, and the caller sees everything released by earlier
+// adders.  Returns the old value.
+__device__ __forceinline__ uint32_t atomic_add_acq_rel(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// Arrive once on `bar` (release at CTA scope: the caller's earlier shared
+// memory writes are visible to the thread that sees the phase complete).
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
 // How long a routing warp waits for a folded query written by other warps
 // before it folds the query itself.
 constexpr uint64_t kFoldWaitNs = 50000ull;
@@ -169,6 +204,10 @@ __device__ __forceinline__ void ldsm_x2_trans(uint32_t& r0, uint32_t& r1, const 
   asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
                : "=r"(r0), "=r"(r1)
                : "r"(smem_addr(row)));
+}
+
+__device__ __forceinline__ void ldsm_x1_trans(uint32_t& r0, const void* row) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x1.trans.shared.b16 {%0}, [%1];" : "=r"(r0) : "r"(smem_addr(row)));
 }
 
 // ---- bf16 tensor-core MMA, fp32 accumulate ----------------------------------
