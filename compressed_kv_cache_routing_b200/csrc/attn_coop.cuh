@@ -3,16 +3,19 @@
 // selected pages to compute exact QK scores"; values stay rank-r latents Z
 // and the weighted latent is expanded by B_v at the end).
 //
-// attn_coop_kernel is persistent: CTA c takes chunk c of the flat list of
-// attention items (sequence-major, then KV head, selected entry, stage of
-// the page; chunks of chunk_items consecutive items, one per CTA by
-// default).  Its warps have three roles:
-//  - the issuing warp takes items 32 at a time, one per lane: a lane looks
-//    its item up (selected entry, then page-table slot), waits until its
-//    stage of the ring is free and starts the stage's bulk copies; a stage
-//    carries TPS tokens of one selected page (K rows, Z rows and, for int8
-//    keys, the token scales) and a descriptor (unit, valid tokens, segment
-//    number);
+// attn_coop_kernel is persistent over the flat list of attention items
+// (sequence-major, then KV head, selected entry, stage of the page), cut
+// into chunks of chunk_items consecutive items: CTA c takes chunks c,
+// c + gridDim.x, ... (one each as the host sizes them).  Its warps have
+// four roles:
+//  - the lookup warp looks items up 32 at a time, one per lane (selected
+//    entry, then page-table slot), numbers the segments and queues the items
+//    in shared memory;
+//  - the issuing warp: lane j owns ring slot j and hands out the stages
+//    j, j + NST, ...: it waits until the slot is free, writes the stage's
+//    descriptor (unit, valid tokens, segment number) and starts the bulk
+//    copies of TPS tokens of one selected page (K rows, Z rows and, for
+//    int8 keys, the token scales);
 //  - kCoopWarps consumer warps take the stages round-robin (stage n goes to
 //    warp n mod kCoopWarps), so they share one deep ring and advance
 //    together; a warp computes exact QK for its stage and the whole GQA
@@ -43,9 +46,14 @@ constexpr int kCoopWarps = 8;   // consumer warps
 // where one warp state is large)
 __host__ __device__ constexpr int coop_bufs(int g, int rr) { return g * rr >= 256 ? 2 : 4; }
 constexpr int kCoopMaxBufs = 4;
-constexpr int kCoopSegs = 64;   // segment descriptors in flight (> kCoopMaxBufs + kCoopMaxStages + 1)
+constexpr int kCoopLookQ = 64;  // looked-up items between the lookup warp and the issuing lanes
+// Segment descriptors in flight: the lookup warp runs at most kCoopLookQ
+// stages ahead of the issuing lanes, which run at most kCoopMaxStages ahead
+// of the slowest consumer (plus one round of kCoopWarps), which runs at most
+// kCoopMaxBufs segments ahead of the merge warps; a segment has a stage.
+constexpr int kCoopSegs = 128;
 constexpr int kCoopMergeWarps = 2;  // merge warps: segment f goes to merge warp f mod 2
-constexpr int kCoopThreads = (kCoopWarps + 1 + kCoopMergeWarps) * 32;
+constexpr int kCoopThreads = (kCoopWarps + 2 + kCoopMergeWarps) * 32;
 
 // Descriptor of one staged item, written by the issuing warp before the
 // copies are started (the barrier's completion makes it visible).
@@ -56,8 +64,38 @@ struct __align__(16) CoopMeta {
   int pad;
 };
 
-// Descriptor of one segment, written by the issuing warp with the
-// segment's first stage, read by the merge warp.
+// One looked-up item, passed from the lookup warp to the issuing lane of its
+// stage through a shared-memory queue (seq = the stage number once filled).
+struct __align__(16) CoopLook {
+  unsigned long long row0;  // first pool row of the stage
+  int u;                    // unit; -1: end marker stage; -2: no more stages for this lane
+  int valid;                // tokens of the stage inside the sequence
+  int sid;                  // segment number within the CTA
+  uint32_t seq;
+};
+
+// Spin until *p == want (shared memory, bounded like mbar_wait; gives up
+// when another warp has set *abort).
+__device__ __forceinline__ bool poll_equal(const uint32_t* p, uint32_t want, uint32_t* status, volatile int* abort) {
+  const volatile uint32_t* v = p;
+  if (*v == want) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if (*v == want) return true;
+    if ((it & 15u) == 0) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        atomicOr(status, kStatusTimeout);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Descriptor of one segment, written by the lookup warp with the segment's
+// first item, read by the merge warps.
 struct __align__(16) CoopSeg {
   int u;          // unit; -1: no more segments
   int kvh;
@@ -134,7 +172,8 @@ __global__ void __launch_bounds__(kCoopThreads, 1) attn_coop_kernel(const __grid
   __shared__ uint64_t full[kCoopMaxStages], empty[kCoopMaxStages], mfull[kCoopMaxBufs], mempty[kCoopMaxBufs];
   __shared__ CoopMeta meta[kCoopMaxStages];
   __shared__ CoopSeg segs[kCoopSegs];
-  __shared__ uint32_t pend[kCoopMaxStages];  // the last stage whose copies each slot received
+  __shared__ CoopLook lookq[kCoopLookQ];     // looked-up items, lookup warp -> issuing lanes
+  __shared__ uint32_t lookd[kCoopLookQ];     // the stage whose entry each queue position last gave out
   __shared__ int abort_flag;
   uint8_t* ring = smem;
   float* mrg = reinterpret_cast<float*>(smem + (size_t)NST * stage_bytes);  // [kCoopBufs][NW][MW]
@@ -154,8 +193,8 @@ __global__ void __launch_bounds__(kCoopThreads, 1) attn_coop_kernel(const __grid
     for (int i = 0; i < NST; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
-      pend[i] = 0xffffffffu;
     }
+    for (int i = 0; i < kCoopLookQ; ++i) lookq[i].seq = lookd[i] = 0xffffffffu;
     for (int i = 0; i < kCoopBufs; ++i) {
       mbar_init(&mfull[i], NW);
       mbar_init(&mempty[i], 1);
@@ -167,7 +206,7 @@ __global__ void __launch_bounds__(kCoopThreads, 1) attn_coop_kernel(const __grid
   volatile int* abort = &abort_flag;
 
   if (warp == NW) {
-    // ---- the issuing warp --------------------------------------------------
+    // ---- the lookup warp ---------------------------------------------------
     // the selection is written by the previous grid: wait for that grid, or,
     // with a tagged selection, for each unit's entries as they are looked up
     if constexpr (!TS) pdl_wait_primary();
@@ -177,24 +216,31 @@ __global__ void __launch_bounds__(kCoopThreads, 1) attn_coop_kernel(const __grid
     const long long T = offsets[a.batch];
     const long long CH = a.chunk_items > 0 ? a.chunk_items : max(1LL, (T + gridDim.x - 1) / gridDim.x);
     const long long nch = (T + CH - 1) / CH;
-    const uint8_t* kpool = static_cast<const uint8_t*>(a.k_pool);
-    const __nv_bfloat16* zpool = static_cast<const __nv_bfloat16*>(a.z_pool);
-    const uint64_t pol = policy_evict_first();
-    uint32_t issued = 0;  // stages handed out so far (the same in every lane)
-    int sid = -1;         // number of the last segment begun
+    uint32_t n = 0;  // next stage number (the same in every lane)
+    int sid = -1;    // number of the last segment begun
     bool ok = true;
+    // lane l waits until queue entry n + l is free, then fills it
+    auto put = [&](uint32_t nn, const CoopLook& lk) -> bool {
+      CoopLook* e = &lookq[nn % kCoopLookQ];
+      if (nn >= (uint32_t)kCoopLookQ && !poll_equal(&lookd[nn % kCoopLookQ], nn - kCoopLookQ, a.status, abort))
+        return false;
+      e->row0 = lk.row0;
+      e->u = lk.u;
+      e->valid = lk.valid;
+      e->sid = lk.sid;
+      __threadfence_block();
+      *reinterpret_cast<volatile uint32_t*>(&e->seq) = nn;
+      return true;
+    };
     for (long long c = blockIdx.x; ok && c < nch; c += gridDim.x) {
       const long long c0 = c * CH, c1 = min(T, c0 + CH);
       for (long long g0 = c0; ok && g0 < c1; g0 += 32) {
         const int n_in = (int)min(32LL, c1 - g0);
-        // lane j looks up item g0 + j (its selected page and the page's slot)
-        // and hands it out as stage issued + j
-        const bool mine = lane < n_in;
-        CoopSeg sg;
-        CoopMeta m;
-        unsigned long long row0 = 0;
+        // lane j looks up item g0 + j: its selected page and the page's slot
+        CoopLook lk;
         bool new_seg = false;
-        if (mine) {
+        CoopSeg sg;
+        if (lane < n_in) {
           const long long f = g0 + lane;
           AttnCursor cj;
           cj.seek(a, offsets, (int)f, sub);
@@ -205,80 +251,93 @@ __global__ void __launch_bounds__(kCoopThreads, 1) attn_coop_kernel(const __grid
             slot = 0;
           }
           const long long uo = cj.uoff, nu = (long long)cj.kb * sub;
-          row0 = ((unsigned long long)slot * a.num_kv_heads + cj.kvh) * P + (unsigned long long)cj.ts * TPS;
+          lk.row0 = ((unsigned long long)slot * a.num_kv_heads + cj.kvh) * P + (unsigned long long)cj.ts * TPS;
+          lk.u = cj.unit(a);
+          lk.valid = cj.L - (page * P + cj.ts * TPS);
           new_seg = f == c0 || f == uo;
-          sg.u = cj.unit(a);
+          sg.u = lk.u;
           sg.kvh = cj.kvh;
           sg.slot = (int)(c - uo / CH);
           sg.seg_items = (int)(min(c1, uo + nu) - max(c0, uo));
           sg.np = (int)((uo + nu - 1) / CH - uo / CH + 1);
           sg.nu = (int)nu;
-          m.u = sg.u;
-          m.valid = cj.L - (page * P + cj.ts * TPS);
         }
         const unsigned starts = __ballot_sync(0xffffffffu, new_seg);
-        m.sid = sid + __popc(starts & (0xffffffffu >> (31 - lane)));
-        m.pad = 0;
-        // in rounds of NST lanes: a lane waits only once the stage NST before
-        // its own has been handed out, so the parity it waits for is the
-        // barrier's current or next phase, never one further
-        for (int r0 = 0; ok && r0 < n_in; r0 += NST) {
-          bool lok = true;
-          if (lane >= r0 && lane < min(n_in, r0 + NST)) {
-            const uint32_t n = issued + lane;
-            const int s = (int)(n % NST);
-            lok = mbar_wait_or_abort(&empty[s], ((n / NST) & 1u) ^ 1u, a.status, abort);
-            if (lok) {
-              if (new_seg) segs[m.sid % kCoopSegs] = sg;
-              meta[s] = m;
-              if (!skip_issue_for_test((int)blockIdx.x, (int)n)) {
-                uint8_t* dst = ring + (size_t)s * stage_bytes;
-                pend[s] = n;
-                mbar_arrive_expect_tx(&full[s], stage_bytes);
-                bulk_load(dst, kpool + row0 * D * KB, kbytes, &full[s], pol);
-                bulk_load(dst + kbytes, zpool + row0 * RR, zbytes, &full[s], pol);
-                if constexpr (K8) bulk_load(dst + kbytes + zbytes, a.k_scale + row0, sbytes, &full[s], pol);
-              }
-            }
-          }
-          ok = __all_sync(0xffffffffu, lok);
+        lk.sid = sid + __popc(starts & (0xffffffffu >> (31 - lane)));
+        bool lok = true;
+        if (lane < n_in) {
+          if (new_seg) segs[lk.sid % kCoopSegs] = sg;
+          lok = put(n + lane, lk);
         }
-        issued += n_in;
+        ok = __all_sync(0xffffffffu, lok);
+        n += n_in;
         sid += __popc(starts);
       }
     }
     if (ok) {
-      // end of the work: one closing segment number per merge warp, and
-      // one stage without copies for every consumer warp
+      // the end: one closing segment number per merge warp, one stage without
+      // copies for every consumer warp, and a stop for the other issuing lanes
       if (lane < kCoopMergeWarps) segs[(sid + 1 + lane) % kCoopSegs].u = -1;
       __syncwarp();
-      bool lok = true;
-      if (lane < NW) {
-        const uint32_t n = issued + lane;
-        const int s = (int)(n % NST);
-        lok = mbar_wait_or_abort(&empty[s], ((n / NST) & 1u) ^ 1u, a.status, abort);
-        if (lok) {
-          meta[s] = CoopMeta{-1, 0, sid + 1, 0};
-          mbar_arrive(&full[s]);
-        }
-      }
-      ok = __all_sync(0xffffffffu, lok);
-    }
-    __syncwarp();
-    if (!ok && lane == 0) {
-      // given up: let the copies still in flight land before the CTA exits
-      // (the last stage each slot received copies for)
-      for (int s = 0; s < NST; ++s) {
-        const uint32_t n = pend[s];
-        if (n != 0xffffffffu) mbar_wait(&full[s], (n / NST) & 1u, a.status);
+      if (lane < NST) {
+        CoopLook lk;
+        lk.row0 = 0;
+        lk.u = lane < NW ? -1 : -2;
+        lk.valid = 0;
+        lk.sid = sid + 1;
+        put(n + lane, lk);
       }
     }
     return;
   }
 
-  if (warp > NW) {
+  if (warp == NW + 1) {
+    // ---- the issuing warp: lane j hands out the stages of ring slot j ------
+    if (lane >= NST) return;
+    const uint8_t* kpool = static_cast<const uint8_t*>(a.k_pool);
+    const __nv_bfloat16* zpool = static_cast<const __nv_bfloat16*>(a.z_pool);
+    const uint64_t pol = policy_evict_first();
+    const int s = lane;
+    uint32_t pend = 0xffffffffu;  // the last stage this slot received copies for
+    bool ok = true;
+    for (uint32_t n = lane;; n += NST) {
+      const CoopLook* e = &lookq[n % kCoopLookQ];
+      if (!poll_equal(&e->seq, n, a.status, abort)) {
+        ok = false;
+        break;
+      }
+      __threadfence_block();
+      const CoopLook lk = *e;
+      if (lk.u == -2) break;
+      // this slot's previous stage (n - NST) was handed out by this lane, so
+      // the barrier is at most one phase behind the one waited for
+      if (!mbar_wait_or_abort(&empty[s], ((n / NST) & 1u) ^ 1u, a.status, abort)) {
+        ok = false;
+        break;
+      }
+      meta[s] = CoopMeta{lk.u, lk.valid, lk.sid, 0};
+      __threadfence_block();
+      *reinterpret_cast<volatile uint32_t*>(&lookd[n % kCoopLookQ]) = n;
+      if (lk.u == -1) {
+        mbar_arrive(&full[s]);  // the end marker of one consumer warp
+        break;
+      }
+      if (skip_issue_for_test((int)blockIdx.x, (int)n)) continue;
+      uint8_t* dst = ring + (size_t)s * stage_bytes;
+      pend = n;
+      mbar_arrive_expect_tx(&full[s], stage_bytes);
+      bulk_load(dst, kpool + lk.row0 * D * KB, kbytes, &full[s], pol);
+      bulk_load(dst + kbytes, zpool + lk.row0 * RR, zbytes, &full[s], pol);
+      if constexpr (K8) bulk_load(dst + kbytes + zbytes, a.k_scale + lk.row0, sbytes, &full[s], pol);
+    }
+    // given up: let this slot's copies still in flight land before the CTA exits
+    if (!ok && pend != 0xffffffffu) mbar_wait(&full[s], (pend / NST) & 1u, a.status);
+    return;
+  }
+
+  if (warp > NW + 1) {
     // ---- the merge warps: segments mw, mw + 2, ... ----------------------------
-    const int mw = warp - NW - 1;
+    const int mw = warp - NW - 2;
     float* zb = zbar + mw * G * RR;
     for (uint32_t f = mw;; f += kCoopMergeWarps) {
       const int b = (int)(f % kCoopBufs);
