@@ -55,10 +55,19 @@ constexpr size_t kAttnSmemBudgetWide = 64 * 1024;  // attention rings when r >= 
 // Cooperative attention: one CTA per SM; its ring takes what is left of the
 // SM's shared memory after the merge buffers.
 constexpr size_t kCoopSmemPerSm = 212 * 1024;
-constexpr long long kCoopMinItems = 8;  // items per CTA at least
+constexpr long long kCoopMinItems = 8;       // items per CTA at least
+constexpr long long kCoopMinUnitItems = 64;  // stages per unit from which the shared ring is used
 
 using KernelFn = void (*)(const RouteArgs);
 using AttnFn = void (*)(const AttnArgs);
+// A persistent attention kernel chosen at create for this shape.
+struct AttnKernel {
+  AttnFn plain = nullptr;   // waits for the selection grid
+  AttnFn tagged = nullptr;  // reads tagged selection entries as they come
+  bool coop = false;        // attn_coop_kernel (shared ring), else attn_mma_kernel (a ring per warp)
+  int threads = kAttnThreads, tps = 0, stages = 0, occ = 1;
+  size_t smem = 0;
+};
 struct AttnFns {
   AttnFn plain;   // waits for the selection grid
   AttnFn tagged;  // reads tagged selection entries as they come
@@ -219,15 +228,12 @@ struct basiskv_handle {
   std::vector<int32_t> h_npages;
   // kernels chosen at create
   KernelFn route_fn = nullptr;
-  AttnFn attn_fn = nullptr;         // persistent attention, waiting for the selection grid
-  AttnFn attn_fn_ts = nullptr;      // the same reading tagged selection entries
-  bool attn_coop = false;           // attn_fn is attn_coop_kernel
-  int attn_threads = kAttnThreads;
-  int attn_tps = 0;
-  int route_stages = 0, attn_stages = 0;
-  size_t route_smem = 0, attn_smem = 0;
+  AttnKernel attn_warp;  // a ring per warp: every shape it is compiled for
+  AttnKernel attn_coop;  // a shared ring per CTA: long units
+  int route_stages = 0;
+  size_t route_smem = 0;
   int topk_keys = 0;  // scores staged in shared memory by the selection kernel
-  int route_occ = 1, attn_occ = 1;  // resident CTAs per SM of the persistent kernels
+  int route_occ = 1;  // resident CTAs per SM of the persistent routing kernel
   // profiling
   std::vector<cudaEvent_t> events;  // kProfEvents per recorded call
   int prof_cap = 0, prof_calls = 0;
@@ -289,8 +295,8 @@ void choose_kernels(basiskv_handle* h) {
     }
   }
   const bool k8 = p.k_format == BASISKV_KEYS_INT8;
-  // the cooperative kernel where a shape of it is compiled: 32-token stages
-  // where pages allow (about twenty stages in flight per SM), one CTA per SM
+  // the shared-ring kernel where a shape of it is compiled: 32-token stages
+  // where pages allow, one CTA per SM, a ring of a multiple of eight stages
   for (int tps : {32, 64, 16}) {
     if (p.page_size % tps) continue;
     auto cit = coop_table().find(AttnKey{p.gqa_group, p.head_dim, p.rank_r, tps, k8});
@@ -302,14 +308,15 @@ void choose_kernels(basiskv_handle* h) {
     if (kCoopSmemPerSm < extra + 2 * kCoopWarps * stage) continue;
     // a multiple of the consumer warps (each warp's stages keep their slots)
     const int st = (int)std::min<size_t>(kCoopMaxStages, (kCoopSmemPerSm - extra) / stage) / kCoopWarps * kCoopWarps;
-    h->attn_fn = cit->second.plain;
-    h->attn_fn_ts = cit->second.tagged;
-    h->attn_coop = true;
-    h->attn_threads = kCoopThreads;
-    h->attn_tps = tps;
-    h->attn_stages = st;
-    h->attn_smem = st * stage + extra;
-    return;
+    AttnKernel& k = h->attn_coop;
+    k.plain = cit->second.plain;
+    k.tagged = cit->second.tagged;
+    k.coop = true;
+    k.threads = kCoopThreads;
+    k.tps = tps;
+    k.stages = st;
+    k.smem = st * stage + extra;
+    break;
   }
   // Where P.Z is heavy (r >= 64) more resident warps pay for shallower
   // rings: a 64 KB ring lets three CTAs share an SM (dense limit, r = 128:
@@ -325,11 +332,12 @@ void choose_kernels(basiskv_handle* h) {
       int st = (int)std::min<size_t>(4, budget / (kAttnWarps * stage));
       if (st < 1) continue;
       if (st < 2 && tps > 16) continue;  // prefer a smaller stage with double buffering
-      h->attn_fn = ait->second.plain;
-      h->attn_fn_ts = ait->second.tagged;
-      h->attn_tps = tps;
-      h->attn_stages = st;
-      h->attn_smem = kAttnWarps * st * stage + sizeof(float) * kAttnWarps * p.gqa_group * p.rank_r;
+      AttnKernel& k = h->attn_warp;
+      k.plain = ait->second.plain;
+      k.tagged = ait->second.tagged;
+      k.tps = tps;
+      k.stages = st;
+      k.smem = kAttnWarps * st * stage + sizeof(float) * kAttnWarps * p.gqa_group * p.rank_r;
       return;
     }
   }
@@ -388,7 +396,8 @@ struct LaunchPlan {
   int attn_pps = 0, attn_splits = 0;
   // persistent kernels
   int route_ctas = 0, attn_ctas = 0;
-  long long attn_chunk = 0;   // cooperative attention: items per CTA
+  long long attn_chunk = 0;   // shared-ring attention: items per CTA
+  const AttnKernel* ak = nullptr;  // the persistent attention kernel, or none (generic)
   int route_static_pct = 100;  // pages of the persistent routing grid handed out in static shares
   int max_routed = 0;          // pages of the longest routed sequence
   // work plans (prefix over sequences), when batch <= kPlanMax
@@ -399,8 +408,7 @@ LaunchPlan plan(const basiskv_handle* h, int batch, int topk, bool force_route) 
   LaunchPlan lp;
   lp.batch = batch;
   const basiskv_params& p = h->p;
-  lp.sub = h->attn_fn ? p.page_size / h->attn_tps : 1;
-  long long route_pages = 0, items = 0;
+  long long route_pages = 0, pages = 0;
   int max_routed = 0, max_kb = 0;
   for (int b = 0; b < batch; ++b) {
     const int n = h->h_npages[b];
@@ -410,8 +418,16 @@ LaunchPlan plan(const basiskv_handle* h, int batch, int topk, bool force_route) 
     }
     const int kb = std::min(topk, n);
     max_kb = std::max(max_kb, kb);
-    items += (long long)kb * lp.sub;
+    pages += kb;
   }
+  // The shared-ring kernel where units are long; with short units (a few
+  // dozen stages) a CTA finishes many units, and the per-warp rings, whose
+  // warps each finish their own, end sooner.
+  const AttnKernel& co = h->attn_coop;
+  if (co.plain && (long long)max_kb * (p.page_size / co.tps) >= kCoopMinUnitItems) lp.ak = &co;
+  else if (h->attn_warp.plain) lp.ak = &h->attn_warp;
+  lp.sub = lp.ak ? p.page_size / lp.ak->tps : 1;
+  const long long items = pages * lp.sub;
   lp.route_pages = route_pages * p.num_kv_heads;
   lp.attn_items = items * p.num_kv_heads;
   if (batch <= kPlanMax) {
@@ -454,10 +470,10 @@ LaunchPlan plan(const basiskv_handle* h, int batch, int topk, bool force_route) 
   lp.route_ctas = (int)std::max<long long>(1, std::min<long long>(
       (long long)h->num_sms * h->route_occ, (lp.route_pages + kRouteWarps * min_per_warp - 1) /
                                                 (kRouteWarps * min_per_warp)));
-  if (h->attn_coop) {
+  if (lp.ak && lp.ak->coop) {
     // one chunk of consecutive items per CTA; a unit must meet at most
     // kPartsCap - 2 chunks
-    long long ctas = std::min<long long>((long long)h->num_sms * h->attn_occ,
+    long long ctas = std::min<long long>((long long)h->num_sms * lp.ak->occ,
                                          std::max<long long>(1, lp.attn_items / kCoopMinItems));
     if (lp.max_unit_items > 0) {
       const long long per = (lp.max_unit_items + kPartsCap - 3) / (kPartsCap - 2);
@@ -467,7 +483,7 @@ LaunchPlan plan(const basiskv_handle* h, int batch, int topk, bool force_route) 
     lp.attn_chunk = std::max<long long>(1, (lp.attn_items + lp.attn_ctas - 1) / lp.attn_ctas);
     return lp;
   }
-  long long attn_warps = std::min<long long>((long long)h->num_sms * h->attn_occ * kAttnWarps,
+  long long attn_warps = std::min<long long>((long long)h->num_sms * (lp.ak ? lp.ak->occ : 1) * kAttnWarps,
                                              std::max<long long>(1, lp.attn_items));
   if (lp.max_unit_items > 0) {
     // a unit must meet at most kPartsCap - 2 warps: each warp gets at least
@@ -642,7 +658,7 @@ int launch_attn(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk
   a.gqa_group = p.gqa_group;
   a.topk = topk;
   a.pages_per_split = lp.attn_pps;
-  a.stages = h->attn_stages;
+  a.stages = lp.ak ? lp.ak->stages : 0;
   a.np_cap = kPartsCap;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.latent = latent;
@@ -653,9 +669,9 @@ int launch_attn(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk
   for (size_t i = 0; i < lp.attn_off.size(); ++i) a.plan_off[i] = lp.attn_off[i];
 
   cudaLaunchAttribute attr[1];
-  if (h->attn_fn) {
-    cudaLaunchConfig_t cfg = launch_cfg(dim3(lp.attn_ctas), h->attn_threads, h->attn_smem, stream, pdl, attr);
-    CUDA_TRY(cudaLaunchKernelEx(&cfg, tagged_sel ? h->attn_fn_ts : h->attn_fn, a));
+  if (lp.ak) {
+    cudaLaunchConfig_t cfg = launch_cfg(dim3(lp.attn_ctas), lp.ak->threads, lp.ak->smem, stream, pdl, attr);
+    CUDA_TRY(cudaLaunchKernelEx(&cfg, tagged_sel ? lp.ak->tagged : lp.ak->plain, a));
     return BASISKV_OK;
   }
   cudaLaunchConfig_t cfg = launch_cfg(dim3(lp.attn_splits, p.num_kv_heads, lp.batch), kAttnThreads,
@@ -758,27 +774,26 @@ int basiskv_create(const basiskv_params* p, basiskv_handle** out) {
   h->topk_keys = std::min(p->max_pages_per_seq, 16384);
   choose_kernels(h);
   int arc = h->route_fn ? set_smem_attr((const void*)h->route_fn, h->route_smem) : BASISKV_OK;
-  if (!arc && h->attn_fn) arc = set_smem_attr((const void*)h->attn_fn, h->attn_smem);
-  if (!arc && h->attn_fn_ts) arc = set_smem_attr((const void*)h->attn_fn_ts, h->attn_smem);
+  for (AttnKernel* k : {&h->attn_warp, &h->attn_coop}) {
+    if (!arc && k->plain) arc = set_smem_attr((const void*)k->plain, k->smem);
+    if (!arc && k->tagged) arc = set_smem_attr((const void*)k->tagged, k->smem);
+  }
   if (!arc)
     arc = set_smem_attr((const void*)&prep_kernel, 0);
   if (!arc) arc = set_smem_attr((const void*)&topk_kernel, sizeof(uint32_t) * (size_t)h->topk_keys);
   if (!arc && h->route_fn &&
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&h->route_occ, h->route_fn, kRouteThreads, h->route_smem) != cudaSuccess)
     arc = fail(BASISKV_ERR_CUDA, "occupancy query failed");
-  if (!arc && h->attn_fn) {
+  for (AttnKernel* k : {&h->attn_warp, &h->attn_coop}) {
+    if (arc || !k->plain) continue;
     // one grid size for both variants: the smaller residency of the two
-    int occ_ts = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&h->attn_occ, h->attn_fn, h->attn_threads, h->attn_smem) !=
-            cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_ts, h->attn_fn_ts, h->attn_threads, h->attn_smem) !=
-            cudaSuccess)
+    int occ = 0, occ_ts = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k->plain, k->threads, k->smem) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_ts, k->tagged, k->threads, k->smem) != cudaSuccess)
       arc = fail(BASISKV_ERR_CUDA, "occupancy query failed");
     else
-      h->attn_occ = std::min(h->attn_occ, occ_ts);
+      k->occ = std::max(1, std::min(occ, occ_ts));
   }
-  h->route_occ = std::max(1, h->route_occ);
-  h->attn_occ = std::max(1, h->attn_occ);
   if (!arc)
     arc = p->dtype == BASISKV_DTYPE_BF16 ? set_generic_attrs<__nv_bfloat16>(*p) : set_generic_attrs<float>(*p);
   if (!arc) {
@@ -945,7 +960,7 @@ static int decode_step(basiskv_handle* h, int batch, const void* q, int topk, fl
   const bool route_tc = lp.any_routed && h->route_fn;
   // the persistent grids read the work plan from their parameters; only a
   // batch too large for that needs the prep grid to write it
-  const bool use_prep = (route_tc || h->attn_fn) && lp.route_off.empty();
+  const bool use_prep = (route_tc || lp.ak) && lp.route_off.empty();
   if (use_prep) {
     rc = launch_prep(h, lp, topk, 0, out, sel_out, nullptr, latent, st);
     if (rc) return rc;
@@ -978,10 +993,10 @@ static int decode_step(basiskv_handle* h, int batch, const void* q, int topk, fl
   }
   h->last_launch[0] = lp.any_routed ? (h->route_fn ? 0 : lp.route_ppc) : 0;
   h->last_launch[1] = lp.any_routed ? (h->route_fn ? lp.route_ctas : lp.route_chunks * h->p.num_kv_heads * batch) : 0;
-  h->last_launch[2] = h->attn_fn ? 0 : lp.attn_splits;
-  h->last_launch[3] = h->attn_fn ? lp.attn_ctas : lp.attn_splits * h->p.num_kv_heads * batch;
+  h->last_launch[2] = lp.ak ? 0 : lp.attn_splits;
+  h->last_launch[3] = lp.ak ? lp.attn_ctas : lp.attn_splits * h->p.num_kv_heads * batch;
   h->last_launch[4] = h->route_fn != nullptr;
-  h->last_launch[5] = h->attn_fn != nullptr;
+  h->last_launch[5] = lp.ak != nullptr;
   return BASISKV_OK;
 }
 

@@ -22,10 +22,12 @@ constexpr int kPlanMax = 512;
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
 #ifdef BASISKV_WAIT_TEST
 // The wait-expiry test build: short waits, and the one copy that
-// skip_issue_for_test names is never issued, so its wait must run out.
+// skip_issue_for_test names (item 1 of issuer 0: a warp of the per-warp-ring
+// kernels, a CTA of the shared-ring one) is never issued, so its wait must
+// run out.
 constexpr uint64_t kWaitLimitNs = 1000000ull;
-__device__ __forceinline__ bool skip_issue_for_test(int warp_in_grid, int item) {
-  return warp_in_grid == 0 && item == 1;
+__device__ __forceinline__ bool skip_issue_for_test(int issuer, int item) {
+  return issuer == 0 && item == 1;
 }
 #else
 constexpr uint64_t kWaitLimitNs = 2000000000ull;

@@ -63,8 +63,8 @@ def decode_int8(kv, w, topk=None, latent=False):
     return out.cpu().numpy(), sel.cpu().numpy()
 
 
-INT8 = ["tiny", "llama3_8b_decode", "long_context", "high_concurrency", "dense_limit", "generic_bf16",
-        "gqa8", "gqa1", "head_dim64", "fp32_llama_shape"]
+INT8 = ["tiny", "llama3_8b_decode", "llama_shared_ring", "long_context", "high_concurrency", "dense_limit",
+        "generic_bf16", "gqa8", "gqa1", "head_dim64", "fp32_llama_shape"]
 
 
 @pytest.mark.parametrize("name", INT8)

@@ -104,6 +104,9 @@ def unit_rows(w, units):
 SMALL = {
     "tiny": W.SPECS["tiny"],
     "llama3_8b_decode": W.shrink("llama3_8b_decode", batch=3, len_lo=2500, len_hi=5000, topk=16),
+    # units of 64 stages and more take the shared-ring attention kernel (here
+    # beside unrouted units of sequences with fewer pages than k)
+    "llama_shared_ring": W.shrink("llama3_8b_decode", batch=3, len_lo=2500, len_hi=5000, topk=40),
     "long_context": W.shrink("long_context", batch=2, len_lo=6000, len_hi=9000, topk=32),
     "high_concurrency": W.shrink("high_concurrency", batch=6, len_lo=700, len_hi=1500, topk=8),
     "dense_limit": W.shrink("dense_limit", batch=2, len_lo=900, len_hi=1100, topk=32),
@@ -487,8 +490,8 @@ def test_append_page_copy_refused_copies_nothing():
 # The planted pages sit just above the best unplanted page (gap >= 1e-2 in
 # float64 on the stored bits, typically 0.05), the regime where a routing
 # score error could move a page across the k-th boundary.
-NEAR = ["tiny", "llama3_8b_decode", "long_context", "high_concurrency", "generic_bf16", "gqa8", "gqa2",
-        "gqa1", "head_dim64", "fp32_llama_shape"]
+NEAR = ["tiny", "llama3_8b_decode", "llama_shared_ring", "long_context", "high_concurrency", "generic_bf16",
+        "gqa8", "gqa2", "gqa1", "head_dim64", "fp32_llama_shape"]
 
 
 def _near(spec):

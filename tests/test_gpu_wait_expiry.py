@@ -3,8 +3,9 @@
 Every wait of the decode kernels on a shared-memory copy gives up after a
 time limit, records BASISKV_STATUS_TIMEOUT and drains the copies it did
 issue before returning.  The test build of the library (BASISKV_WAIT_TEST:
-1 ms limit, and the first warp of each grid never issues the copies of its
-second item) makes such a wait run out on purpose: nothing faults, no copy
+1 ms limit, and the first warp of each grid, or in the shared-ring
+attention kernel the first CTA, never issues the copies of its second item)
+makes such a wait run out on purpose: nothing faults, no copy
 is left in flight, the call returns, the status says TIMEOUT, and the CUDA
 context stays usable, so a following call of the normal library on a fresh
 handle is correct.
@@ -25,13 +26,16 @@ from test_gpu_parity import OUT_TOL, out_error, gpu_decode
 pytestmark = pytest.mark.gpu
 
 
-def test_wait_runs_out_and_is_reported():
+# k = 16 pages (32 stages per unit) runs the per-warp-ring attention kernel,
+# k = 48 (96 stages) the shared-ring one
+@pytest.mark.parametrize("topk", [16, 48])
+def test_wait_runs_out_and_is_reported(topk):
     if not torch.cuda.is_available():
         pytest.fail("needs a CUDA device")
     from compressed_kv_cache_routing_b200 import build
     build.build()
     lib = bk.load(build.build_wait_test())
-    spec = W.shrink("llama3_8b_decode", batch=3, len_lo=4096, len_hi=4096, topk=16)
+    spec = W.shrink("llama3_8b_decode", batch=3, len_lo=4096, len_hi=4096, topk=topk)
     w = W.generate(spec, device="cuda")
     s = w.spec
     ref = bk.BasisKV.for_workload(w)            # normal library: only for its params
