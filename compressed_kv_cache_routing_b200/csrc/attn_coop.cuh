@@ -179,16 +179,6 @@ __global__ void __launch_bounds__(kCoopThreads, 1) attn_coop_kernel(const __grid
   float* mrg = reinterpret_cast<float*>(smem + (size_t)NST * stage_bytes);  // [kCoopBufs][NW][MW]
   float* zbar = mrg + kCoopBufs * NW * MW;                                  // [kCoopMergeWarps][G][RR]
 
-  // sequences no warp visits: without pages they get out = 0 and a -1
-  // selection; with every page used (no routing) the identity selection
-  const int ow = a.latent ? RR : D;
-  for (int u = blockIdx.x; u < a.batch * a.num_kv_heads; u += gridDim.x) {
-    const int n = (a.seq_lens[u / a.num_kv_heads] + a.page_size - 1) / a.page_size;
-    if (n == 0)
-      for (int i = threadIdx.x; i < G * ow; i += blockDim.x) a.out[(size_t)u * G * ow + i] = 0.f;
-    if (a.sel_out && a.topk >= n)
-      for (int i = threadIdx.x; i < a.topk; i += blockDim.x) a.sel_out[(size_t)u * a.topk + i] = i < n ? i : -1;
-  }
   if (threadIdx.x == 0) {
     for (int i = 0; i < NST; ++i) {
       mbar_init(&full[i], 1);
@@ -241,22 +231,46 @@ __global__ void __launch_bounds__(kCoopThreads, 1) attn_coop_kernel(const __grid
         bool new_seg = false;
         CoopSeg sg;
         if (lane < n_in) {
-          const long long f = g0 + lane;
-          AttnCursor cj;
-          cj.seek(a, offsets, (int)f, sub);
-          const int page = cj.page<TS>(a);
-          int slot = __ldg(a.page_table + (size_t)cj.b * a.ld_pt + page);
+          // the item's place from the plan alone (sequence, KV head, selected
+          // entry, stage), so that the length and the selected entry are
+          // read together; the entry is used only where the unit is routed
+          const int f = (int)(g0 + lane);
+          int lo = 0, hi = a.batch;
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (offsets[mid] <= f) lo = mid + 1;
+            else hi = mid;
+          }
+          const int b = lo - 1;
+          const int per_unit = (offsets[b + 1] - offsets[b]) / a.num_kv_heads;  // kb * sub
+          const int rel = f - offsets[b];
+          const int kvh = rel / per_unit, jj = (rel % per_unit) / sub, ts = (rel % per_unit) % sub;
+          const int u = b * a.num_kv_heads + kvh;
+          const size_t e = (size_t)u * a.ld_sel + jj;
+          const int L = a.seq_lens[b];
+          uint64_t w = TS ? ld_relaxed_u64(a.sel64 + e) : (uint64_t)(uint32_t)__ldcg(a.sel + e);
+          const int n = (L + P - 1) / P;
+          int page = jj;
+          if (a.topk < n) {
+            if (TS && (uint32_t)(w >> 32) != a.sel_tag) w = wait_selected(a.sel64 + e, a.sel_tag, a.status);
+            page = (int)(uint32_t)w;
+            if (page < 0 || page >= n) {
+              atomicOr(a.status, kStatusBadPage);
+              page = 0;
+            }
+          }
+          int slot = __ldg(a.page_table + (size_t)b * a.ld_pt + page);
           if (slot < 0 || slot >= a.num_slots) {
             atomicOr(a.status, kStatusBadSlot);
             slot = 0;
           }
-          const long long uo = cj.uoff, nu = (long long)cj.kb * sub;
-          lk.row0 = ((unsigned long long)slot * a.num_kv_heads + cj.kvh) * P + (unsigned long long)cj.ts * TPS;
-          lk.u = cj.unit(a);
-          lk.valid = cj.L - (page * P + cj.ts * TPS);
+          const long long uo = offsets[b] + (long long)kvh * per_unit, nu = per_unit;
+          lk.row0 = ((unsigned long long)slot * a.num_kv_heads + kvh) * P + (unsigned long long)ts * TPS;
+          lk.u = u;
+          lk.valid = L - (page * P + ts * TPS);
           new_seg = f == c0 || f == uo;
           sg.u = lk.u;
-          sg.kvh = cj.kvh;
+          sg.kvh = kvh;
           sg.slot = (int)(c - uo / CH);
           sg.seg_items = (int)(min(c1, uo + nu) - max(c0, uo));
           sg.np = (int)((uo + nu - 1) / CH - uo / CH + 1);
@@ -339,6 +353,16 @@ __global__ void __launch_bounds__(kCoopThreads, 1) attn_coop_kernel(const __grid
     // ---- the merge warps: segments mw, mw + 2, ... ----------------------------
     const int mw = warp - NW - 2;
     float* zb = zbar + mw * G * RR;
+    // sequences no warp visits: without pages they get out = 0 and a -1
+    // selection; with every page used (no routing) the identity selection
+    const int ow = a.latent ? RR : D;
+    for (int u = blockIdx.x * kCoopMergeWarps + mw; u < a.batch * a.num_kv_heads; u += gridDim.x * kCoopMergeWarps) {
+      const int n = (a.seq_lens[u / a.num_kv_heads] + a.page_size - 1) / a.page_size;
+      if (n == 0)
+        for (int i = lane; i < G * ow; i += 32) a.out[(size_t)u * G * ow + i] = 0.f;
+      if (a.sel_out && a.topk >= n)
+        for (int i = lane; i < a.topk; i += 32) a.sel_out[(size_t)u * a.topk + i] = i < n ? i : -1;
+    }
     for (uint32_t f = mw;; f += kCoopMergeWarps) {
       const int b = (int)(f % kCoopBufs);
       if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&mfull[b], (f / kCoopBufs) & 1u, a.status, abort))) return;
