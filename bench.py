@@ -513,7 +513,8 @@ def run_ours(args, rank, world, local):
         kname = "route_mma_kernel" if launch["route_tensor_core"] else "route_generic_kernel"
     else:
         dom_bytes, dom_ms = nbytes["attn"], attn_mean
-        kname = "attn_mma_kernel" if launch["attn_tensor_core"] else "attn_generic_kernel"
+        kname = ("attn_coop_kernel" if launch["attn_shared_ring"] else "attn_mma_kernel") \
+            if launch["attn_tensor_core"] else "attn_generic_kernel"
     # routing (+ its selection grid on the tensor-core path), attention, prep past 512 sequences
     launches_per_step = (1 + launch["route_tensor_core"] if launch["route_ctas"] else 0) + 1 + \
         (1 if s.batch > 512 else 0)

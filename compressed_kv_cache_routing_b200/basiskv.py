@@ -243,7 +243,10 @@ def basiskv_last_launch(h):
     _check(load().basiskv_last_launch(h, ctypes.byref(info)))
     keys = ("route_pages_per_cta", "route_ctas", "attn_splits", "attn_ctas", "route_tensor_core",
             "attn_tensor_core")
-    return dict(zip(keys, list(info)))
+    d = dict(zip(keys, list(info)))
+    d["attn_shared_ring"] = int(d["attn_tensor_core"] == 2)  # 1: a ring per warp, 2: one per CTA
+    d["attn_tensor_core"] = int(d["attn_tensor_core"] > 0)
+    return d
 
 
 def basiskv_decode_attn_noalloc(params, page_table, seq_lens, q, topk, softmax_scale, out,

@@ -996,7 +996,7 @@ static int decode_step(basiskv_handle* h, int batch, const void* q, int topk, fl
   h->last_launch[2] = lp.ak ? 0 : lp.attn_splits;
   h->last_launch[3] = lp.ak ? lp.attn_ctas : lp.attn_splits * h->p.num_kv_heads * batch;
   h->last_launch[4] = h->route_fn != nullptr;
-  h->last_launch[5] = lp.ak != nullptr;
+  h->last_launch[5] = lp.ak ? (lp.ak->coop ? 2 : 1) : 0;
   return BASISKV_OK;
 }
 

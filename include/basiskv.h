@@ -296,8 +296,11 @@ BASISKV_API int basiskv_profile_begin(basiskv_handle *h, int max_calls);
 BASISKV_API int basiskv_profile_end(basiskv_handle *h, float *ms, int *ncalls);
 
 /* Launch shape chosen for the last decode call (for reports): routing pages
- * per CTA and CTA count, attention splits per unit and CTA count, and
- * whether the tensor-core kernels ran (1) or the generic ones (0). */
+ * per CTA and CTA count, attention splits per unit and CTA count, whether
+ * the tensor-core routing kernel ran (1) or the generic one (0), and which
+ * attention kernel ran: 0 generic, 1 tensor-core with a copy ring per warp,
+ * 2 tensor-core with one shared copy ring per CTA (units of 64 stages and
+ * more). */
 BASISKV_API int basiskv_last_launch(basiskv_handle *h, int info[6]);
 
 /* Allocation-free decode step.  The BasisKV paper has no counterpart to
