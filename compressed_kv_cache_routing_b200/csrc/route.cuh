@@ -248,12 +248,11 @@ __device__ __forceinline__ float route_page_score(const __nv_bfloat16* zs, const
 struct RouteCursor {
   int b, kvh, j, n, L;
   const int32_t* off;  // prefix of routed pages x Hkv over sequences
+  // sequence b's page count from the plan (its routed pages x Hkv), so the
+  // page-table address never waits for the length, which is read beside it
   __device__ __forceinline__ void load(const RouteArgs& a) {
+    n = (off[b + 1] - off[b]) / a.num_kv_heads;
     L = a.seq_lens[b];
-    n = (L + a.page_size - 1) / a.page_size;
-  }
-  __device__ __forceinline__ bool routed(const RouteArgs& a) const {
-    return n > 0 && (a.force || a.topk < n);
   }
   // first page at or after flat index f (route_off[b] <= f < route_off[b+1])
   __device__ void seek(const RouteArgs& a, const int32_t* offsets, int f) {
@@ -275,10 +274,11 @@ struct RouteCursor {
     j = 0;
     if (++kvh < a.num_kv_heads) return;
     kvh = 0;
-    for (++b; b < a.batch; ++b) {
-      load(a);
-      if (routed(a)) return;
-    }
+    for (++b; b < a.batch; ++b)
+      if (off[b + 1] > off[b]) {  // a routed sequence
+        load(a);
+        return;
+      }
   }
   __device__ __forceinline__ int unit(const RouteArgs& a) const { return b * a.num_kv_heads + kvh; }
 };
@@ -701,6 +701,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_c
   uint32_t fr[FR];
   int cur_u = -1;
   RouteCursor cc;  // compute cursor, set from each stage's bookkeeping
+  cc.off = offsets;  // (it steps across sequences within a stage)
 
   bool ok = true;
   int i = 0;
