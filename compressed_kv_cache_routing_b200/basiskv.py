@@ -28,6 +28,7 @@ BASISKV_STATUS_TIMEOUT = 2
 BASISKV_STATUS_BAD_PAGE = 4
 BASISKV_STATUS_PART_OVERFLOW = 8
 BASISKV_STATUS_BAD_LENGTH = 16
+BASISKV_STATUS_DEBUG_BOUNDS = 32  # debug build only
 
 BASISKV_DTYPE_BF16 = 0
 BASISKV_DTYPE_F32 = 1

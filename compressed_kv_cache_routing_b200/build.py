@@ -72,6 +72,19 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return _compile(LIB, [], verbose)
 
 
+# The debug build: the same sources with BASISKV_DEBUG, which checks the
+# indices the kernels keep in range by construction (ring stage, unit, KV
+# head, pool row, score and selection entries) and records
+# BASISKV_STATUS_DEBUG_BOUNDS instead of making a bad access.
+DEBUG_LIB = os.path.join(HERE, "libbasiskv_debug.so")
+
+
+def build_debug(force: bool = False) -> str:
+    if not force and not _stale_lib(DEBUG_LIB):
+        return DEBUG_LIB
+    return _compile(DEBUG_LIB, ["-DBASISKV_DEBUG"], False)
+
+
 def build_wait_test(force: bool = False) -> str:
     if not force and not _stale_lib(WAIT_TEST_LIB):
         return WAIT_TEST_LIB

@@ -507,7 +507,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_mma_kernel(const __grid_con
       atomicOr(a.status, kStatusBadSlot);
       slot = 0;
     }
-    const size_t row0 = ((size_t)slot * a.num_kv_heads + ic.kvh) * P + (size_t)ic.ts * TPS;
+    const size_t row0 = BASISKV_DEBUG_INDEX(((long long)slot * a.num_kv_heads + ic.kvh) * P + (long long)ic.ts * TPS,
+                                            (long long)a.num_slots * a.num_kv_heads * P - TPS + 1, a.status);
     tok0s[warp][s] = page * P + ic.ts * TPS;
     uint64_t* bar = &bars[warp][s];
     uint8_t* dst = ring + (size_t)s * stage_bytes;

@@ -339,10 +339,12 @@ __global__ void __launch_bounds__(kCoopThreads, 1) attn_coop_kernel(const __grid
       if (skip_issue_for_test((int)blockIdx.x, (int)n)) continue;
       uint8_t* dst = ring + (size_t)s * stage_bytes;
       pend = n;
+      const unsigned long long row0 = BASISKV_DEBUG_INDEX(
+          (long long)lk.row0, (long long)a.num_slots * a.num_kv_heads * P - TPS + 1, a.status);
       mbar_arrive_expect_tx(&full[s], stage_bytes);
-      bulk_load(dst, kpool + lk.row0 * D * KB, kbytes, &full[s], pol);
-      bulk_load(dst + kbytes, zpool + lk.row0 * RR, zbytes, &full[s], pol);
-      if constexpr (K8) bulk_load(dst + kbytes + zbytes, a.k_scale + lk.row0, sbytes, &full[s], pol);
+      bulk_load(dst, kpool + row0 * D * KB, kbytes, &full[s], pol);
+      bulk_load(dst + kbytes, zpool + row0 * RR, zbytes, &full[s], pol);
+      if constexpr (K8) bulk_load(dst + kbytes + zbytes, a.k_scale + row0, sbytes, &full[s], pol);
     }
     // given up: let this slot's copies still in flight land before the CTA exits
     if (!ok && pend != 0xffffffffu) mbar_wait(&full[s], (pend / NST) & 1u, a.status);
@@ -366,8 +368,10 @@ __global__ void __launch_bounds__(kCoopThreads, 1) attn_coop_kernel(const __grid
     for (uint32_t f = mw;; f += kCoopMergeWarps) {
       const int b = (int)(f % kCoopBufs);
       if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&mfull[b], (f / kCoopBufs) & 1u, a.status, abort))) return;
-      const CoopSeg sg = segs[f % kCoopSegs];
+      CoopSeg sg = segs[f % kCoopSegs];
       if (sg.u < 0) return;
+      sg.u = (int)BASISKV_DEBUG_INDEX(sg.u, a.batch * a.num_kv_heads, a.status);
+      sg.kvh = (int)BASISKV_DEBUG_INDEX(sg.kvh, a.num_kv_heads, a.status);
       MergeOut<G, RR> mo;
       merge_warp_states<G, RR, NW>(mrg + (size_t)b * NW * MW, mo);
       __syncwarp();
@@ -462,7 +466,7 @@ __global__ void __launch_bounds__(kCoopThreads, 1) attn_coop_kernel(const __grid
       return;
     }
     if (m.u != q_u) {
-      load_q_frags<G, D, K8>(a, m.u, qa);
+      load_q_frags<G, D, K8>(a, (int)BASISKV_DEBUG_INDEX(m.u, a.batch * a.num_kv_heads, a.status), qa);
       q_u = m.u;
     }
     if (m.valid > 0)

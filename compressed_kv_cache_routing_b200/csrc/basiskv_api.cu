@@ -1,6 +1,7 @@
 // Host side of the BasisKV decode-attention library: argument validation,
 // library-owned state, launch shapes and the C ABI declared in basiskv.h.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -25,6 +26,16 @@ using namespace basiskv;
 namespace {
 
 thread_local std::string g_last_error;
+
+// An NVTX range over the host side of a library call or grid launch, so a
+// timeline tool shows which call and which grid each launch belongs to
+// (header-only NVTX: without a tool attached a push and a pop cost a branch).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 int fail(int code, const char* fmt, ...) {
   char buf[512];
@@ -497,6 +508,7 @@ LaunchPlan plan(const basiskv_handle* h, int batch, int topk, bool force_route) 
 
 int launch_prep(basiskv_handle* h, const LaunchPlan& lp, int topk, int force, float* out, int32_t* sel_out,
                 float* fill_scores, int latent, cudaStream_t stream) {
+  NvtxRange range("basiskv prep grid");
   const basiskv_params& p = h->p;
   PrepArgs a;
   a.seq_lens = h->d_seq_lens;
@@ -582,6 +594,7 @@ cudaLaunchConfig_t launch_cfg(dim3 grid, int threads, size_t smem, cudaStream_t 
 // Routing after the prep grid: the persistent tensor-core kernel (PDL: it
 // waits for the prep grid before reading the plan), else the generic one.
 int launch_route(basiskv_handle* h, const LaunchPlan& lp, const RouteArgs& a, bool pdl, cudaStream_t stream) {
+  NvtxRange range("basiskv routing grid");
   const basiskv_params& p = h->p;
   cudaLaunchAttribute attr[1];
   if (h->route_fn) {
@@ -601,6 +614,7 @@ int launch_route(basiskv_handle* h, const LaunchPlan& lp, const RouteArgs& a, bo
 // Selection for the persistent routing kernel (PDL behind it).
 int launch_topk(basiskv_handle* h, const LaunchPlan& lp, int topk, const float* scores, int32_t* sel_out,
                 int force, bool pdl, bool poll, cudaStream_t stream) {
+  NvtxRange range("basiskv selection grid");
   const basiskv_params& p = h->p;
   TopkArgs a;
   a.scores = scores;
@@ -628,6 +642,7 @@ int launch_topk(basiskv_handle* h, const LaunchPlan& lp, int topk, const float* 
 
 int launch_attn(basiskv_handle* h, const LaunchPlan& lp, const void* q, int topk, float scale, int latent,
                 float* out, int32_t* sel_out, bool pdl, bool tagged_sel, cudaStream_t stream) {
+  NvtxRange range("basiskv attention grid");
   const basiskv_params& p = h->p;
   const size_t U = (size_t)p.max_batch * p.num_kv_heads;
   AttnArgs a;
@@ -849,6 +864,7 @@ int basiskv_append_page(basiskv_handle* h, int seq, int slot, int n_tokens, basi
 
 int basiskv_append_page_copy(basiskv_handle* h, int seq, int slot, int n_tokens, const void* z, const void* r,
                              const void* k, const float* k_scale, basiskv_stream_t stream) {
+  NvtxRange range("basiskv_append_page_copy");
   int rc = check_handle(h);
   if (rc) return rc;
   const basiskv_params& p = h->p;
@@ -947,6 +963,7 @@ int basiskv_load_page_table(basiskv_handle* h, int batch, const int32_t* page_ta
 // [batch][Hq][r]).
 static int decode_step(basiskv_handle* h, int batch, const void* q, int topk, float softmax_scale, float* out,
                        int32_t* sel_out, basiskv_stream_t stream, int latent) {
+  NvtxRange range(latent ? "basiskv_decode_attn_latent" : "basiskv_decode_attn");
   int rc = check_call(h, batch, q, topk);
   if (rc) return rc;
   if (!out) return fail(BASISKV_ERR_INVALID_ARG, "out is NULL");
@@ -1076,6 +1093,7 @@ extern "C" {
 
 int basiskv_encode_rows(basiskv_handle* h, int slot, int row0, int n_rows, const void* k, const void* v,
                         basiskv_stream_t stream) {
+  NvtxRange range("basiskv_encode_rows");
   int rc = check_handle(h);
   if (rc) return rc;
   const basiskv_params& p = h->p;
@@ -1096,6 +1114,7 @@ int basiskv_encode_rows(basiskv_handle* h, int slot, int row0, int n_rows, const
 
 int basiskv_encode_tokens(basiskv_handle* h, int n, const int32_t* slots, const int32_t* rows, const void* k,
                           const void* v, basiskv_stream_t stream) {
+  NvtxRange range("basiskv_encode_tokens");
   int rc = check_handle(h);
   if (rc) return rc;
   if (n < 0) return fail(BASISKV_ERR_INVALID_ARG, "n %d < 0", n);
@@ -1115,6 +1134,7 @@ int basiskv_encode_tokens(basiskv_handle* h, int n, const int32_t* slots, const 
 
 int basiskv_quantize_keys(basiskv_handle* h, const void* k, int64_t row0, int64_t n_rows,
                           basiskv_stream_t stream) {
+  NvtxRange range("basiskv_quantize_keys");
   int rc = check_handle(h);
   if (rc) return rc;
   const basiskv_params& p = h->p;
@@ -1181,6 +1201,7 @@ int basiskv_decode_attn_host(basiskv_handle* h, int batch, const void* q_host, i
 
 int basiskv_route(basiskv_handle* h, int batch, const void* q, int topk, float* scores_out, int32_t* sel_out,
                   basiskv_stream_t stream) {
+  NvtxRange range("basiskv_route");
   int rc = check_call(h, batch, q, topk);
   if (rc) return rc;
   if (batch == 0) return BASISKV_OK;

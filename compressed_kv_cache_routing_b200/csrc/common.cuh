@@ -14,6 +14,22 @@ constexpr uint32_t kStatusTimeout = 2u;
 constexpr uint32_t kStatusBadPage = 4u;
 constexpr uint32_t kStatusPartOverflow = 8u;  // a unit met more partials than it has slots
 constexpr uint32_t kStatusBadLength = 16u;    // a length needs more pages than a table row holds
+constexpr uint32_t kStatusDebugBounds = 32u;  // debug build: an index out of its range by construction
+
+// Debug build (BASISKV_DEBUG): indices that the kernels keep in range by
+// construction are checked where they are used; a failed check records
+// kStatusDebugBounds and the access goes to index 0.  In the normal build the
+// index passes through unchanged.
+#ifdef BASISKV_DEBUG
+__device__ __forceinline__ long long debug_index(long long i, long long bound, uint32_t* status) {
+  if (i >= 0 && i < bound) return i;
+  atomicOr(status, kStatusDebugBounds);
+  return 0;
+}
+#define BASISKV_DEBUG_INDEX(i, bound, status) debug_index((i), (bound), (status))
+#else
+#define BASISKV_DEBUG_INDEX(i, bound, status) (i)
+#endif
 
 // Largest batch whose work plan travels in the kernel parameters; larger
 // batches read the plan the prep grid writes to global memory.

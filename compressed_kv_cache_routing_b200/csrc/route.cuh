@@ -637,7 +637,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_c
           atomicOr(a.status, kStatusBadSlot);
           slot = 0;
         }
-        const size_t row0 = ((size_t)slot * a.num_kv_heads + nkvh[k]) * P;
+        const size_t row0 = BASISKV_DEBUG_INDEX(((long long)slot * a.num_kv_heads + nkvh[k]) * P,
+                                                (long long)a.num_slots * a.num_kv_heads * P, a.status);
         bulk_load(dst + k * page_bytes, zpool + row0 * RR, zbytes, bar, pol);
         if (RS > 0) bulk_load(dst + k * page_bytes + zbytes, rpool + row0 * RS, rbytes, bar, pol);
       }
@@ -747,11 +748,13 @@ __global__ void __launch_bounds__(kRouteThreads) route_mma_kernel(const __grid_c
         const __nv_bfloat16* zs = reinterpret_cast<const __nv_bfloat16*>(stage + k * page_bytes);
         const float best = route_page_score<G, RR, RS, P, FR>(zs, zs + P * RR, min(P, cc.L - cc.j * P), fr);
         if (lane == 0) {
+          const size_t e = BASISKV_DEBUG_INDEX((long long)cur_u * a.ld_pt + cc.j,
+                                               (long long)a.batch * a.num_kv_heads * a.ld_pt, a.status);
           if (a.tagged_scores)
-            st_relaxed_u64(a.scores64 + (size_t)cur_u * a.ld_pt + cc.j,
+            st_relaxed_u64(a.scores64 + e,
                            ((uint64_t)a.tag << 32) | __float_as_uint(best));
           else
-            a.scores[(size_t)cur_u * a.ld_pt + cc.j] = best;
+            a.scores[e] = best;
         }
         cc.advance(a);
       }

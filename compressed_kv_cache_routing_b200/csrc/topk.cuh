@@ -285,6 +285,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkArgs a) {
     for (int i = i0; i < i1; ++i) {
       const uint32_t key = keys[i] & tmask;
       if (kb >= n || key > thr || (key == thr && e < need)) {
+        pos = (int)BASISKV_DEBUG_INDEX(pos, a.ld_sel, a.status);
         sel[pos] = i;
         if (sel64) st_relaxed_u64(sel64 + pos, ((uint64_t)a.tag << 32) | (uint32_t)i);
         if (so) so[pos] = i;

@@ -80,10 +80,15 @@ enum {
     BASISKV_STATUS_BAD_PAGE = 4u,   /* a selected page outside [0, n_b)          */
     BASISKV_STATUS_PART_OVERFLOW = 8u, /* a unit met more split partials than its
                                           slots; that unit's output is invalid  */
-    BASISKV_STATUS_BAD_LENGTH = 16u /* a sequence length needing more pages than
+    BASISKV_STATUS_BAD_LENGTH = 16u, /* a sequence length needing more pages than
                                        a page-table row holds (device lengths of
                                        basiskv_decode_attn_noalloc only): the
                                        sequence is cut to the row              */
+    BASISKV_STATUS_DEBUG_BOUNDS = 32u /* debug build (BASISKV_DEBUG) only: an index
+                                       the kernels keep in range by construction
+                                       (ring stage, unit, KV head, pool row,
+                                       score or selection entry) was not; the
+                                       access went to index 0 instead          */
 };
 
 enum { BASISKV_DTYPE_BF16 = 0, BASISKV_DTYPE_F32 = 1 };
