@@ -227,6 +227,27 @@ def test_edge_lengths_and_mixed_routing():
     assert out_error(out, ref_out) <= OUT_TOL
 
 
+def test_shared_ring_with_many_short_units():
+    """Two long sequences take the shared-ring attention kernel (units of 80
+    stages); the other 46 sequences have from 0 to 7 pages, so most units
+    are unrouted and a few stages long, and a CTA's chunk holds dozens of
+    segments."""
+    batch = 48
+    rng = np.random.default_rng(11)
+    lens = rng.integers(0, 7 * 64, size=batch)
+    lens[:6] = [0, 1, 64, 65, 5000, 6000]
+    spec = W.shrink("llama3_8b_decode", batch=batch, len_lo=6000, len_hi=6000, topk=40)
+    w = _with_lengths(spec, lens)
+    kv = bk.BasisKV.for_workload(w)
+    ref_out, ref_sel, _, _ = oracle.decode(to_problem(w))
+    out, sel = gpu_decode(w, kv=kv)
+    assert bk.basiskv_last_launch(kv.handle)["attn_shared_ring"] == 1
+    kv.close()
+    assert np.array_equal(sel, ref_sel)
+    assert (sel[0] == -1).all() and (out[0] == 0).all()
+    assert out_error(out, ref_out) <= OUT_TOL
+
+
 def test_topk_one_and_max():
     spec = W.shrink("high_concurrency", batch=3, len_lo=900, len_hi=1400, topk=1)
     w = W.generate(spec, device="cuda")
